@@ -1,0 +1,337 @@
+"""CPU oracle for the STARFlow-V affine autoregressive flow (AF) block.
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import or call
+this module.  The product path (``video_generation_b200``) never does, and the
+two share no code.
+
+Plain, slow, float64 numpy.  Library primitives used as steps: matmul, exp,
+sqrt and ``scipy.special.erf``.  Every function follows the pages step by step
+with no blocking or fusion beyond what they state.  Sources, by page and
+section:
+
+  [N]  "STARFlow-V: End-to-End Video Generative Modeling with Autoregressive
+       Normalizing Flows", CVPR 2026 paper notes (papernotes.org):
+       - "Key design 1: global-local architecture" -- the affine AF equation
+         z = (x - mu(x*m)) / sigma(x*m), sigma > 0, with m the self-exclusive
+         causal mask; T >= 3 blocks of alternating direction; the
+         deep/shallow split f = f_D o f_S; f_S inside one frame (alternating
+         L->R / R->L), f_D causal across frames.
+       - "Key design 3: video-aware block-wise Jacobi iteration" -- the
+         fixed-point system x = mu(x*m) + sigma(x*m) * z, the update
+         x^(k+1) = mu(x^(k)*m) + sigma(x^(k)*m) * z, the stopping rule
+         ||x^(k+1) - x^(k)||^2 / ||x^(k+1)||^2 < tau (tau = 1e-3), blocks of
+         size B run in sequence with parallel updates inside a block,
+         finished blocks feeding a KV cache, and the warm start
+         x^(0)_{n+1} = x^(k)_n from the previous frame's converged state.
+       - "Loss / training strategy" -- L_NF = E[log p0(f(x)) + log|det J|],
+         which fixes the sign of the log-determinant.
+  The pages never spell out the Transformer inside the AF block beyond
+  "causal Transformer".  Readings taken where they are silent (each stated
+  where used):
+    R1 mask m: a one-token input shift (token 0 sees a zero vector) followed
+       by inclusive causal attention, so mu_i and sigma_i depend on x_{<i}.
+    R2 sigma = exp(s), no clamp.
+    R3 logdet = -sum_{i,c} s_{i,c} per sample (a sum, not a mean).
+    R4 the residual norm runs over one block's B*C entries of one sample;
+       strict '<'; 0/0 counts as converged, num>0 over 0 does not.
+    R5 x^(0) = z for a block with no warm start.
+    R6 the output of a block is the iterate that passed the test; ``iters``
+       counts the updates computed.
+    R7 the KV cache of a finished block is computed from its final x.
+    R8 each sample of a batch converges on its own.
+    R9 pre-LN Transformer: LayerNorm eps 1e-5, multi-head attention with
+       scale 1/sqrt(head_dim), exact-erf GELU MLP of width mlp_ratio*d,
+       final LayerNorm, linear head [mu | s] (mu = first C outputs).
+    R10 positions: pos[p] = P_space[p mod frame_len] + P_time[p div frame_len].
+    R11 direction R->L reverses the token order of each sample's sequence
+       before the block and restores it after.
+    R12 bf16 models: the weights are rounded to bf16 (round to nearest even)
+       once; the oracle then computes in float64 with those values.
+"""
+from __future__ import annotations
+
+import math
+from typing import List, Sequence, Tuple
+
+import numpy as np
+from scipy.special import erf
+
+L2R, R2L = 0, 1
+
+
+# ----------------------------------------------------------------------------
+# weights
+
+def bf16_round(a: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest bfloat16 (ties to even); float32 out.
+
+    bfloat16 keeps the top 16 bits of an IEEE float32.  Rounding to nearest
+    even adds 0x7FFF plus the lowest kept bit before truncating.  (No NaN/Inf
+    in the synthetic weights.)
+    """
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return u.astype(np.uint32).view(np.float32)
+
+
+class Block:
+    """Weights of one AF block, indexed like ``synthetic.tensor_specs``.
+
+    Arrays stay float32 in memory (bf16 values are exact in float32) and are
+    widened to float64 at each use.
+    """
+
+    def __init__(self, shape, tensors: Sequence[np.ndarray]):
+        self.C, self.d, self.heads = shape.C, shape.d, shape.heads
+        self.layers, self.frame_len = shape.layers, shape.frame_len
+        self.max_frames = shape.max_frames
+        t = [np.asarray(a, np.float32) for a in tensors]
+        if shape.dtype == "bf16":                     # R12
+            t = [bf16_round(a) for a in t]
+        self.w_in, self.b_in, self.pos_space, self.pos_time = t[0:4]
+        self.L_ = []
+        for l in range(shape.layers):
+            g = t[4 + 12 * l: 4 + 12 * (l + 1)]
+            self.L_.append(dict(ln1_g=g[0], ln1_b=g[1], w_qkv=g[2], b_qkv=g[3],
+                                w_o=g[4], b_o=g[5], ln2_g=g[6], ln2_b=g[7],
+                                w_1=g[8], b_1=g[9], w_2=g[10], b_2=g[11]))
+        self.lnf_g, self.lnf_b, self.w_head, self.b_head = t[4 + 12 * shape.layers:]
+
+
+def _f(a):
+    return np.asarray(a, dtype=np.float64)
+
+
+# ----------------------------------------------------------------------------
+# the causal Transformer inside one AF block (R9)
+
+def layer_norm(h, g, b, eps=1e-5):
+    mu = h.mean(axis=-1, keepdims=True)
+    var = ((h - mu) ** 2).mean(axis=-1, keepdims=True)
+    return (h - mu) / np.sqrt(var + eps) * _f(g) + _f(b)
+
+
+def gelu(u):
+    return 0.5 * u * (1.0 + erf(u / math.sqrt(2.0)))
+
+
+def linear(a, w, b):
+    return a @ _f(w).T + _f(b)
+
+
+def positions(blk: Block, p: np.ndarray) -> np.ndarray:
+    """Learned absolute position vectors of sequence positions p (R10)."""
+    return _f(blk.pos_space)[p % blk.frame_len] + _f(blk.pos_time)[p // blk.frame_len]
+
+
+def causal_attention(q, K, V, p0, heads):
+    """softmax(q K^T / sqrt(hd) restricted to keys j <= query position) V.
+
+    q holds the queries of positions p0 .. p0+n-1; K, V hold keys and values
+    of positions 0 .. p0+n-1 (the cache of positions < p0, then the rows
+    themselves).  Plain softmax: subtract the row max, exponentiate, divide.
+    """
+    n, d = q.shape
+    hd = d // heads
+    allowed = np.arange(K.shape[0])[None, :] <= (p0 + np.arange(n))[:, None]
+    out = np.empty_like(q)
+    for h in range(heads):
+        sl = slice(h * hd, (h + 1) * hd)
+        S = (q[:, sl] @ K[:, sl].T) / math.sqrt(hd)
+        S = np.where(allowed, S, -np.inf)
+        S = S - S.max(axis=1, keepdims=True)
+        E = np.exp(S)
+        out[:, sl] = (E / E.sum(axis=1, keepdims=True)) @ V[:, sl]
+    return out
+
+
+def transformer_rows(blk: Block, x_in: np.ndarray, p0: int, cache=None):
+    """mu, s for the rows at positions p0 .. p0+n-1 of one sample.
+
+    ``x_in`` [n, C] are the already-masked inputs of those positions (R1: the
+    input at position p is x_{p-1}, zero at p = 0).  ``cache`` is a list, per
+    layer, of (K, V) of positions 0 .. p0-1 (None when p0 = 0).  Returns
+    (mu [n, C], s [n, C], kv) where kv holds the rows' own (K, V) per layer.
+    """
+    n = x_in.shape[0]
+    d, C = blk.d, blk.C
+    h = linear(_f(x_in), blk.w_in, blk.b_in) + positions(blk, p0 + np.arange(n))
+    kv = []
+    for l, P in enumerate(blk.L_):
+        a = layer_norm(h, P["ln1_g"], P["ln1_b"])
+        qkv = linear(a, P["w_qkv"], P["b_qkv"])
+        q, k, v = qkv[:, :d], qkv[:, d:2 * d], qkv[:, 2 * d:]
+        kv.append((k, v))
+        if cache is not None and p0 > 0:
+            K = np.concatenate([cache[l][0], k])
+            V = np.concatenate([cache[l][1], v])
+        else:
+            K, V = k, v
+        h = h + linear(causal_attention(q, K, V, p0, blk.heads), P["w_o"], P["b_o"])
+        a = layer_norm(h, P["ln2_g"], P["ln2_b"])
+        h = h + linear(gelu(linear(a, P["w_1"], P["b_1"])), P["w_2"], P["b_2"])
+    out = linear(layer_norm(h, blk.lnf_g, blk.lnf_b), blk.w_head, blk.b_head)
+    return out[:, :C], out[:, C:], kv
+
+
+def masked_inputs(xw: np.ndarray, p0: int, p1: int) -> np.ndarray:
+    """Inputs of positions p0..p1-1 under the self-exclusive mask (R1)."""
+    C = xw.shape[1]
+    prev = xw[p0 - 1:p1 - 1] if p0 > 0 else np.concatenate([np.zeros((1, C)), xw[:p1 - 1]])
+    return _f(prev)
+
+
+def _work(a, direction):            # R11
+    return a[::-1] if direction == R2L else a
+
+
+# ----------------------------------------------------------------------------
+# forward: z and logdet ([N] key design 1, affine AF equation; loss section)
+
+def af_forward_one(blk: Block, x: np.ndarray, direction: int):
+    xw = _f(_work(x, direction))
+    L = xw.shape[0]
+    mu, s, _ = transformer_rows(blk, masked_inputs(xw, 0, L), 0)
+    zw = (xw - mu) * np.exp(-s)               # sigma = exp(s)   (R2)
+    logdet = -s.sum()                         # log|det dz/dx| = -sum log sigma (R3)
+    return _work(zw, direction).copy(), float(logdet)
+
+
+def af_forward(blk: Block, x: np.ndarray, direction: int):
+    """x [batch, L, C] -> z [batch, L, C], logdet [batch] (float64)."""
+    out = [af_forward_one(blk, xb, direction) for xb in x]
+    return np.stack([o[0] for o in out]), np.array([o[1] for o in out])
+
+
+# ----------------------------------------------------------------------------
+# sequential inverse (textbook autoregressive inverse, token by token)
+
+def af_inverse_seq_one(blk: Block, z: np.ndarray, direction: int):
+    zw = _f(_work(z, direction))
+    L, C = zw.shape
+    xw = np.zeros_like(zw)
+    cache = [(np.zeros((0, blk.d)), np.zeros((0, blk.d))) for _ in range(blk.layers)]
+    for i in range(L):
+        x_in = xw[i - 1:i] if i > 0 else np.zeros((1, C))
+        mu, s, kv = transformer_rows(blk, x_in, i, cache)
+        xw[i] = mu[0] + np.exp(s[0]) * zw[i]
+        cache = [(np.concatenate([cache[l][0], kv[l][0]]),
+                  np.concatenate([cache[l][1], kv[l][1]])) for l in range(blk.layers)]
+    return _work(xw, direction).copy()
+
+
+def af_inverse_seq(blk: Block, z: np.ndarray, direction: int):
+    return np.stack([af_inverse_seq_one(blk, zb, direction) for zb in z])
+
+
+# ----------------------------------------------------------------------------
+# block-wise Jacobi inverse ([N] key design 3)
+
+def jacobi_residual(x_new, x_old):
+    """||x_new - x_old||^2 / ||x_new||^2 and the converged test (R4)."""
+    num = float(((x_new - x_old) ** 2).sum())
+    den = float((x_new ** 2).sum())
+    return num, den
+
+
+def converged(num, den, tau):
+    if den == 0.0:
+        return num == 0.0
+    return num / den < tau
+
+
+def af_inverse_jacobi_one(blk: Block, z: np.ndarray, direction: int, B: int, tau: float,
+                          max_iter: int, warm_start: bool, x0=None, trace=None):
+    """One sample.  Returns (x, iters [L/B], converged [L/B]).
+
+    ``x0`` optionally overrides the first block's starting guess (used by the
+    any-start prefix-exactness pin); ``trace`` collects every iterate of every
+    block when given a list.
+    """
+    zw = _f(_work(z, direction))
+    L, C = zw.shape
+    assert L % B == 0
+    nb = L // B
+    xw = np.zeros_like(zw)
+    cache = None
+    iters = np.zeros(nb, np.int64)
+    conv = np.zeros(nb, bool)
+    for b in range(nb):
+        P = b * B
+        zb = zw[P:P + B]
+        if b == 0 and x0 is not None:
+            xk = _f(_work(x0, direction))[P:P + B].copy()
+        elif warm_start and b > 0:
+            xk = xw[P - B:P].copy()                       # warm start from block b-1
+        else:
+            xk = zb.copy()                                # R5
+        for k in range(max_iter):
+            xw[P:P + B] = xk
+            mu, s, _ = transformer_rows(blk, masked_inputs(xw, P, P + B), P, cache)
+            x_new = mu + np.exp(s) * zb
+            num, den = jacobi_residual(x_new, xk)
+            xk = x_new
+            iters[b] = k + 1
+            if trace is not None:
+                trace.append((b, k + 1, xk.copy()))
+            if converged(num, den, tau):
+                conv[b] = True
+                break
+        xw[P:P + B] = xk                                  # R6
+        if b + 1 < nb:                                    # commit K/V of the final x (R7)
+            _, _, kv = transformer_rows(blk, masked_inputs(xw, P, P + B), P, cache)
+            if cache is None:
+                cache = [(k_, v_) for (k_, v_) in kv]
+            else:
+                cache = [(np.concatenate([cache[l][0], kv[l][0]]),
+                          np.concatenate([cache[l][1], kv[l][1]])) for l in range(blk.layers)]
+    return _work(xw, direction).copy(), iters, conv
+
+
+def af_inverse_jacobi(blk: Block, z: np.ndarray, direction: int, B: int, tau: float,
+                      max_iter: int, warm_start: bool):
+    """z [batch, L, C] -> x [batch, L, C], iters [batch, L/B], converged [batch, L/B]."""
+    out = [af_inverse_jacobi_one(blk, zb, direction, B, tau, max_iter, warm_start) for zb in z]
+    return (np.stack([o[0] for o in out]), np.stack([o[1] for o in out]),
+            np.stack([o[2] for o in out]))
+
+
+# ----------------------------------------------------------------------------
+# stacks of alternating-direction blocks ([N] key design 1: T >= 3 blocks of
+# alternating direction; inversion undoes them last-to-first)
+
+def stack_forward(blocks: List[Block], dirs: Sequence[int], x: np.ndarray):
+    z = _f(x)
+    total = np.zeros(x.shape[0])
+    for blk, dr in zip(blocks, dirs):
+        z, ld = af_forward(blk, z, dr)
+        total = total + ld
+    return z, total
+
+
+def stack_inverse(blocks: List[Block], dirs: Sequence[int], z: np.ndarray, B: int,
+                  tau: float, max_iter: int, warm_start: bool):
+    x = _f(z)
+    all_iters = [None] * len(blocks)
+    for t in reversed(range(len(blocks))):
+        x, it, _ = af_inverse_jacobi(blocks[t], x, dirs[t], B, tau, max_iter, warm_start)
+        all_iters[t] = it
+    return x, np.stack(all_iters)
+
+
+# ----------------------------------------------------------------------------
+# brute-force Jacobian (pins the log-determinant on tiny inputs)
+
+def jacobian_bruteforce(blk: Block, x: np.ndarray, direction: int, h: float = 1e-6):
+    """Central-difference d z / d x of one sample, [L*C, L*C]."""
+    x = _f(x)
+    n = x.size
+    J = np.empty((n, n))
+    for j in range(n):
+        e = np.zeros(n)
+        e[j] = h
+        zp, _ = af_forward_one(blk, (x.ravel() + e).reshape(x.shape), direction)
+        zm, _ = af_forward_one(blk, (x.ravel() - e).reshape(x.shape), direction)
+        J[:, j] = (zp.ravel() - zm.ravel()) / (2 * h)
+    return J
