@@ -1,0 +1,707 @@
+// af_api.cu -- the C ABI of libaf (declared in include/af.h): model packing,
+// workspace layout, the pass of one AF block, the forward and block-Jacobi
+// graphs, and the stacks of alternating-direction blocks.
+//
+// The AF block and its inverse follow "STARFlow-V: End-to-End Video Generative
+// Modeling with Autoregressive Normalizing Flows" (CVPR 2026 paper notes):
+// key design 1 (the affine AF equation, alternating-direction stacks) and key
+// design 3 (block-wise Jacobi with KV cache, warm start and the tau test).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <map>
+#include <string>
+#include <vector>
+
+#include "../../include/af.h"
+#include "af_kernels.h"
+
+using namespace af;
+
+namespace {
+
+thread_local char g_errbuf[512] = "";
+
+void set_err(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_errbuf, sizeof g_errbuf, fmt, ap);
+  va_end(ap);
+}
+
+#define CK(call)                                                                     \
+  do {                                                                               \
+    cudaError_t e_ = (call);                                                         \
+    if (e_ != cudaSuccess) {                                                         \
+      set_err("%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_), __FILE__, __LINE__); \
+      return AF_ERR_CUDA;                                                            \
+    }                                                                                \
+  } while (0)
+
+size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
+
+uint16_t f2bf(float f) {     // float -> bfloat16 bits, round to nearest even
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+struct LayerW {
+  void *w_qkv, *w_o, *w_1, *w_2;   // bf16 or fp32 [out, in]
+  float *ln1_g, *ln1_b, *b_qkv, *b_o, *ln2_g, *ln2_b, *b_1, *b_2;
+};
+
+}  // namespace
+
+struct af_model {
+  af_config cfg;
+  int fd, hd;
+  bool bf;
+  void* w_in;
+  float *b_in, *pos_space, *pos_time;
+  std::vector<LayerW> layers;
+  float *lnf_g, *lnf_b;
+  void* w_head;       // rows interleaved: 2c -> mu_c, 2c+1 -> s_c
+  float* b_head;      // interleaved the same way
+  int* d_err;
+  int num_sms;
+  std::vector<void*> allocs;
+  // graph cache (keyed by every pointer and scalar baked into the graph)
+  std::map<std::string, cudaGraphExec_t> graphs;
+  std::vector<std::string> graph_order;
+  cudaStream_t cap, cap2;   // private streams used for capture only
+};
+
+namespace {
+
+// ------------------------------------------------------------------ workspace
+
+struct Bufs {
+  Ctl* ctl;
+  int* active;
+  float* part;
+  float* h;
+  void* xin;
+  void* a;
+  void* q;
+  void* u;
+  void* kv;
+  float* tmp;
+  size_t total;
+};
+
+int rows_per_sample(int L, int B) { return B >= L ? L : 2 * B; }
+
+Bufs carve(const af_model* m, void* ws, int batch, int L, int B) {
+  const af_config& c = m->cfg;
+  const size_t es = m->bf ? 2 : 4;
+  const size_t mmax = (size_t)batch * rows_per_sample(L, B);
+  const int G = (2 * c.C) / 16;
+  Bufs b{};
+  size_t off = 0;
+  char* base = static_cast<char*>(ws);
+  auto take = [&](size_t bytes) {
+    void* p = base ? base + off : nullptr;
+    off += align256(bytes);
+    return p;
+  };
+  b.ctl = (Ctl*)take(sizeof(Ctl));
+  b.active = (int*)take(sizeof(int) * batch);
+  b.part = (float*)take(sizeof(float) * mmax * G * 2);
+  b.h = (float*)take(sizeof(float) * mmax * c.d);
+  b.xin = take(es * mmax * c.C);
+  b.a = take(es * mmax * c.d);
+  b.q = take(es * mmax * c.d);
+  b.u = take(es * mmax * m->fd);
+  b.kv = take(es * (size_t)c.layers * 2 * batch * L * c.d);
+  b.tmp = (float*)take(sizeof(float) * (size_t)batch * L * c.C);
+  b.total = off;
+  return b;
+}
+
+// ------------------------------------------------------------------ one pass
+
+struct HeadIO {
+  int mode;             // 0 forward, 1 Jacobi update
+  const float* xin_f;   // forward: x   inverse: z
+  float* xout_f;        // forward: z   inverse: x
+};
+
+// One pass of the AF block over the rows described by ctl (see af_common.cuh):
+// shifted gather, input projection + positions, `layers` pre-LN Transformer
+// blocks writing K/V into the cache, final LayerNorm and the fused head.
+af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int dir, int m_max, int r_max,
+                       const float* xsrc, const HeadIO& hio, cudaStream_t st) {
+  const af_config& c = m->cfg;
+  const int d = c.d, C = c.C, fd = m->fd;
+  const int G = (2 * C) / 16;
+  EpiArgs e{};
+  e.ctl = b.ctl;
+  e.h = b.h;
+  e.d = d;
+  e.Lc = L;
+  e.pos_space = m->pos_space;
+  e.pos_time = m->pos_time;
+  e.frame_len = c.frame_len;
+  const size_t es = m->bf ? 2 : 4;
+  const size_t kv_layer = (size_t)batch * L * d * es;
+
+  EpiArgs eh = e;
+  eh.bias = m->b_head;
+  eh.head_mode = hio.mode;
+  eh.L = L;
+  eh.C = C;
+  eh.dir = dir;
+  eh.xin_f = hio.xin_f;
+  eh.xout_f = hio.xout_f;
+  eh.active = b.active;
+  eh.part = b.part;
+
+  if (!m->bf) {
+    float* xin = (float*)b.xin;
+    float* a = (float*)b.a;
+    float* q = (float*)b.q;
+    float* u = (float*)b.u;
+    launch_gather<float>(b.ctl, xsrc, L, C, dir, xin, m_max, st);
+    e.bias = m->b_in;
+    launch_gemm_simt(EPI_INPROJ, xin, (const float*)m->w_in, d, C, m_max, e, st);
+    for (int l = 0; l < c.layers; ++l) {
+      const LayerW& w = m->layers[l];
+      char* kvl = (char*)b.kv + 2 * l * kv_layer;
+      launch_layernorm<float>(b.ctl, b.h, w.ln1_g, w.ln1_b, a, d, m_max, st);
+      EpiArgs eq = e;
+      eq.bias = w.b_qkv;
+      eq.out = q;
+      eq.kc = kvl;
+      eq.vc = kvl + kv_layer;
+      launch_gemm_simt(EPI_QKV, a, (const float*)w.w_qkv, 3 * d, d, m_max, eq, st);
+      launch_attn_simt(b.ctl, q, (const float*)kvl, (const float*)(kvl + kv_layer), a, batch, L, d, c.heads, m_max, st);
+      EpiArgs eo = e;
+      eo.bias = w.b_o;
+      launch_gemm_simt(EPI_RESID, a, (const float*)w.w_o, d, d, m_max, eo, st);
+      launch_layernorm<float>(b.ctl, b.h, w.ln2_g, w.ln2_b, a, d, m_max, st);
+      EpiArgs eu = e;
+      eu.bias = w.b_1;
+      eu.out = u;
+      eu.ldo = fd;
+      launch_gemm_simt(EPI_GELU, a, (const float*)w.w_1, fd, d, m_max, eu, st);
+      EpiArgs ed = e;
+      ed.bias = w.b_2;
+      launch_gemm_simt(EPI_RESID, u, (const float*)w.w_2, d, fd, m_max, ed, st);
+    }
+    launch_layernorm<float>(b.ctl, b.h, m->lnf_g, m->lnf_b, a, d, m_max, st);
+    launch_head_simt(a, (const float*)m->w_head, 2 * C, d, m_max, eh, st);
+  } else {
+    bf16* xin = (bf16*)b.xin;
+    bf16* a = (bf16*)b.a;
+    bf16* q = (bf16*)b.q;
+    bf16* u = (bf16*)b.u;
+    const int ns = m->num_sms;
+    CUtensorMap tA_x, tA_a, tA_u, tB;
+    bool ok = make_tmap_bf16(&tA_x, xin, m_max, C, 128) && make_tmap_bf16(&tA_a, a, m_max, d, 128) &&
+              make_tmap_bf16(&tA_u, u, m_max, fd, 128);
+    if (!ok) { set_err("cuTensorMapEncodeTiled failed for an activation"); return AF_ERR_CUDA; }
+    auto gemm = [&](int epi, const CUtensorMap& tA, const void* W, int N, int K, const EpiArgs& ea) -> bool {
+      const int bn = gemm_tc_pick_bn(N, m_max, ns);
+      if (!bn || !make_tmap_bf16(&tB, W, N, K, bn)) return false;
+      launch_gemm_tc(epi, tA, tB, bn, N, K, m_max, ea, m->d_err, ns, st);
+      return true;
+    };
+    launch_gather<bf16>(b.ctl, xsrc, L, C, dir, xin, m_max, st);
+    e.bias = m->b_in;
+    if (!gemm(EPI_INPROJ, tA_x, m->w_in, d, C, e)) { set_err("GEMM plan failed (in-proj)"); return AF_ERR_CUDA; }
+    for (int l = 0; l < c.layers; ++l) {
+      const LayerW& w = m->layers[l];
+      char* kvl = (char*)b.kv + 2 * l * kv_layer;
+      launch_layernorm<bf16>(b.ctl, b.h, w.ln1_g, w.ln1_b, a, d, m_max, st);
+      EpiArgs eq = e;
+      eq.bias = w.b_qkv;
+      eq.out = q;
+      eq.kc = kvl;
+      eq.vc = kvl + kv_layer;
+      if (!gemm(EPI_QKV, tA_a, w.w_qkv, 3 * d, d, eq)) { set_err("GEMM plan failed (qkv)"); return AF_ERR_CUDA; }
+      launch_attn_tc(b.ctl, q, (const bf16*)kvl, (const bf16*)(kvl + kv_layer), a, batch, L, d, c.heads, r_max, st);
+      EpiArgs eo = e;
+      eo.bias = w.b_o;
+      if (!gemm(EPI_RESID, tA_a, w.w_o, d, d, eo)) { set_err("GEMM plan failed (out)"); return AF_ERR_CUDA; }
+      launch_layernorm<bf16>(b.ctl, b.h, w.ln2_g, w.ln2_b, a, d, m_max, st);
+      EpiArgs eu = e;
+      eu.bias = w.b_1;
+      eu.out = u;
+      eu.ldo = fd;
+      if (!gemm(EPI_GELU, tA_a, w.w_1, fd, d, eu)) { set_err("GEMM plan failed (mlp up)"); return AF_ERR_CUDA; }
+      EpiArgs ed = e;
+      ed.bias = w.b_2;
+      if (!gemm(EPI_RESID, tA_u, w.w_2, d, fd, ed)) { set_err("GEMM plan failed (mlp down)"); return AF_ERR_CUDA; }
+    }
+    launch_layernorm<bf16>(b.ctl, b.h, m->lnf_g, m->lnf_b, a, d, m_max, st);
+    if (!gemm(EPI_HEAD, tA_a, m->w_head, 2 * C, d, eh)) { set_err("GEMM plan failed (head)"); return AF_ERR_CUDA; }
+  }
+  (void)G;
+  CK(cudaGetLastError());
+  return AF_OK;
+}
+
+// ------------------------------------------------------------------ graphs
+
+af_status add_while(cudaStream_t cs, cudaGraphConditionalHandle* h, unsigned dflt, unsigned flags,
+                    cudaGraph_t* body) {
+  cudaStreamCaptureStatus stat;
+  cudaGraph_t g;
+  const cudaGraphNode_t* deps = nullptr;
+  size_t nd = 0;
+  CK(cudaStreamGetCaptureInfo(cs, &stat, nullptr, &g, &deps, &nd));
+  if (stat != cudaStreamCaptureStatusActive) { set_err("stream not capturing"); return AF_ERR_CUDA; }
+  CK(cudaGraphConditionalHandleCreate(h, g, dflt, flags));
+  alignas(cudaGraphNodeParams) unsigned char pbuf[sizeof(cudaGraphNodeParams)] = {};
+  cudaGraphNodeParams& p = *reinterpret_cast<cudaGraphNodeParams*>(pbuf);
+  p.type = cudaGraphNodeTypeConditional;
+  p.conditional.handle = *h;
+  p.conditional.type = cudaGraphCondTypeWhile;
+  p.conditional.size = 1;
+  cudaGraphNode_t node;
+  CK(cudaGraphAddNode(&node, g, deps, nd, &p));
+  *body = p.conditional.phGraph_out[0];
+  CK(cudaStreamUpdateCaptureDependencies(cs, &node, 1, cudaStreamSetCaptureDependencies));
+  return AF_OK;
+}
+
+struct JacobiJob {
+  const af_model* m;
+  const float* z;
+  float* x;
+  int dir;
+  int32_t* iters;
+  bool reset_nonconv;
+};
+
+// Capture the block-Jacobi inverse of one AF block into the stream `cs`,
+// which is capturing: [call init] WHILE(blocks) { [block init]
+// WHILE(updates) { pass; [jacobi step] } [block advance] }.
+af_status capture_jacobi(const JacobiJob& jb, const Bufs& b, int batch, int L, int B, float tau, int max_iter,
+                         int warm, cudaStream_t cs) {
+  const af_model* m = jb.m;
+  const int nb = L / B;
+  const int G = (2 * m->cfg.C) / 16;
+  const int r_max = rows_per_sample(L, B);
+  const int m_max = batch * r_max;
+  launch_call_init(b.ctl, jb.reset_nonconv ? 1 : 0, cs);
+  cudaGraphConditionalHandle h_outer, h_inner;
+  cudaGraph_t body_outer, body_inner;
+  af_status s = add_while(cs, &h_outer, 1, cudaGraphCondAssignDefault, &body_outer);
+  if (s) return s;
+  // The outer body and the inner body are captured with a second private stream.
+  cudaStream_t cs2 = m->cap2;
+  af_status rc = AF_OK;
+  do {
+    if (cudaStreamBeginCaptureToGraph(cs2, body_outer, nullptr, nullptr, 0, cudaStreamCaptureModeRelaxed) != cudaSuccess) {
+      set_err("capture of the block loop failed"); rc = AF_ERR_CUDA; break;
+    }
+    // the inner handle lives in the outer body; block init sets it to 1
+    cudaStreamCaptureStatus stat;
+    cudaGraph_t gcap;
+    if (cudaStreamGetCaptureInfo(cs2, &stat, nullptr, &gcap, nullptr, nullptr) != cudaSuccess ||
+        cudaGraphConditionalHandleCreate(&h_inner, gcap, 0, 0) != cudaSuccess) {
+      set_err("conditional handle creation failed"); rc = AF_ERR_CUDA;
+    }
+    if (!rc) {
+      launch_block_init(b.ctl, b.active, jb.z, jb.x, batch, L, m->cfg.C, B, jb.dir, warm, h_inner, cs2);
+      cudaStreamCaptureStatus st2;
+      cudaGraph_t g2;
+      const cudaGraphNode_t* deps = nullptr;
+      size_t nd = 0;
+      alignas(cudaGraphNodeParams) unsigned char pbuf[sizeof(cudaGraphNodeParams)] = {};
+      cudaGraphNodeParams& p = *reinterpret_cast<cudaGraphNodeParams*>(pbuf);
+      cudaGraphNode_t node;
+      if (cudaStreamGetCaptureInfo(cs2, &st2, nullptr, &g2, &deps, &nd) != cudaSuccess) { rc = AF_ERR_CUDA; }
+      else {
+        p.type = cudaGraphNodeTypeConditional;
+        p.conditional.handle = h_inner;
+        p.conditional.type = cudaGraphCondTypeWhile;
+        p.conditional.size = 1;
+        if (cudaGraphAddNode(&node, g2, deps, nd, &p) != cudaSuccess ||
+            cudaStreamUpdateCaptureDependencies(cs2, &node, 1, cudaStreamSetCaptureDependencies) != cudaSuccess) {
+          set_err("adding the update loop failed"); rc = AF_ERR_CUDA;
+        } else {
+          body_inner = p.conditional.phGraph_out[0];
+        }
+      }
+      if (!rc) launch_block_advance(b.ctl, nb, h_outer, cs2);
+    }
+    cudaGraph_t dummy;
+    if (cudaStreamEndCapture(cs2, &dummy) != cudaSuccess && !rc) { set_err("end of block-loop capture failed"); rc = AF_ERR_CUDA; }
+    if (rc) break;
+    // the update body
+    if (cudaStreamBeginCaptureToGraph(cs2, body_inner, nullptr, nullptr, 0, cudaStreamCaptureModeRelaxed) != cudaSuccess) {
+      set_err("capture of the update loop failed"); rc = AF_ERR_CUDA; break;
+    }
+    HeadIO hio{1, jb.z, jb.x};
+    rc = enqueue_pass(m, b, batch, L, jb.dir, m_max, r_max, jb.x, hio, cs2);
+    if (!rc) launch_jacobi_step(b.ctl, b.active, b.part, batch, B, G, tau, max_iter, jb.iters, nb, h_inner, cs2);
+    if (cudaStreamEndCapture(cs2, &dummy) != cudaSuccess && !rc) { set_err("end of update capture failed"); rc = AF_ERR_CUDA; }
+  } while (0);
+  return rc;
+}
+
+af_status graph_run(const af_model* mc, const std::string& key, cudaStream_t st,
+                    af_status (*build)(void*, cudaStream_t), void* ctx) {
+  af_model* m = const_cast<af_model*>(mc);
+  auto it = m->graphs.find(key);
+  if (it == m->graphs.end()) {
+    cudaGraph_t g;
+    CK(cudaGraphCreate(&g, 0));
+    CK(cudaStreamBeginCaptureToGraph(m->cap, g, nullptr, nullptr, 0, cudaStreamCaptureModeRelaxed));
+    af_status s = build(ctx, m->cap);
+    cudaGraph_t g2;
+    cudaError_t ee = cudaStreamEndCapture(m->cap, &g2);
+    if (s) { cudaGraphDestroy(g); return s; }
+    if (ee != cudaSuccess) { cudaGraphDestroy(g); set_err("graph capture failed: %s", cudaGetErrorString(ee)); return AF_ERR_CUDA; }
+    cudaGraphExec_t ex;
+    cudaError_t ie = cudaGraphInstantiate(&ex, g, 0);
+    cudaGraphDestroy(g);
+    if (ie != cudaSuccess) { set_err("graph instantiation failed: %s", cudaGetErrorString(ie)); return AF_ERR_CUDA; }
+    if (m->graph_order.size() >= 16) {
+      cudaGraphExecDestroy(m->graphs[m->graph_order.front()]);
+      m->graphs.erase(m->graph_order.front());
+      m->graph_order.erase(m->graph_order.begin());
+    }
+    it = m->graphs.emplace(key, ex).first;
+    m->graph_order.push_back(key);
+  }
+  CK(cudaGraphLaunch(it->second, st));
+  return AF_OK;
+}
+
+std::string keyf(const char* tag, std::initializer_list<long long> v) {
+  std::string s(tag);
+  char buf[32];
+  for (long long x : v) { snprintf(buf, sizeof buf, ":%llx", x); s += buf; }
+  return s;
+}
+
+// ------------------------------------------------------------------ argument checks
+
+af_status check_model(const af_model* m) {
+  if (!m) { set_err("null model"); return AF_ERR_ARG; }
+  return AF_OK;
+}
+
+af_status check_ws(const af_model* m, void* ws, size_t ws_bytes, int batch, int L, int B) {
+  const size_t need = af_workspace_bytes(m, batch, L, B);
+  if (!need) { set_err("bad batch/L/B for this model"); return AF_ERR_ARG; }
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < need) {
+    set_err("workspace: need %zu bytes, 256-aligned; got %zu at %p", need, ws_bytes, ws);
+    return AF_ERR_WORKSPACE;
+  }
+  return AF_OK;
+}
+
+bool same_cfg(const af_config& a, const af_config& b) {
+  return a.C == b.C && a.d == b.d && a.heads == b.heads && a.layers == b.layers && a.mlp_ratio == b.mlp_ratio &&
+         a.frame_len == b.frame_len && a.max_frames == b.max_frames && a.dtype == b.dtype;
+}
+
+// ------------------------------------------------------------------ forward / stacks
+
+struct FwdCtx {
+  const af_model* const* blocks;
+  const af_dir* dirs;
+  int T, batch, L;
+  const float* x;
+  float* z;
+  float* logdet;
+  Bufs b;
+};
+
+af_status build_forward(void* vctx, cudaStream_t cs) {
+  FwdCtx* c = static_cast<FwdCtx*>(vctx);
+  const int G = (2 * c->blocks[0]->cfg.C) / 16;
+  const int m_max = c->batch * c->L;
+  for (int t = 0; t < c->T; ++t) {
+    // block t writes z when T-1-t is even, else tmp; block t reads what t-1 wrote
+    const float* in = t == 0 ? c->x : (((c->T - t) % 2 == 0) ? c->z : c->b.tmp);
+    float* out = ((c->T - 1 - t) % 2 == 0) ? c->z : c->b.tmp;
+    launch_ctl_forward(c->b.ctl, c->batch, c->L, cs);
+    HeadIO hio{0, in, out};
+    af_status s = enqueue_pass(c->blocks[t], c->b, c->batch, c->L, c->dirs[t], m_max, c->L, in, hio, cs);
+    if (s) return s;
+    launch_logdet_finalize(c->b.part, c->batch, c->L, G, c->logdet, t > 0, cs);
+  }
+  CK(cudaGetLastError());
+  return AF_OK;
+}
+
+struct InvCtx {
+  const af_model* const* blocks;
+  const af_dir* dirs;
+  int T, batch, L, B, max_iter, warm;
+  float tau;
+  const float* z;
+  float* x;
+  int32_t* iters;
+  Bufs b;
+};
+
+af_status build_inverse(void* vctx, cudaStream_t cs) {
+  InvCtx* c = static_cast<InvCtx*>(vctx);
+  const int nb = c->L / c->B;
+  for (int t = c->T - 1; t >= 0; --t) {
+    float* out = (t % 2 == 0) ? c->x : c->b.tmp;
+    const float* in = (t == c->T - 1) ? c->z : ((((t + 1) % 2) == 0) ? c->x : c->b.tmp);
+    JacobiJob jb{c->blocks[t], in, out, c->dirs[t], c->iters + (size_t)t * c->batch * nb, t == c->T - 1};
+    af_status s = capture_jacobi(jb, c->b, c->batch, c->L, c->B, c->tau, c->max_iter, c->warm, cs);
+    if (s) return s;
+  }
+  CK(cudaGetLastError());
+  return AF_OK;
+}
+
+af_status stack_checks(const af_model* const* blocks, const af_dir* dirs, int T) {
+  if (!blocks || !dirs || T < 1) { set_err("blocks/dirs/T"); return AF_ERR_ARG; }
+  for (int t = 0; t < T; ++t) {
+    if (!blocks[t]) { set_err("null block %d", t); return AF_ERR_ARG; }
+    if (!same_cfg(blocks[t]->cfg, blocks[0]->cfg)) { set_err("blocks must share one config"); return AF_ERR_ARG; }
+    if (dirs[t] != AF_L2R && dirs[t] != AF_R2L) { set_err("bad direction"); return AF_ERR_ARG; }
+  }
+  return AF_OK;
+}
+
+}  // namespace
+
+// ============================================================================ C ABI
+
+extern "C" {
+
+int af_num_tensors(const af_config* cfg) { return cfg ? 4 + 12 * cfg->layers + 4 : 0; }
+
+af_status af_model_create(const af_config* cfg, const float* const* tensors, int n_tensors, af_model** out) {
+  if (!cfg || !tensors || !out) { set_err("null argument"); return AF_ERR_ARG; }
+  const af_config c = *cfg;
+  if (c.C <= 0 || c.d <= 0 || c.heads <= 0 || c.layers <= 0 || c.mlp_ratio <= 0 || c.frame_len <= 0 ||
+      c.max_frames <= 0 || c.d % c.heads || c.C % 8 || c.d % 4) {
+    set_err("invalid config");
+    return AF_ERR_ARG;
+  }
+  const int hd = c.d / c.heads;
+  if (c.dtype == AF_FP32) {
+    if (hd != 16 && hd != 32 && hd != 64 && hd != 128) { set_err("fp32 path: head dim must be 16/32/64/128"); return AF_ERR_ARG; }
+  } else if (c.dtype == AF_BF16) {
+    if (c.C % 64 || c.d % 128 || (hd != 64 && hd != 128) || (c.mlp_ratio * c.d) % 128) {
+      set_err("bf16 path: needs C%%64==0, d%%128==0, head dim 64 or 128");
+      return AF_ERR_ARG;
+    }
+  } else {
+    set_err("bad dtype");
+    return AF_ERR_ARG;
+  }
+  if (n_tensors != af_num_tensors(cfg)) { set_err("expected %d tensors, got %d", af_num_tensors(cfg), n_tensors); return AF_ERR_ARG; }
+  for (int i = 0; i < n_tensors; ++i)
+    if (!tensors[i]) { set_err("null tensor %d", i); return AF_ERR_ARG; }
+
+  af_model* m = new af_model();
+  m->cfg = c;
+  m->fd = c.mlp_ratio * c.d;
+  m->hd = hd;
+  m->bf = c.dtype == AF_BF16;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (cudaDeviceGetAttribute(&m->num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    set_err("no CUDA device");
+    delete m;
+    return AF_ERR_CUDA;
+  }
+  bool fail = false;
+  auto upload_f32 = [&](const float* src, size_t n) -> float* {
+    void* p = nullptr;
+    if (cudaMalloc(&p, n * 4) != cudaSuccess || cudaMemcpy(p, src, n * 4, cudaMemcpyHostToDevice) != cudaSuccess) {
+      fail = true;
+      return nullptr;
+    }
+    m->allocs.push_back(p);
+    return (float*)p;
+  };
+  auto upload_w = [&](const float* src, size_t n) -> void* {   // matrices: bf16 or fp32
+    if (!m->bf) return upload_f32(src, n);
+    std::vector<uint16_t> tmp(n);
+    for (size_t i = 0; i < n; ++i) tmp[i] = f2bf(src[i]);
+    void* p = nullptr;
+    if (cudaMalloc(&p, n * 2) != cudaSuccess || cudaMemcpy(p, tmp.data(), n * 2, cudaMemcpyHostToDevice) != cudaSuccess) {
+      fail = true;
+      return nullptr;
+    }
+    m->allocs.push_back(p);
+    return p;
+  };
+  // vectors: bf16 models use bf16-rounded values held in fp32
+  auto upload_v = [&](const float* src, size_t n) -> float* {
+    if (!m->bf) return upload_f32(src, n);
+    std::vector<float> tmp(n);
+    for (size_t i = 0; i < n; ++i) {
+      const uint32_t u = (uint32_t)f2bf(src[i]) << 16;
+      memcpy(&tmp[i], &u, 4);
+    }
+    return upload_f32(tmp.data(), n);
+  };
+  const size_t d = c.d, C = c.C, fd = m->fd;
+  int k = 0;
+  m->w_in = upload_w(tensors[k++], d * C);
+  m->b_in = upload_v(tensors[k++], d);
+  m->pos_space = upload_v(tensors[k++], (size_t)c.frame_len * d);
+  m->pos_time = upload_v(tensors[k++], (size_t)c.max_frames * d);
+  for (int l = 0; l < c.layers; ++l) {
+    LayerW w;
+    w.ln1_g = upload_v(tensors[k++], d);
+    w.ln1_b = upload_v(tensors[k++], d);
+    w.w_qkv = upload_w(tensors[k++], 3 * d * d);
+    w.b_qkv = upload_v(tensors[k++], 3 * d);
+    w.w_o = upload_w(tensors[k++], d * d);
+    w.b_o = upload_v(tensors[k++], d);
+    w.ln2_g = upload_v(tensors[k++], d);
+    w.ln2_b = upload_v(tensors[k++], d);
+    w.w_1 = upload_w(tensors[k++], fd * d);
+    w.b_1 = upload_v(tensors[k++], fd);
+    w.w_2 = upload_w(tensors[k++], d * fd);
+    w.b_2 = upload_v(tensors[k++], d);
+    m->layers.push_back(w);
+  }
+  m->lnf_g = upload_v(tensors[k++], d);
+  m->lnf_b = upload_v(tensors[k++], d);
+  {
+    const float* wh = tensors[k++];
+    const float* bh = tensors[k++];
+    std::vector<float> wi(2 * C * d), bi(2 * C);
+    for (size_t ch = 0; ch < C; ++ch) {
+      memcpy(&wi[(2 * ch) * d], wh + ch * d, d * 4);
+      memcpy(&wi[(2 * ch + 1) * d], wh + (C + ch) * d, d * 4);
+      bi[2 * ch] = bh[ch];
+      bi[2 * ch + 1] = bh[C + ch];
+    }
+    m->w_head = upload_w(wi.data(), 2 * C * d);
+    m->b_head = upload_v(bi.data(), 2 * C);
+  }
+  void* e = nullptr;
+  if (cudaMalloc(&e, 256) != cudaSuccess || cudaMemset(e, 0, 256) != cudaSuccess) fail = true;
+  else m->allocs.push_back(e);
+  m->d_err = (int*)e;
+  if (!fail && (cudaStreamCreateWithFlags(&m->cap, cudaStreamNonBlocking) != cudaSuccess ||
+                cudaStreamCreateWithFlags(&m->cap2, cudaStreamNonBlocking) != cudaSuccess))
+    fail = true;
+  if (fail) {
+    set_err("device allocation/copy failed: %s", cudaGetErrorString(cudaGetLastError()));
+    for (void* p : m->allocs) cudaFree(p);
+    delete m;
+    return AF_ERR_CUDA;
+  }
+  *out = m;
+  return AF_OK;
+}
+
+af_status af_model_destroy(af_model* m) {
+  if (!m) return AF_ERR_ARG;
+  cudaDeviceSynchronize();
+  for (auto& kv : m->graphs) cudaGraphExecDestroy(kv.second);
+  for (void* p : m->allocs) cudaFree(p);
+  cudaStreamDestroy(m->cap);
+  cudaStreamDestroy(m->cap2);
+  delete m;
+  return AF_OK;
+}
+
+size_t af_workspace_bytes(const af_model* m, int batch, int L, int B) {
+  if (!m || batch < 1 || L < 1 || B < 1 || L > m->cfg.frame_len * m->cfg.max_frames || L % B) return 0;
+  return carve(m, nullptr, batch, L, B).total;
+}
+
+af_status af_forward(const af_model* m, const float* x, int batch, int L, af_dir dir, float* z, float* logdet,
+                     void* ws, size_t ws_bytes, void* stream) {
+  af_dir dirs[1] = {dir};
+  const af_model* blocks[1] = {m};
+  if (af_status s = check_model(m)) return s;
+  return flow_stack_forward(blocks, dirs, 1, x, batch, L, z, logdet, ws, ws_bytes, stream);
+}
+
+af_status flow_stack_forward(const af_model* const* blocks, const af_dir* dirs, int T, const float* x, int batch,
+                             int L, float* z, float* logdet, void* ws, size_t ws_bytes, void* stream) {
+  if (af_status s = stack_checks(blocks, dirs, T)) return s;
+  if (!x || !z || !logdet || x == z) { set_err("x/z/logdet (x and z must not alias)"); return AF_ERR_ARG; }
+  if (af_status s = check_ws(blocks[0], ws, ws_bytes, batch, L, L)) return s;
+  FwdCtx c{blocks, dirs, T, batch, L, x, z, logdet, carve(blocks[0], ws, batch, L, L)};
+  std::vector<long long> kv = {(long long)x, (long long)z, (long long)logdet, (long long)ws, batch, L, T};
+  std::string key = keyf("fwd", {});
+  for (int t = 0; t < T; ++t) key += keyf("", {(long long)blocks[t], dirs[t]});
+  for (long long v : kv) key += keyf("", {v});
+  return graph_run(blocks[0], key, (cudaStream_t)stream, build_forward, &c);
+}
+
+af_status af_inverse_jacobi(const af_model* m, const float* z, int batch, int L, af_dir dir, int B, float tau,
+                            int max_iter, int warm_start, float* x, int32_t* iters, void* ws, size_t ws_bytes,
+                            void* stream) {
+  af_dir dirs[1] = {dir};
+  const af_model* blocks[1] = {m};
+  if (af_status s = check_model(m)) return s;
+  return flow_stack_inverse(blocks, dirs, 1, z, batch, L, B, tau, max_iter, warm_start, x, iters, ws, ws_bytes,
+                            stream);
+}
+
+af_status flow_stack_inverse(const af_model* const* blocks, const af_dir* dirs, int T, const float* z, int batch,
+                             int L, int B, float tau, int max_iter, int warm_start, float* x, int32_t* iters,
+                             void* ws, size_t ws_bytes, void* stream) {
+  if (af_status s = stack_checks(blocks, dirs, T)) return s;
+  if (!z || !x || !iters || x == z) { set_err("z/x/iters (x and z must not alias)"); return AF_ERR_ARG; }
+  if (B < 1 || L % B || max_iter < 1 || !(tau >= 0.f) || tau == INFINITY) {
+    set_err("need L %% B == 0, max_iter >= 1, finite tau >= 0");
+    return AF_ERR_ARG;
+  }
+  if (af_status s = check_ws(blocks[0], ws, ws_bytes, batch, L, B)) return s;
+  InvCtx c{blocks, dirs, T, batch, L, B, max_iter, warm_start ? 1 : 0, tau, z, x, iters,
+           carve(blocks[0], ws, batch, L, B)};
+  uint32_t taubits;
+  memcpy(&taubits, &tau, 4);
+  std::string key = keyf("inv", {(long long)z, (long long)x, (long long)iters, (long long)ws, batch, L, B,
+                                 (long long)taubits, max_iter, c.warm, T});
+  for (int t = 0; t < T; ++t) key += keyf("", {(long long)blocks[t], dirs[t]});
+  return graph_run(blocks[0], key, (cudaStream_t)stream, build_inverse, &c);
+}
+
+af_status af_last_convergence(void* ws, int* n_unconverged, void* stream) {
+  if (!ws || !n_unconverged) { set_err("null argument"); return AF_ERR_ARG; }
+  CK(cudaStreamSynchronize((cudaStream_t)stream));
+  Ctl c;
+  CK(cudaMemcpy(&c, ws, sizeof c, cudaMemcpyDeviceToHost));
+  *n_unconverged = c.nonconv;
+  return c.nonconv ? AF_NOT_CONVERGED : AF_OK;
+}
+
+af_status af_device_error(const af_model* m, int* code) {
+  if (!m) { set_err("null model"); return AF_ERR_ARG; }
+  CK(cudaDeviceSynchronize());
+  int v = 0;
+  CK(cudaMemcpy(&v, m->d_err, sizeof v, cudaMemcpyDeviceToHost));
+  if (code) *code = v;
+  if (v) {
+    CK(cudaMemset(m->d_err, 0, sizeof v));
+    set_err("device error code %d", v);
+    return AF_ERR_DEVICE;
+  }
+  return AF_OK;
+}
+
+const char* af_status_string(af_status s) {
+  switch (s) {
+    case AF_OK: return "AF_OK";
+    case AF_ERR_ARG: return "AF_ERR_ARG: bad argument";
+    case AF_ERR_CUDA: return "AF_ERR_CUDA: a CUDA call failed";
+    case AF_ERR_WORKSPACE: return "AF_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case AF_NOT_CONVERGED: return "AF_NOT_CONVERGED: a block stopped at max_iter";
+    case AF_ERR_DEVICE: return "AF_ERR_DEVICE: a kernel gave up a bounded wait";
+  }
+  return "unknown af_status";
+}
+
+const char* af_last_error_string(void) { return g_errbuf; }
+
+}  // extern "C"

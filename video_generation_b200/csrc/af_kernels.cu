@@ -1,0 +1,425 @@
+// af_kernels.cu -- row-wise kernels, the Jacobi driver kernels and the fp32 SIMT path.
+//
+// Jacobi driver ("STARFlow-V ... paper notes", key design 3): the inverse of an
+// AF block runs as one CUDA graph with two nested device-side WHILE loops.
+// The outer loop walks the blocks of B tokens in sequence; the inner loop runs
+// Jacobi updates x^(k+1) = mu(x^(k)*m) + sigma(x^(k)*m) * z of the current
+// block until every sample's residual ||x^(k+1)-x^(k)||^2 / ||x^(k+1)||^2 is
+// below tau or max_iter updates ran.  The kernels below keep the iteration
+// counter, the per-sample convergence flags and the loop conditions in device
+// memory, so no iteration returns to the host.
+#include "af_kernels.h"
+
+namespace af {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Deterministic block sum (fixed shuffle tree, then warps in index order).
+__device__ float block_sum(float v) {
+  __shared__ float red[32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  float t = 0.f;
+  if (w == 0) {
+    t = lane < (int)(blockDim.x >> 5) ? red[lane] : 0.f;
+    t = warp_sum(t);
+  }
+  return t;   // valid in thread 0
+}
+
+int grid_for(long long work, int per_block) {
+  long long g = (work + per_block - 1) / per_block;
+  if (g < 1) g = 1;
+  if (g > 148 * 16) g = 148 * 16;
+  return (int)g;
+}
+
+// ------------------------------------------------------------------ control
+
+__global__ void k_ctl_forward(Ctl* ctl, int batch, int L) {
+  ctl->P = 0; ctl->p0 = 0; ctl->R = L; ctl->M = batch * L;
+  ctl->block = 0; ctl->iter = 0; ctl->n_active = 0;
+}
+
+__global__ void k_call_init(Ctl* ctl, int reset_nonconv) {
+  ctl->block = 0;
+  if (reset_nonconv) ctl->nonconv = 0;
+}
+
+// Start of Jacobi block b = ctl->block: the row layout of the first update
+// (block b-1 rides along to commit its K/V), fresh per-sample flags, and the
+// starting guess x^(0) = z_b, or block b-1's final x when warm starting.
+__global__ void k_block_init(Ctl* ctl, int* active, const float* __restrict__ z, float* x, int batch,
+                             int L, int C, int B, int dir, int warm,
+                             cudaGraphConditionalHandle inner) {
+  const int b = ctl->block;
+  const int P = b * B;
+  const int nvec = C >> 2;
+  const long long n = (long long)batch * B * nvec;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int cv = (int)(i % nvec);
+    const long long st = i / nvec;
+    const int t = (int)(st % B);
+    const int s = (int)(st / B);
+    const size_t dst = ((size_t)s * L + tok_of(P + t, L, dir)) * C + cv * 4;
+    float4 v;
+    if (warm && b > 0)
+      v = *reinterpret_cast<const float4*>(x + ((size_t)s * L + tok_of(P - B + t, L, dir)) * C + cv * 4);
+    else
+      v = *reinterpret_cast<const float4*>(z + dst);
+    *reinterpret_cast<float4*>(x + dst) = v;
+  }
+  if (blockIdx.x == 0) {
+    for (int s = threadIdx.x; s < batch; s += blockDim.x) active[s] = 1;
+    if (threadIdx.x == 0) {
+      const int p0 = b > 0 ? P - B : P;
+      ctl->P = P;
+      ctl->p0 = p0;
+      ctl->R = P + B - p0;
+      ctl->M = batch * (P + B - p0);
+      ctl->iter = 0;
+      ctl->n_active = batch;
+      cudaGraphSetConditional(inner, 1u);
+    }
+  }
+}
+
+// End of one Jacobi update: per-sample residual from the head's partial sums
+// (fixed summation order), the stopping test, the iteration counters and the
+// inner loop condition.  One block of 1024 threads; one warp per sample.
+__global__ void __launch_bounds__(1024) k_jacobi_step(Ctl* ctl, int* active, const float* __restrict__ part,
+                                                      int batch, int B, int G, float tau, int max_iter,
+                                                      int32_t* iters, int nblocks,
+                                                      cudaGraphConditionalHandle inner) {
+  const int R = ctl->R, p0 = ctl->p0, P = ctl->P, iter = ctl->iter, blk = ctl->block;
+  const int skip = P - p0;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int s = w; s < batch; s += nw) {
+    if (!active[s]) continue;
+    const float* p = part + ((size_t)s * R + skip) * G * 2;
+    const int n = B * G;
+    float num = 0.f, den = 0.f;
+    for (int i = lane; i < n; i += 32) {
+      num += p[2 * i];
+      den += p[2 * i + 1];
+    }
+    num = warp_sum(num);
+    den = warp_sum(den);
+    if (lane == 0) {
+      iters[(size_t)s * nblocks + blk] = iter + 1;
+      const bool conv = (den == 0.f) ? (num == 0.f) : (num / den < tau);
+      if (conv) active[s] = 0;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int na = 0;
+    for (int s = 0; s < batch; ++s) na += active[s];
+    ctl->iter = iter + 1;
+    ctl->n_active = na;
+    const bool cont = na > 0 && iter + 1 < max_iter;
+    if (!cont) ctl->nonconv += na;
+    ctl->p0 = P;
+    ctl->R = B;
+    ctl->M = batch * B;
+    cudaGraphSetConditional(inner, cont ? 1u : 0u);
+  }
+}
+
+__global__ void k_block_advance(Ctl* ctl, int nblocks, cudaGraphConditionalHandle outer) {
+  const int b = ctl->block + 1;
+  ctl->block = b;
+  cudaGraphSetConditional(outer, b < nblocks ? 1u : 0u);
+}
+
+// ------------------------------------------------------------------ row-wise
+
+// Self-exclusive mask as a one-token shift: the input of position p is
+// x_{p-1} (zero at p = 0), read through the direction flip.
+template <typename T>
+__global__ void k_gather(const Ctl* ctl, const float* __restrict__ x, int L, int C, int dir, T* xin) {
+  const int M = ctl->M, R = ctl->R, p0 = ctl->p0;
+  const int nvec = C >> 2;
+  const long long n = (long long)M * nvec;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int row = (int)(i / nvec);
+    const int c = (int)(i - (long long)row * nvec) * 4;
+    const int s = row / R;
+    const int p = p0 + (row - s * R);
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (p > 0) v = *reinterpret_cast<const float4*>(x + ((size_t)s * L + tok_of(p - 1, L, dir)) * C + c);
+    store4(xin + (size_t)row * C + c, v.x, v.y, v.z, v.w);
+  }
+}
+
+// LayerNorm (eps 1e-5), one warp per row, fp32 statistics (two passes over
+// registers: mean, then the centred variance).  NV = d / 128 float4 per lane.
+template <typename T, int NV>
+__global__ void k_layernorm_reg(const Ctl* ctl, const float* __restrict__ h, const float* __restrict__ g,
+                                const float* __restrict__ b, T* out, int d) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (row >= ctl->M) return;
+  const float4* hr = reinterpret_cast<const float4*>(h + (size_t)row * d);
+  float4 v[NV];
+  float sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    v[i] = hr[lane + 32 * i];
+    sum += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+  }
+  const float mean = warp_sum(sum) / d;
+  float sq = 0.f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const float a = v[i].x - mean, bb = v[i].y - mean, c = v[i].z - mean, e = v[i].w - mean;
+    sq += (a * a + bb * bb) + (c * c + e * e);
+  }
+  const float rstd = 1.0f / sqrtf(warp_sum(sq) / d + 1e-5f);
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = (lane + 32 * i) * 4;
+    const float4 gg = *reinterpret_cast<const float4*>(g + c);
+    const float4 bv = *reinterpret_cast<const float4*>(b + c);
+    store4(out + (size_t)row * d + c, (v[i].x - mean) * rstd * gg.x + bv.x,
+           (v[i].y - mean) * rstd * gg.y + bv.y, (v[i].z - mean) * rstd * gg.z + bv.z,
+           (v[i].w - mean) * rstd * gg.w + bv.w);
+  }
+}
+
+template <typename T>
+__global__ void k_layernorm_gen(const Ctl* ctl, const float* __restrict__ h, const float* __restrict__ g,
+                                const float* __restrict__ b, T* out, int d) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (row >= ctl->M) return;
+  const float* hr = h + (size_t)row * d;
+  float sum = 0.f;
+  for (int c = lane; c < d; c += 32) sum += hr[c];
+  const float mean = warp_sum(sum) / d;
+  float sq = 0.f;
+  for (int c = lane; c < d; c += 32) {
+    const float a = hr[c] - mean;
+    sq += a * a;
+  }
+  const float rstd = 1.0f / sqrtf(warp_sum(sq) / d + 1e-5f);
+  for (int c = lane; c < d; c += 32) out[(size_t)row * d + c] = to_act<T>((hr[c] - mean) * rstd * g[c] + b[c]);
+}
+
+// logdet[s] = -sum of s over the sample's rows and head groups (fixed order).
+__global__ void k_logdet_finalize(const float* __restrict__ part, int L, int G, float* logdet,
+                                  int accumulate) {
+  const int s = blockIdx.x;
+  const float* p = part + (size_t)s * L * G * 2;
+  float acc = 0.f;
+  for (int i = threadIdx.x; i < L * G; i += blockDim.x) acc += p[2 * i];
+  acc = block_sum(acc);
+  if (threadIdx.x == 0) logdet[s] = accumulate ? logdet[s] - acc : -acc;
+}
+
+// ------------------------------------------------------------------ fp32 SIMT path
+
+// C = A W^T, 64x64 tile, BK 16, 256 threads of 4x4 outputs.
+template <int EPI>
+__global__ void __launch_bounds__(256) k_gemm_simt(const float* __restrict__ A, const float* __restrict__ W,
+                                                   int N, int K, EpiArgs e) {
+  __shared__ float As[16][64 + 4];
+  __shared__ float Ws[16][64 + 4];
+  const int M = e.ctl->M;
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  if (m0 >= M) return;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    for (int i = tid; i < 64 * 16; i += 256) {
+      const int r = i >> 4, k = i & 15;
+      As[k][r] = (m0 + r < M && k0 + k < K) ? A[(size_t)(m0 + r) * K + k0 + k] : 0.f;
+      Ws[k][r] = (n0 + r < N && k0 + k < K) ? W[(size_t)(n0 + r) * K + k0 + k] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      float a[4], w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { a[i] = As[k][ty * 4 + i]; w[i] = Ws[k][tx * 4 + i]; }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], w[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  const int col = n0 + tx * 4;
+  if (col >= N) return;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int row = m0 + ty * 4 + i;
+    if (row < M) epi4<EPI, float>(e, row, col, acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+  }
+}
+
+// Head in fp32: one thread per (row, 16-column group), then the shared affine epilogue.
+__global__ void k_head_simt(const float* __restrict__ A, const float* __restrict__ W, int N, int K, EpiArgs e) {
+  const int G = N >> 4;
+  const int M = e.ctl->M;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= M * G) return;
+  const int row = i / G, g = i - row * G;
+  const float* a = A + (size_t)row * K;
+  float v[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const float* w = W + (size_t)(g * 16 + j) * K;
+    float s = 0.f;
+    for (int k = 0; k < K; ++k) s = fmaf(a[k], w[k], s);
+    v[j] = s;
+  }
+  head_group(e, row, g * 16, v);
+}
+
+// Causal attention in fp32: one warp per (row, head); lanes take keys
+// j = lane, lane+32, ... <= p with a running max / sum, merged at the end.
+template <int HD>
+__global__ void __launch_bounds__(256) k_attn_simt(const Ctl* ctl, const float* __restrict__ q,
+                                                   const float* __restrict__ kc, const float* __restrict__ vc,
+                                                   float* o, int Lc, int d, int heads) {
+  __shared__ float qs[8][HD];
+  const int wib = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * 8 + wib;
+  const int M = ctl->M;
+  if (gw >= M * heads) return;
+  const int row = gw / heads, hh = gw - row * heads;
+  const int R = ctl->R, s = row / R, p = ctl->p0 + (row - s * R);
+  const float scale = 1.0f / sqrtf((float)HD);
+  for (int i = lane; i < HD; i += 32) qs[wib][i] = q[(size_t)row * d + hh * HD + i];
+  __syncwarp();
+  const float* K = kc + (size_t)s * Lc * d + hh * HD;
+  const float* V = vc + (size_t)s * Lc * d + hh * HD;
+  float m = -INFINITY, l = 0.f, acc[HD];
+#pragma unroll
+  for (int i = 0; i < HD; ++i) acc[i] = 0.f;
+  for (int j = lane; j <= p; j += 32) {
+    float sc = 0.f;
+#pragma unroll
+    for (int i = 0; i < HD; ++i) sc = fmaf(qs[wib][i], K[(size_t)j * d + i], sc);
+    sc *= scale;
+    const float mn = fmaxf(m, sc);
+    const float corr = expf(m - mn), pj = expf(sc - mn);
+    l = l * corr + pj;
+#pragma unroll
+    for (int i = 0; i < HD; ++i) acc[i] = fmaf(pj, V[(size_t)j * d + i], acc[i] * corr);
+    m = mn;
+  }
+  const float mx = warp_max(m);
+  const float f = (m == -INFINITY) ? 0.f : expf(m - mx);
+  const float lt = warp_sum(l * f);
+#pragma unroll
+  for (int i = 0; i < HD; ++i) {
+    const float a = warp_sum(acc[i] * f);
+    if (lane == (i & 31)) o[(size_t)row * d + hh * HD + i] = a / lt;
+  }
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ launchers
+
+void launch_ctl_forward(Ctl* ctl, int batch, int L, cudaStream_t st) {
+  k_ctl_forward<<<1, 1, 0, st>>>(ctl, batch, L);
+}
+void launch_call_init(Ctl* ctl, int reset_nonconv, cudaStream_t st) {
+  k_call_init<<<1, 1, 0, st>>>(ctl, reset_nonconv);
+}
+
+template <typename T>
+void launch_gather(const Ctl* ctl, const float* x, int L, int C, int dir, T* xin, int m_max,
+                   cudaStream_t st) {
+  k_gather<T><<<grid_for((long long)m_max * (C / 4), kThreads), kThreads, 0, st>>>(ctl, x, L, C, dir, xin);
+}
+template void launch_gather<float>(const Ctl*, const float*, int, int, int, float*, int, cudaStream_t);
+template void launch_gather<bf16>(const Ctl*, const float*, int, int, int, bf16*, int, cudaStream_t);
+
+template <typename T>
+void launch_layernorm(const Ctl* ctl, const float* h, const float* g, const float* b, T* out, int d,
+                      int m_max, cudaStream_t st) {
+  const int grid = (m_max + 7) / 8;
+  switch (d % 128 == 0 ? d / 128 : 0) {
+    case 2: k_layernorm_reg<T, 2><<<grid, 256, 0, st>>>(ctl, h, g, b, out, d); break;
+    case 4: k_layernorm_reg<T, 4><<<grid, 256, 0, st>>>(ctl, h, g, b, out, d); break;
+    case 6: k_layernorm_reg<T, 6><<<grid, 256, 0, st>>>(ctl, h, g, b, out, d); break;
+    case 8: k_layernorm_reg<T, 8><<<grid, 256, 0, st>>>(ctl, h, g, b, out, d); break;
+    case 16: k_layernorm_reg<T, 16><<<grid, 256, 0, st>>>(ctl, h, g, b, out, d); break;
+    default: k_layernorm_gen<T><<<grid, 256, 0, st>>>(ctl, h, g, b, out, d); break;
+  }
+}
+template void launch_layernorm<float>(const Ctl*, const float*, const float*, const float*, float*, int, int, cudaStream_t);
+template void launch_layernorm<bf16>(const Ctl*, const float*, const float*, const float*, bf16*, int, int, cudaStream_t);
+
+void launch_logdet_finalize(const float* part, int batch, int L, int G, float* logdet, int accumulate,
+                            cudaStream_t st) {
+  k_logdet_finalize<<<batch, 256, 0, st>>>(part, L, G, logdet, accumulate);
+}
+
+void launch_block_init(Ctl* ctl, int* active, const float* z, float* x, int batch, int L, int C, int B,
+                       int dir, int warm, cudaGraphConditionalHandle inner, cudaStream_t st) {
+  k_block_init<<<grid_for((long long)batch * B * (C / 4), kThreads), kThreads, 0, st>>>(
+      ctl, active, z, x, batch, L, C, B, dir, warm, inner);
+}
+
+void launch_jacobi_step(Ctl* ctl, int* active, const float* part, int batch, int B, int G, float tau,
+                        int max_iter, int32_t* iters, int nblocks, cudaGraphConditionalHandle inner,
+                        cudaStream_t st) {
+  k_jacobi_step<<<1, 1024, 0, st>>>(ctl, active, part, batch, B, G, tau, max_iter, iters, nblocks, inner);
+}
+
+void launch_block_advance(Ctl* ctl, int nblocks, cudaGraphConditionalHandle outer, cudaStream_t st) {
+  k_block_advance<<<1, 1, 0, st>>>(ctl, nblocks, outer);
+}
+
+void launch_gemm_simt(int epi, const float* A, const float* W, int N, int K, int m_max, const EpiArgs& e,
+                      cudaStream_t st) {
+  dim3 grid((N + 63) / 64, (m_max + 63) / 64);
+  switch (epi) {
+    case EPI_INPROJ: k_gemm_simt<EPI_INPROJ><<<grid, 256, 0, st>>>(A, W, N, K, e); break;
+    case EPI_QKV: k_gemm_simt<EPI_QKV><<<grid, 256, 0, st>>>(A, W, N, K, e); break;
+    case EPI_RESID: k_gemm_simt<EPI_RESID><<<grid, 256, 0, st>>>(A, W, N, K, e); break;
+    case EPI_GELU: k_gemm_simt<EPI_GELU><<<grid, 256, 0, st>>>(A, W, N, K, e); break;
+    default: k_gemm_simt<EPI_RAW><<<grid, 256, 0, st>>>(A, W, N, K, e); break;
+  }
+}
+
+void launch_head_simt(const float* A, const float* W, int N, int K, int m_max, const EpiArgs& e,
+                      cudaStream_t st) {
+  const long long n = (long long)m_max * (N / 16);
+  k_head_simt<<<(int)((n + 127) / 128), 128, 0, st>>>(A, W, N, K, e);
+}
+
+void launch_attn_simt(const Ctl* ctl, const float* q, const float* kc, const float* vc, float* o, int batch,
+                      int Lc, int d, int heads, int m_max, cudaStream_t st) {
+  (void)batch;
+  const int grid = (int)(((long long)m_max * heads + 7) / 8);
+  switch (d / heads) {
+    case 16: k_attn_simt<16><<<grid, 256, 0, st>>>(ctl, q, kc, vc, o, Lc, d, heads); break;
+    case 32: k_attn_simt<32><<<grid, 256, 0, st>>>(ctl, q, kc, vc, o, Lc, d, heads); break;
+    case 64: k_attn_simt<64><<<grid, 256, 0, st>>>(ctl, q, kc, vc, o, Lc, d, heads); break;
+    default: k_attn_simt<128><<<grid, 256, 0, st>>>(ctl, q, kc, vc, o, Lc, d, heads); break;
+  }
+}
+
+}  // namespace af

@@ -1,0 +1,53 @@
+// af_kernels.h -- host-side launchers of libaf's kernels (internal, C++ linkage).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include "af_common.cuh"
+
+namespace af {
+
+// ---- small kernels (af_kernels.cu) -----------------------------------------
+// All row-wise kernels read the live row count from ctl->M and are launched
+// for `m_max` rows.
+void launch_ctl_forward(Ctl* ctl, int batch, int L, cudaStream_t st);
+template <typename T>
+void launch_gather(const Ctl* ctl, const float* x, int L, int C, int dir, T* xin, int m_max,
+                   cudaStream_t st);
+template <typename T>
+void launch_layernorm(const Ctl* ctl, const float* h, const float* g, const float* b, T* out,
+                      int d, int m_max, cudaStream_t st);
+void launch_logdet_finalize(const float* part, int batch, int L, int G, float* logdet,
+                            int accumulate, cudaStream_t st);
+void launch_call_init(Ctl* ctl, int reset_nonconv, cudaStream_t st);
+void launch_block_init(Ctl* ctl, int* active, const float* z, float* x, int batch, int L, int C,
+                       int B, int dir, int warm, cudaGraphConditionalHandle inner,
+                       cudaStream_t st);
+void launch_jacobi_step(Ctl* ctl, int* active, const float* part, int batch, int B, int G,
+                        float tau, int max_iter, int32_t* iters, int nblocks,
+                        cudaGraphConditionalHandle inner, cudaStream_t st);
+void launch_block_advance(Ctl* ctl, int nblocks, cudaGraphConditionalHandle outer,
+                          cudaStream_t st);
+
+// ---- fp32 SIMT path (af_kernels.cu) -----------------------------------------
+void launch_gemm_simt(int epi, const float* A, const float* W, int N, int K, int m_max,
+                      const EpiArgs& e, cudaStream_t st);
+void launch_head_simt(const float* A, const float* W, int N, int K, int m_max, const EpiArgs& e,
+                      cudaStream_t st);
+void launch_attn_simt(const Ctl* ctl, const float* q, const float* kc, const float* vc, float* o,
+                      int batch, int Lc, int d, int heads, int m_max, cudaStream_t st);
+
+// ---- tensor-core bf16 path ---------------------------------------------------
+// TMA descriptor of a row-major bf16 matrix [rows, cols] tiled as boxes of
+// [box_rows, 64 columns] with 128-byte swizzle (af_gemm_tc.cu).
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int rows, int cols, int box_rows);
+// C[M, N] = A[M, K] W[N, K]^T with epilogue `epi`; N % bn == 0, K % 64 == 0.
+void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, int bn, int N, int K,
+                    int m_max, const EpiArgs& e, int* err, int num_sms, cudaStream_t st);
+int gemm_tc_pick_bn(int N, int m_max, int num_sms);
+
+// Causal attention over the KV cache, bf16 tensor cores (af_attn.cu).
+void launch_attn_tc(const Ctl* ctl, const bf16* q, const bf16* kc, const bf16* vc, bf16* o,
+                    int batch, int Lc, int d, int heads, int r_max, cudaStream_t st);
+
+}  // namespace af

@@ -1,0 +1,191 @@
+"""Thin Python binding of libaf (include/af.h): argument marshalling only.
+
+Every step of the affine-autoregressive-flow path runs in libaf's CUDA
+kernels; PyTorch only provides device memory and the current stream.  If
+libaf.so is missing or cannot load, importing this module raises: there is no
+fallback path.
+
+Names follow the C ABI: ``af_forward``, ``af_inverse_jacobi``,
+``flow_stack_forward``, ``flow_stack_inverse``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import List, Sequence
+
+import numpy as np
+import torch
+
+L2R, R2L = 0, 1
+FP32, BF16 = 0, 1
+
+AF_OK, AF_ERR_ARG, AF_ERR_CUDA, AF_ERR_WORKSPACE, AF_NOT_CONVERGED, AF_ERR_DEVICE = range(6)
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libaf.so")
+
+EXPORTS = ("af_num_tensors", "af_model_create", "af_model_destroy", "af_workspace_bytes", "af_forward",
+           "af_inverse_jacobi", "flow_stack_forward", "flow_stack_inverse", "af_last_convergence",
+           "af_device_error", "af_status_string", "af_last_error_string")
+
+
+class AFConfigC(ctypes.Structure):
+    _fields_ = [("C", ctypes.c_int), ("d", ctypes.c_int), ("heads", ctypes.c_int), ("layers", ctypes.c_int),
+                ("mlp_ratio", ctypes.c_int), ("frame_len", ctypes.c_int), ("max_frames", ctypes.c_int),
+                ("dtype", ctypes.c_int)]
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise RuntimeError(f"libaf.so not built at {path}: run `python -m video_generation_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i, sz, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    P = ctypes.POINTER
+    lib.af_num_tensors.argtypes = [P(AFConfigC)]
+    lib.af_num_tensors.restype = i
+    lib.af_model_create.argtypes = [P(AFConfigC), P(vp), i, P(vp)]
+    lib.af_model_destroy.argtypes = [vp]
+    lib.af_workspace_bytes.argtypes = [vp, i, i, i]
+    lib.af_workspace_bytes.restype = sz
+    lib.af_forward.argtypes = [vp, vp, i, i, i, vp, vp, vp, sz, vp]
+    lib.af_inverse_jacobi.argtypes = [vp, vp, i, i, i, i, f, i, i, vp, vp, vp, sz, vp]
+    lib.flow_stack_forward.argtypes = [P(vp), P(i), i, vp, i, i, vp, vp, vp, sz, vp]
+    lib.flow_stack_inverse.argtypes = [P(vp), P(i), i, vp, i, i, i, f, i, i, vp, vp, vp, sz, vp]
+    lib.af_last_convergence.argtypes = [vp, P(i), vp]
+    lib.af_device_error.argtypes = [vp, P(i)]
+    lib.af_status_string.argtypes = [i]
+    lib.af_status_string.restype = ctypes.c_char_p
+    lib.af_last_error_string.argtypes = []
+    lib.af_last_error_string.restype = ctypes.c_char_p
+    for name in EXPORTS:
+        if name not in ("af_status_string", "af_last_error_string", "af_num_tensors", "af_workspace_bytes"):
+            getattr(lib, name).restype = i
+    return lib
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        _lib = load_library()
+    return _lib
+
+
+class AFError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        L = lib()
+        msg = f"{L.af_status_string(status).decode()}: {L.af_last_error_string().decode()}"
+        super().__init__(f"{what}: {msg}" if what else msg)
+        self.status = status
+
+
+def _check(status: int, what: str):
+    if status != AF_OK:
+        raise AFError(status, what)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class AFModel:
+    """One AF block's weights on the current CUDA device (owned by libaf)."""
+
+    def __init__(self, shape, tensors: Sequence[np.ndarray]):
+        self.shape = shape
+        self.cfg = AFConfigC(shape.C, shape.d, shape.heads, shape.layers, shape.mlp_ratio, shape.frame_len,
+                             shape.max_frames, BF16 if shape.dtype == "bf16" else FP32)
+        arrs = [np.ascontiguousarray(t, dtype=np.float32) for t in tensors]
+        ptrs = (ctypes.c_void_p * len(arrs))(*[a.ctypes.data for a in arrs])
+        h = ctypes.c_void_p()
+        _check(lib().af_model_create(ctypes.byref(self.cfg), ptrs, len(arrs), ctypes.byref(h)), "af_model_create")
+        self.handle = h
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lib().af_model_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def workspace_bytes(self, batch: int, L: int, B: int | None = None) -> int:
+        return int(lib().af_workspace_bytes(self.handle, batch, L, L if B is None else B))
+
+    def workspace(self, batch: int, L: int, B: int | None = None, device=None) -> torch.Tensor:
+        n = self.workspace_bytes(batch, L, B)
+        if n == 0:
+            raise AFError(AF_ERR_ARG, "af_workspace_bytes")
+        return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+    def device_error(self) -> int:
+        code = ctypes.c_int(0)
+        lib().af_device_error(self.handle, ctypes.byref(code))
+        return code.value
+
+
+def af_forward(model: AFModel, x: torch.Tensor, direction: int, ws: torch.Tensor | None = None,
+               z: torch.Tensor | None = None, logdet: torch.Tensor | None = None, stream=None):
+    """z = (x - mu) * exp(-s), logdet = -sum s per sample; x [batch, L, C] fp32 on the device."""
+    return flow_stack_forward([model], [direction], x, ws=ws, z=z, logdet=logdet, stream=stream)
+
+
+def af_inverse_jacobi(model: AFModel, z: torch.Tensor, direction: int, B: int, tau: float, max_iter: int,
+                      warm_start: bool, ws: torch.Tensor | None = None, x: torch.Tensor | None = None,
+                      iters: torch.Tensor | None = None, stream=None):
+    """Block-Jacobi inverse; returns (x, iters [batch, L/B])."""
+    x, it = flow_stack_inverse([model], [direction], z, B, tau, max_iter, warm_start, ws=ws, x=x,
+                               iters=None if iters is None else iters.view(1, *iters.shape), stream=stream)
+    return x, it[0]
+
+
+def flow_stack_forward(models: List[AFModel], dirs: Sequence[int], x: torch.Tensor, ws: torch.Tensor | None = None,
+                       z: torch.Tensor | None = None, logdet: torch.Tensor | None = None, stream=None):
+    batch, L, _ = x.shape
+    if ws is None:
+        ws = models[0].workspace(batch, L, device=x.device)
+    z = torch.empty_like(x) if z is None else z
+    logdet = torch.empty(batch, dtype=torch.float32, device=x.device) if logdet is None else logdet
+    T = len(models)
+    hs = (ctypes.c_void_p * T)(*[m.handle for m in models])
+    ds = (ctypes.c_int * T)(*dirs)
+    _check(lib().flow_stack_forward(hs, ds, T, _ptr(x), batch, L, _ptr(z), _ptr(logdet), _ptr(ws), ws.numel(),
+                                    _stream(stream)), "flow_stack_forward")
+    return z, logdet
+
+
+def flow_stack_inverse(models: List[AFModel], dirs: Sequence[int], z: torch.Tensor, B: int, tau: float,
+                       max_iter: int, warm_start: bool, ws: torch.Tensor | None = None,
+                       x: torch.Tensor | None = None, iters: torch.Tensor | None = None, stream=None):
+    batch, L, _ = z.shape
+    T = len(models)
+    if ws is None:
+        ws = models[0].workspace(batch, L, B, device=z.device)
+    x = torch.empty_like(z) if x is None else x
+    if iters is None:
+        iters = torch.zeros((T, batch, L // max(B, 1)), dtype=torch.int32, device=z.device)
+    hs = (ctypes.c_void_p * T)(*[m.handle for m in models])
+    ds = (ctypes.c_int * T)(*dirs)
+    _check(lib().flow_stack_inverse(hs, ds, T, _ptr(z), batch, L, B, float(tau), int(max_iter), int(bool(warm_start)),
+                                    _ptr(x), _ptr(iters), _ptr(ws), ws.numel(), _stream(stream)),
+           "flow_stack_inverse")
+    return x, iters
+
+
+def last_convergence(ws: torch.Tensor, stream=None) -> int:
+    """Synchronises and returns how many (sample, block) pairs stopped at max_iter unconverged."""
+    n = ctypes.c_int(0)
+    s = lib().af_last_convergence(_ptr(ws), ctypes.byref(n), _stream(stream))
+    if s not in (AF_OK, AF_NOT_CONVERGED):
+        _check(s, "af_last_convergence")
+    return n.value
