@@ -206,9 +206,11 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
               make_tmap_bf16(&tA_u, u, m_max, fd, 128);
     if (!ok) { set_err("cuTensorMapEncodeTiled failed for an activation"); return AF_ERR_CUDA; }
     auto gemm = [&](int epi, const CUtensorMap& tA, const void* W, int N, int K, const EpiArgs& ea) -> bool {
-      const int bn = gemm_tc_pick_bn(N, m_max, ns);
-      if (!bn || !make_tmap_bf16(&tB, W, N, K, bn)) return false;
-      launch_gemm_tc(epi, tA, tB, bn, N, K, m_max, ea, m->d_err, ns, st);
+      // a QKV tile must fall inside one of q, k, v; the position-add epilogue
+      // keeps two row sets in flight and stays at <= 192 columns
+      const int pick = gemm_tc_pick(N, m_max, ns, epi == EPI_QKV ? d : 0, epi == EPI_INPROJ ? 192 : 256);
+      if (!pick || !make_tmap_bf16(&tB, W, N, K, (pick / 10) / (pick % 10))) return false;
+      launch_gemm_tc(epi, tA, tB, pick, N, K, m_max, ea, m->d_err, ns, st);
       return true;
     };
     launch_gather<bf16>(b.ctl, xsrc, L, C, dir, xin, m_max, st);

@@ -7,14 +7,16 @@
 // block's causal Transformer: input projection, QKV, attention output
 // projection, the two MLP matrices and the (mu, log-sigma) head.
 //
-// Design (one persistent CTA per SM, 256 threads):
+// Design (one persistent CTA per SM, 384 threads):
 //   warp 0      TMA producer: 128x64 A tile + BNx64 W tile per stage,
 //               128-byte swizzle, mbarrier transaction counts.
 //   warp 1      owns 512 TMEM columns; one thread issues tcgen05.mma
 //               (M=128, N=BN, K=16) into one of two accumulators and commits
 //               to the stage's "empty" barrier and the accumulator's "full".
-//   warps 4..7  epilogue: tcgen05.ld 32 lanes x 16 columns per warp, apply
-//               the fused epilogue, release the accumulator.
+//   warps 4..11 epilogue, two warps per TMEM lane quarter (each takes half
+//               of the tile's columns): tcgen05.ld 32 lanes x 16 columns,
+//               transpose through shared memory, apply the fused epilogue
+//               with row-coalesced stores, release the accumulator.
 // With two accumulators the epilogue of tile i overlaps the MMAs of tile i+1.
 // No cluster, no multicast: each CTA loads its own tiles.
 // Every wait is bounded (2 s); on expiry the CTA raises its abort flag, drains
@@ -28,16 +30,20 @@ namespace {
 constexpr int BM = 128, BK = 64;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-template <int BN> struct TcCfg {
-  static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 192 ? 5 : 6);
+template <int BN, int CG> struct TcCfg {
+  // CG = CTAs per MMA: 1, or 2 for the SM-pair MMA (tile of 256 rows, each CTA
+  // holding 128 rows of A and BN/2 rows of W).
+  static constexpr int STAGES = CG == 2 ? (BN >= 256 ? 6 : (BN >= 192 ? 6 : 7)) : (BN >= 256 ? 4 : (BN >= 192 ? 5 : 6));
   static constexpr uint32_t A_BYTES = BM * BK * 2;
-  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr uint32_t B_BYTES = (BN / CG) * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t NBARS = 2 * STAGES + 5;
-  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + NBARS * 8 + 16;
+  // per epilogue warp (8 of them): a 32 x 16 fp32 staging tile, 16-byte chunks XOR-swizzled
+  static constexpr uint32_t EPI_BYTES = 8 * 32 * 16 * 4;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + NBARS * 8 + 16;
   // instruction descriptor: F32 accumulate, BF16 A and B, both K-major, N>>3, M>>4
   static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                                    ((uint32_t)(BM >> 4) << 24);
+                                    ((uint32_t)((BM * CG) >> 4) << 24);
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -113,25 +119,100 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-template <int BN, int EPI>
-__global__ void __launch_bounds__(256, 1)
+// ---- SM-pair (cta_group::2) helpers
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// TMA load into this CTA's shared memory whose completion is counted on an
+// mbarrier of either CTA of the pair (no multicast).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
+                                                 int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+      "[%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                               uint32_t accum) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accum));
+}
+// commit of the pair's MMAs, arriving on the barrier at this offset in both CTAs
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
+  const uint16_t mask = 3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit_pair_local(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// GELU with erf from Abramowitz & Stegun, Handbook of Mathematical Functions,
+// formula 7.1.26 (Hastings): erf(u) = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5))))
+// exp(-u^2), t = 1 / (1 + p u), u >= 0, |error| <= 1.5e-7 -- far below the bf16
+// rounding of the MLP activations it feeds.  The fp32 SIMT path keeps erff.
+__device__ __forceinline__ float gelu_as7126(float v) {
+  const float u = fabsf(v) * 0.70710678118654752f;
+  const float t = __fdividef(1.0f, fmaf(0.3275911f, u, 1.0f));
+  float q = fmaf(t, 1.061405429f, -1.453152027f);
+  q = fmaf(t, q, 1.421413741f);
+  q = fmaf(t, q, -0.284496736f);
+  q = fmaf(t, q, 0.254829592f);
+  const float erf_abs = 1.0f - q * t * __expf(-u * u);
+  return 0.5f * v * (1.0f + copysignf(erf_abs, v));
+}
+
+__device__ __forceinline__ void st_bf16x4(bf16* dst, float a, float b, float c, float d) {
+  __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&lo);
+  u.y = *reinterpret_cast<uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(dst) = u;
+}
+
+template <int BN, int EPI, int CG>
+__global__ void __launch_bounds__(384, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int N, int K,
               EpiArgs e, int* err) {
-  using Cfg = TcCfg<BN>;
+  using Cfg = TcCfg<BN, CG>;
   constexpr int S = Cfg::STAGES;
+  constexpr int TM = BM * CG;               // accumulator rows per tile (both CTAs)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* sA = smem;
   uint8_t* sB = smem + S * Cfg::A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + S * Cfg::B_BYTES);
+  float* sEpi = reinterpret_cast<float*>(sB + S * Cfg::B_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + S * Cfg::B_BYTES + Cfg::EPI_BYTES);
   // bars: full[S], empty[S], tfull[2], tempty[2], drain
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   volatile int* abort_flag = &s_abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = CG == 2 ? cluster_rank() : 0u;   // 0 = the pair's leader (issues the MMAs)
+  const int unit = CG == 2 ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int nunits = CG == 2 ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   const int M = e.ctl->M;
-  const int tiles_m = (M + BM - 1) / BM, tiles_n = N / BN;
+  const int tiles_m = (M + TM - 1) / TM, tiles_n = N / BN;
   const int ntiles = tiles_m * tiles_n;
   const int kbn = K / BK;
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S);
@@ -146,7 +227,7 @@ __global__ void __launch_bounds__(256, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(tfull0 + 8 * i, 1);
-      mbar_init(tempty0 + 8 * i, 128);
+      mbar_init(tempty0 + 8 * i, 256 * CG);
     }
     mbar_init(drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -154,53 +235,75 @@ __global__ void __launch_bounds__(256, 1)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
-                 "r"(512));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    if (CG == 2) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
+                   "r"(512));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
+                   "r"(512));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if (CG == 2) cluster_sync();   // the peer's barriers exist before any remote signal
   tc_fence_after();
   const uint32_t tmem = s_tmem;
+  const uint32_t full_lead = CG == 2 ? map_to_rank(full0, 0) : full0;
+  const uint32_t tempty_lead = CG == 2 ? map_to_rank(tempty0, 0) : tempty0;
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------------------------------------------------------- producer
+      // ---------------------------------------------------------------- producer (both CTAs)
       int stage = 0;
       uint32_t phase = 0;
       long long issued = 0;
-      for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      for (int t = unit; t < ntiles; t += nunits) {
         const int mb = t % tiles_m, nb = t / tiles_m;
+        const int arow = mb * TM + (int)rank * BM;
+        const int brow = nb * BN + (int)rank * (BN / CG);
         bool ok = true;
         for (int kb = 0; kb < kbn; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag)) { ok = false; break; }
-          mbar_expect_tx(full0 + 8 * stage, Cfg::STAGE_BYTES);
-          tma_load_2d(smem_u32(sA + stage * Cfg::A_BYTES), &tmA, full0 + 8 * stage, kb * BK, mb * BM);
-          tma_load_2d(smem_u32(sB + stage * Cfg::B_BYTES), &tmB, full0 + 8 * stage, kb * BK, nb * BN);
+          if (rank == 0) mbar_expect_tx(full0 + 8 * stage, CG * Cfg::STAGE_BYTES);
+          if (CG == 2) {
+            tma_load_2d_pair(smem_u32(sA + stage * Cfg::A_BYTES), &tmA, full_lead + 8 * stage, kb * BK, arow);
+            tma_load_2d_pair(smem_u32(sB + stage * Cfg::B_BYTES), &tmB, full_lead + 8 * stage, kb * BK, brow);
+          } else {
+            tma_load_2d(smem_u32(sA + stage * Cfg::A_BYTES), &tmA, full0 + 8 * stage, kb * BK, arow);
+            tma_load_2d(smem_u32(sB + stage * Cfg::B_BYTES), &tmB, full0 + 8 * stage, kb * BK, brow);
+          }
           ++issued;
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
       }
-      // drain: the last load of every stage has landed before the CTA exits
-      const long long n = issued < S ? issued : S;
-      for (long long j = 1; j <= n; ++j) {
-        const long long idx = issued - j;
-        const int st = (int)(idx % S);
-        const uint32_t ph = (uint32_t)((idx / S) & 1);
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try(full0 + 8 * st, ph)) {
-          if (globaltimer_ns() - t0 > kWaitLimitNs) { atomicExch(err, ERR_GEMM_DRAIN); break; }
+      if (CG == 1) {
+        // drain: the last load of every stage has landed before the CTA exits
+        const long long n = issued < S ? issued : S;
+        for (long long j = 1; j <= n; ++j) {
+          const long long idx = issued - j;
+          const int st = (int)(idx % S);
+          const uint32_t ph = (uint32_t)((idx / S) & 1);
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try(full0 + 8 * st, ph)) {
+            if (globaltimer_ns() - t0 > kWaitLimitNs) { atomicExch(err, ERR_GEMM_DRAIN); break; }
+          }
         }
+      } else if (*abort_flag) {
+        // the pair's completion counts live on the leader; give in-flight copies time to land
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0 && rank == 0) {
+      // ---------------------------------------------------------------- MMA issuer (leader only)
       int stage = 0;
       uint32_t phase = 0;
       int i = 0;
-      for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
+      for (int t = unit; t < ntiles; t += nunits, ++i) {
         const int acc = i & 1;
         const uint32_t use = (uint32_t)(i >> 1);
         if (!mbar_wait(tempty0 + 8 * acc, (use & 1u) ^ 1u, abort_flag)) break;
@@ -213,87 +316,230 @@ __global__ void __launch_bounds__(256, 1)
           const uint64_t da = sw128_desc(smem_u32(sA + stage * Cfg::A_BYTES));
           const uint64_t db = sw128_desc(smem_u32(sB + stage * Cfg::B_BYTES));
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            umma_bf16(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), Cfg::IDESC, (kb | k) != 0);
-          umma_commit(empty0 + 8 * stage);
+          for (int k = 0; k < BK / 16; ++k) {
+            if (CG == 2) umma_bf16_pair(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), Cfg::IDESC, (kb | k) != 0);
+            else umma_bf16(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), Cfg::IDESC, (kb | k) != 0);
+          }
+          if (CG == 2) umma_commit_pair(empty0 + 8 * stage);
+          else umma_commit(empty0 + 8 * stage);
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        umma_commit(tfull0 + 8 * acc);
+        if (CG == 2) umma_commit_pair(tfull0 + 8 * acc);
+        else umma_commit(tfull0 + 8 * acc);
       }
       // drain: every MMA issued by this thread has completed
-      umma_commit(drain);
+      if (CG == 2) umma_commit_pair_local(drain);
+      else umma_commit(drain);
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try(drain, 0)) {
         if (globaltimer_ns() - t0 > kWaitLimitNs) { atomicExch(err, ERR_GEMM_DRAIN); break; }
       }
     }
   } else if (warp >= 4) {
-    // ------------------------------------------------------------------ epilogue
+      // ---------------------------------------------------------------- epilogue
+    // Warp 4+ew owns TMEM lane quarter q = ew % 4 (rows 32q..32q+31 of the
+    // tile) and column half ew / 4.  A 16-column chunk is read from TMEM
+    // (thread = row), transposed through a swizzled 32x16 staging tile, and
+    // applied with lane l on row 8*it + l/4, columns 4*(l%4)..+3: each store
+    // covers eight 64-byte row segments.  Row -> (sample, position) and the
+    // destination row pointers are computed once per tile.
     const int ew = warp - 4;
+    const int q = ew & 3, hf = ew >> 2;
+    constexpr int HALF = BN / 2;
+    float* stg = sEpi + ew * 32 * 16;
+    const int rl = lane >> 2, cq = lane & 3;
+    const int sw_w = (lane >> 1) & 3;            // swizzle of the row this lane writes
+    const int sw_r = (rl >> 1) & 3;              // swizzle of the rows this lane reads
+    const Ctl* ctl = e.ctl;
+    const int R = ctl->R, p0 = ctl->p0;
     int i = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
+    for (int t = unit; t < ntiles; t += nunits, ++i) {
       const int acc = i & 1;
       const uint32_t use = (uint32_t)(i >> 1);
-      if (!mbar_wait(tfull0 + 8 * acc, use & 1u, abort_flag)) break;
-      tc_fence_after();
       const int mb = t % tiles_m, nb = t / tiles_m;
-      const int row = mb * BM + ew * 32 + lane;
-      const int n0 = nb * BN;
-      const uint32_t taddr = tmem + (uint32_t)(acc * BN) + ((uint32_t)(ew * 32) << 16);
-#pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
-        float v[32];
-        tmem_ld16(taddr + c, v);
-        tmem_ld16(taddr + c + 16, v + 16);
-        tmem_wait_ld();
-        if (row < M) {
-          if (EPI == EPI_HEAD) {
-            head_group(e, row, n0 + c, v);
-            head_group(e, row, n0 + c + 16, v + 16);
-          } else {
+      const int row0 = mb * TM + (int)rank * BM + q * 32;
+      const int n0 = nb * BN + hf * HALF;
+      const uint32_t taddr = tmem + (uint32_t)(acc * BN + hf * HALF) + ((uint32_t)(q * 32) << 16);
+      // per-tile row info for the 4 rows this lane stores
+      char* rowp[4];
+      const float* pos_s[4];
+      const float* pos_t[4];
+      int colbase = 0;
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              epi4<EPI, bf16>(e, row, n0 + c + 4 * j, v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+      for (int it = 0; it < 4; ++it) {
+        const int r = row0 + it * 8 + rl;
+        if (EPI == EPI_RESID) rowp[it] = reinterpret_cast<char*>(e.h + (size_t)r * e.d);
+        if (EPI == EPI_GELU) rowp[it] = reinterpret_cast<char*>(reinterpret_cast<bf16*>(e.out) + (size_t)r * e.ldo);
+        if (EPI == EPI_INPROJ || EPI == EPI_QKV) {
+          const int sm = r / R;
+          const int p = p0 + (r - sm * R);
+          if (EPI == EPI_INPROJ) {
+            rowp[it] = reinterpret_cast<char*>(e.h + (size_t)r * e.d);
+            pos_s[it] = e.pos_space + (size_t)(p % e.frame_len) * e.d;
+            pos_t[it] = e.pos_time + (size_t)(p / e.frame_len) * e.d;
+          } else {
+            const int which = (nb * BN) / e.d;            // the whole tile is q, k or v
+            if (which == 0) rowp[it] = reinterpret_cast<char*>(reinterpret_cast<bf16*>(e.out) + (size_t)r * e.d);
+            else
+              rowp[it] = reinterpret_cast<char*>(reinterpret_cast<bf16*>(which == 1 ? e.kc : e.vc) +
+                                                 ((size_t)sm * e.Lc + p) * e.d);
+            colbase = which * e.d;
           }
         }
       }
+      // Loads that do not depend on the accumulator are issued before waiting
+      // for it (bias, and the first chunk's residual / position rows), and
+      // every chunk's TMEM load and global loads are in flight while the
+      // previous chunk is transposed and stored.
+      constexpr int NCH = HALF / 16;
+      float4 bias4[NCH];
+#pragma unroll
+      for (int k = 0; k < NCH; ++k) bias4[k] = *reinterpret_cast<const float4*>(e.bias + n0 + k * 16 + cq * 4);
+      float4 pre[2][4], pre2[2][4];
+      auto load_rows = [&](int k, float4* dst, float4* dst2) {
+        const int col = n0 + k * 16 + cq * 4;
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+          if (row0 + it * 8 + rl < M) {
+            if (EPI == EPI_RESID) dst[it] = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(rowp[it]) + col);
+            if (EPI == EPI_INPROJ) {
+              dst[it] = *reinterpret_cast<const float4*>(pos_s[it] + col);
+              dst2[it] = *reinterpret_cast<const float4*>(pos_t[it] + col);
+            }
+          }
+        }
+      };
+      if (EPI == EPI_RESID || EPI == EPI_INPROJ) load_rows(0, pre[0], pre2[0]);
+      if (!mbar_wait(tfull0 + 8 * acc, use & 1u, abort_flag)) break;
+      tc_fence_after();
+      float vb[2][16];
+      tmem_ld16(taddr, vb[0]);
+#pragma unroll
+      for (int k = 0; k < NCH; ++k) {
+        const int c = k * 16;
+        tmem_wait_ld();
+        if (k + 1 < NCH) {
+          tmem_ld16(taddr + c + 16, vb[(k + 1) & 1]);
+          if (EPI == EPI_RESID || EPI == EPI_INPROJ) load_rows(k + 1, pre[(k + 1) & 1], pre2[(k + 1) & 1]);
+        }
+        const float* v = vb[k & 1];
+        if (EPI == EPI_HEAD) {
+          if (row0 + lane < M) head_group(e, row0 + lane, n0 + c, v);
+          continue;
+        }
+        float4* srow = reinterpret_cast<float4*>(stg + lane * 16);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) srow[j ^ sw_w] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        __syncwarp();
+        float4 a[4];
+#pragma unroll
+        for (int it = 0; it < 4; ++it) a[it] = reinterpret_cast<const float4*>(stg + (it * 8 + rl) * 16)[cq ^ sw_r];
+        __syncwarp();
+        const int col = n0 + c + cq * 4;
+        const float4 bb = bias4[k];
+        if (EPI == EPI_RESID) {
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            if (row0 + it * 8 + rl < M) {
+              float4 hv = pre[k & 1][it];
+              hv.x += a[it].x + bb.x; hv.y += a[it].y + bb.y;
+              hv.z += a[it].z + bb.z; hv.w += a[it].w + bb.w;
+              *reinterpret_cast<float4*>(reinterpret_cast<float*>(rowp[it]) + col) = hv;
+            }
+          }
+        } else if (EPI == EPI_INPROJ) {
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            if (row0 + it * 8 + rl < M) {
+              const float4 ps = pre[k & 1][it], pt = pre2[k & 1][it];
+              *reinterpret_cast<float4*>(reinterpret_cast<float*>(rowp[it]) + col) =
+                  make_float4(a[it].x + bb.x + ps.x + pt.x, a[it].y + bb.y + ps.y + pt.y,
+                              a[it].z + bb.z + ps.z + pt.z, a[it].w + bb.w + ps.w + pt.w);
+            }
+          }
+        } else if (EPI == EPI_GELU) {
+#pragma unroll
+          for (int it = 0; it < 4; ++it)
+            if (row0 + it * 8 + rl < M)
+              st_bf16x4(reinterpret_cast<bf16*>(rowp[it]) + col, gelu_as7126(a[it].x + bb.x),
+                        gelu_as7126(a[it].y + bb.y), gelu_as7126(a[it].z + bb.z), gelu_as7126(a[it].w + bb.w));
+        } else if (EPI == EPI_QKV) {
+#pragma unroll
+          for (int it = 0; it < 4; ++it)
+            if (row0 + it * 8 + rl < M)
+              st_bf16x4(reinterpret_cast<bf16*>(rowp[it]) + (col - colbase), a[it].x + bb.x, a[it].y + bb.y,
+                        a[it].z + bb.z, a[it].w + bb.w);
+        }
+      }
       tc_fence_before();
-      mbar_arrive(tempty0 + 8 * acc);
+      if (CG == 2) mbar_arrive_cluster(tempty_lead + 8 * acc);
+      else mbar_arrive(tempty0 + 8 * acc);
     }
   }
   tc_fence_before();
   __syncthreads();
+  if (CG == 2) cluster_sync();   // the leader's MMAs (writing both TMEMs) are drained
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+    if (CG == 2) asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+    else asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
   }
   if (threadIdx.x == 0 && s_abort) atomicExch(err, ERR_GEMM_WAIT);
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, int CG>
 void launch_bn_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, int N, int K, int m_max, const EpiArgs& e,
                    int* err, int num_sms, cudaStream_t st) {
-  using Cfg = TcCfg<BN>;
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_gemm_tc<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM);
-    attr = true;
+  using Cfg = TcCfg<BN, CG>;
+  static int max_units = 0;
+  if (!max_units) {
+    cudaFuncSetAttribute(k_gemm_tc<BN, EPI, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM);
+    max_units = num_sms / CG;
+    if (CG == 2) {
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(2 * max_units);
+      q.blockDim = dim3(384);
+      q.dynamicSmemBytes = Cfg::SMEM;
+      cudaLaunchAttribute a[1];
+      a[0].id = cudaLaunchAttributeClusterDimension;
+      a[0].val.clusterDim.x = 2; a[0].val.clusterDim.y = 1; a[0].val.clusterDim.z = 1;
+      q.attrs = a;
+      q.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, k_gemm_tc<BN, EPI, CG>, &q) == cudaSuccess && clusters > 0 &&
+          clusters < max_units)
+        max_units = clusters;
+    }
   }
-  const int tiles = ((m_max + BM - 1) / BM) * (N / BN);
-  const int grid = tiles < num_sms ? tiles : num_sms;
-  k_gemm_tc<BN, EPI><<<grid, 256, Cfg::SMEM, st>>>(tmA, tmB, N, K, e, err);
+  const int tiles = ((m_max + BM * CG - 1) / (BM * CG)) * (N / BN);
+  const int units = tiles < max_units ? tiles : max_units;
+  if (CG == 1) {
+    k_gemm_tc<BN, EPI, 1><<<units, 384, Cfg::SMEM, st>>>(tmA, tmB, N, K, e, err);
+  } else {
+    cudaLaunchConfig_t c = {};
+    c.gridDim = dim3(2 * units);
+    c.blockDim = dim3(384);
+    c.dynamicSmemBytes = Cfg::SMEM;
+    c.stream = st;
+    cudaLaunchAttribute a[1];
+    a[0].id = cudaLaunchAttributeClusterDimension;
+    a[0].val.clusterDim.x = 2; a[0].val.clusterDim.y = 1; a[0].val.clusterDim.z = 1;
+    c.attrs = a;
+    c.numAttrs = 1;
+    cudaLaunchKernelEx(&c, k_gemm_tc<BN, EPI, CG>, tmA, tmB, N, K, e, err);
+  }
 }
 
-template <int BN>
+template <int BN, int CG>
 void launch_bn(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, int N, int K, int m_max,
                const EpiArgs& e, int* err, int num_sms, cudaStream_t st) {
   switch (epi) {
-    case EPI_INPROJ: launch_bn_epi<BN, EPI_INPROJ>(tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
-    case EPI_QKV: launch_bn_epi<BN, EPI_QKV>(tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
-    case EPI_RESID: launch_bn_epi<BN, EPI_RESID>(tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
-    case EPI_GELU: launch_bn_epi<BN, EPI_GELU>(tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
-    default: launch_bn_epi<BN, EPI_HEAD>(tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
+    case EPI_INPROJ: launch_bn_epi<BN, EPI_INPROJ, CG>(tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
+    case EPI_QKV: launch_bn_epi<BN, EPI_QKV, CG>(tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
+    case EPI_RESID: launch_bn_epi<BN, EPI_RESID, CG>(tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
+    case EPI_GELU: launch_bn_epi<BN, EPI_GELU, CG>(tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
+    default: launch_bn_epi<BN, EPI_HEAD, CG>(tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
   }
 }
 
@@ -323,27 +569,40 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int rows, int cols, int 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Tile width: the candidate (dividing N) with the fewest column-waves of
-// work, ceil(tiles / SMs) * BN; ties go to the wider tile.
-int gemm_tc_pick_bn(int N, int m_max, int num_sms) {
+// Tile shape: SM-pair MMAs (256-row tiles) when there are at least 256 rows,
+// and the width (<= max_bn, dividing N, and `unit` when non-zero) with the fewest waves of
+// work, ceil(tiles / units) * BN; ties go to the wider tile.  Returns
+// BN * 10 + CG.
+int gemm_tc_pick(int N, int m_max, int num_sms, int unit, int max_bn) {
   const int cands[3] = {256, 192, 128};
+  const int cg = m_max >= 256 ? 2 : 1;
+  const int units = num_sms / cg;
   int best = 0;
   long long best_cost = 0;
   for (int bn : cands) {
-    if (N % bn) continue;
-    const long long tiles = (long long)((m_max + BM - 1) / BM) * (N / bn);
-    const long long cost = ((tiles + num_sms - 1) / num_sms) * bn;
+    if (N % bn || (unit && unit % bn) || bn > max_bn) continue;
+    const long long tiles = (long long)((m_max + BM * cg - 1) / (BM * cg)) * (N / bn);
+    const long long cost = ((tiles + units - 1) / units) * bn;
     if (!best || cost < best_cost) { best = bn; best_cost = cost; }
   }
-  return best;
+  return best ? best * 10 + cg : 0;
 }
 
-void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, int bn, int N, int K, int m_max,
+void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, int pick, int N, int K, int m_max,
                     const EpiArgs& e, int* err, int num_sms, cudaStream_t st) {
-  switch (bn) {
-    case 256: launch_bn<256>(epi, tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
-    case 192: launch_bn<192>(epi, tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
-    default: launch_bn<128>(epi, tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
+  const int bn = pick / 10, cg = pick % 10;
+  if (cg == 2) {
+    switch (bn) {
+      case 256: launch_bn<256, 2>(epi, tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
+      case 192: launch_bn<192, 2>(epi, tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
+      default: launch_bn<128, 2>(epi, tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
+    }
+  } else {
+    switch (bn) {
+      case 256: launch_bn<256, 1>(epi, tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
+      case 192: launch_bn<192, 1>(epi, tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
+      default: launch_bn<128, 1>(epi, tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
+    }
   }
 }
 

@@ -41,10 +41,12 @@ void launch_attn_simt(const Ctl* ctl, const float* q, const float* kc, const flo
 // TMA descriptor of a row-major bf16 matrix [rows, cols] tiled as boxes of
 // [box_rows, 64 columns] with 128-byte swizzle (af_gemm_tc.cu).
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int rows, int cols, int box_rows);
-// C[M, N] = A[M, K] W[N, K]^T with epilogue `epi`; N % bn == 0, K % 64 == 0.
-void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, int bn, int N, int K,
+// C[M, N] = A[M, K] W[N, K]^T with epilogue `epi`, K % 64 == 0.  `pick` =
+// BN * 10 + CG from gemm_tc_pick (N % BN == 0); tmA boxes are 128 rows, tmB
+// boxes BN / CG rows.
+void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, int pick, int N, int K,
                     int m_max, const EpiArgs& e, int* err, int num_sms, cudaStream_t st);
-int gemm_tc_pick_bn(int N, int m_max, int num_sms);
+int gemm_tc_pick(int N, int m_max, int num_sms, int unit, int max_bn);
 
 // Causal attention over the KV cache, bf16 tensor cores (af_attn.cu).
 void launch_attn_tc(const Ctl* ctl, const bf16* q, const bf16* kc, const bf16* vc, bf16* o,
