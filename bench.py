@@ -33,6 +33,7 @@ sys.path.insert(0, ROOT)
 
 import synthetic as syn  # noqa: E402
 from video_generation_b200 import flops as FL  # noqa: E402
+from video_generation_b200 import replicas  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -162,7 +163,7 @@ def reference_arm(args, w, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", type=int, default=3, help="workload id (3 = f_S stack, the default)")
@@ -194,8 +195,8 @@ def main():
 
     models = [flow.AFModel(w.shape, syn.make_weights(w.shape, block=t)) for t in range(w.T)]
     # each rank inverts its own clip: distinct seeds per rank
-    x_np = syn.make_latents(w.batch, w.L, w.shape.C, syn.DATA_SEED + w.cid + 1000 * rank)
-    z_np = syn.make_latents(w.batch, w.L, w.shape.C, syn.DATA_SEED + w.cid + 100 + 1000 * rank)
+    x_np = syn.make_latents(w.batch, w.L, w.shape.C, replicas.rank_seed(syn.DATA_SEED + w.cid, rank))
+    z_np = syn.make_latents(w.batch, w.L, w.shape.C, replicas.rank_seed(syn.DATA_SEED + w.cid + 100, rank))
     x = torch.from_numpy(x_np).to(dev)
     z_in = torch.from_numpy(z_np).to(dev)
     ws_f = models[0].workspace(w.batch, w.L, w.L, device=dev)
@@ -241,9 +242,7 @@ def main():
         dist.barrier()
     t_fwd = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
     t_inv = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
-    t = torch.tensor([t_fwd, t_inv], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    t = replicas.max_over_ranks(torch.tensor([t_fwd, t_inv], dtype=torch.float64, device=dev), dist)
     t_fwd, t_inv = float(t[0]), float(t[1])
 
     # algorithmic work from the iterations actually run
@@ -273,9 +272,8 @@ def main():
         x_host.copy_(xi, non_blocking=True)
     e2e_ev[1].record(st)
     torch.cuda.synchronize()
-    t_e2e = torch.tensor([e2e_ev[0].elapsed_time(e2e_ev[1]) / 1e3], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_e2e, op=dist.ReduceOp.MAX)
+    t_e2e = replicas.max_over_ranks(
+        torch.tensor([e2e_ev[0].elapsed_time(e2e_ev[1]) / 1e3], dtype=torch.float64, device=dev), dist)
     e2e_val = tok / float(t_e2e[0])
     bytes_step = w.batch * w.L * w.shape.C * 4
 
