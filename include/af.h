@@ -123,6 +123,21 @@ af_status flow_stack_inverse(const af_model* const* blocks, const af_dir* dirs, 
                              int warm_start, float* x, int32_t* iters, void* ws,
                              size_t ws_bytes, void* stream);
 
+/* af_forward for callers that cannot allocate device memory -- a host that
+ * owns the whole GPU memory through its own allocator, or a plugin that is
+ * handed only its input and output buffers, and so cannot provide a
+ * workspace.  No counterpart in the paper.  Same arguments and
+ * results as af_forward minus the workspace: the call runs in a scratch array
+ * inside the library, 32 MiB per device, held by every GPU that loads libaf.so
+ * until the process exits.  Returns AF_ERR_WORKSPACE (with a message in
+ * af_last_error_string) when af_workspace_bytes(m, batch, L, L) exceeds
+ * 32 MiB.  The first call on a device looks up the array's address; make it
+ * before any stream capture.  Calls share the array: calls whose GPU work
+ * overlaps (other streams, other threads) race; serialise them.  Allocates
+ * nothing and launches its kernels directly on `stream`. */
+af_status af_forward_noalloc(const af_model* m, const float* x, int batch, int L, af_dir dir,
+                             float* z, float* logdet, void* stream);
+
 /* Synchronises `stream` and reports how many (sample, block) pairs of the
  * last inverse call on this workspace stopped at max_iter without passing
  * the test: AF_OK if none, AF_NOT_CONVERGED otherwise (*n_unconverged set). */

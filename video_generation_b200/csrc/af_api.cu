@@ -474,6 +474,26 @@ af_status stack_checks(const af_model* const* blocks, const af_dir* dirs, int T)
 
 }  // namespace
 
+// ------------------------------------------------------------------ direct launch (no graph)
+
+namespace af {
+
+void set_error_text(const char* msg) { set_err("%s", msg); }
+
+// The forward pass of one block launched kernel by kernel on `st`, with the
+// workspace at `ws`; used by af_forward_noalloc.
+af_status forward_direct(const af_model* m, const float* x, int batch, int L, af_dir dir, float* z, float* logdet,
+                         void* ws, size_t ws_bytes, cudaStream_t st) {
+  const af_model* blocks[1] = {m};
+  af_dir dirs[1] = {dir};
+  if (af_status s = stack_checks(blocks, dirs, 1)) return s;
+  if (af_status s = check_ws(m, ws, ws_bytes, batch, L, L)) return s;
+  FwdCtx c{blocks, dirs, 1, batch, L, x, z, logdet, carve(m, ws, batch, L, L)};
+  return build_forward(&c, st);
+}
+
+}  // namespace af
+
 // ============================================================================ C ABI
 
 extern "C" {

@@ -26,7 +26,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libaf.so")
 
 EXPORTS = ("af_num_tensors", "af_model_create", "af_model_destroy", "af_workspace_bytes", "af_forward",
            "af_inverse_jacobi", "flow_stack_forward", "flow_stack_inverse", "af_last_convergence",
-           "af_device_error", "af_status_string", "af_last_error_string")
+           "af_device_error", "af_status_string", "af_last_error_string", "af_forward_noalloc")
 
 
 class AFConfigC(ctypes.Structure):
@@ -51,6 +51,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.af_inverse_jacobi.argtypes = [vp, vp, i, i, i, i, f, i, i, vp, vp, vp, sz, vp]
     lib.flow_stack_forward.argtypes = [P(vp), P(i), i, vp, i, i, vp, vp, vp, sz, vp]
     lib.flow_stack_inverse.argtypes = [P(vp), P(i), i, vp, i, i, i, f, i, i, vp, vp, vp, sz, vp]
+    lib.af_forward_noalloc.argtypes = [vp, vp, i, i, i, vp, vp, vp]
     lib.af_last_convergence.argtypes = [vp, P(i), vp]
     lib.af_device_error.argtypes = [vp, P(i)]
     lib.af_status_string.argtypes = [i]
