@@ -115,11 +115,17 @@ def count_launches(w, iters_np):
 def run_oracle_sample(w, frames: int):
     """The CPU oracle on `frames` frames of the workload: forward stack and Jacobi inverse.
 
+    Frames are batch entries for the per-frame shallow stack, and the first
+    `frames` blocks of the sequence (a causal prefix) for the deep flow.
     Returns (tokens, fwd seconds, inverse seconds, threads used)."""
     from oracle import af_oracle as O
     blocks = [O.Block(w.shape, syn.make_weights(w.shape, block=t)) for t in range(w.T)]
-    x = syn.workload_latents(w, "x")[:frames]
-    z = syn.workload_latents(w, "z")[:frames]
+    if w.L > w.B:
+        x = syn.workload_latents(w, "x")[:1, :frames * w.B]
+        z = syn.workload_latents(w, "z")[:1, :frames * w.B]
+    else:
+        x = syn.workload_latents(w, "x")[:frames]
+        z = syn.workload_latents(w, "z")[:frames]
     t0 = time.perf_counter()
     O.stack_forward(blocks, w.dirs, x)
     t1 = time.perf_counter()
@@ -130,7 +136,7 @@ def run_oracle_sample(w, frames: int):
         threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:
         threads = os.cpu_count()
-    return frames * w.L, t1 - t0, t2 - t1, threads
+    return x.shape[0] * x.shape[1], t1 - t0, t2 - t1, threads
 
 
 def reference_arm(args, w, rank, world):
@@ -152,7 +158,7 @@ def reference_arm(args, w, rank, world):
             "ms_per_step": 1e3 * (ti + tf) / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "fwd_tokens_per_s": tok / tf,
-            "config": {"workload": w.name, "frames_per_step": frames, "tokens_per_step": frames * w.L},
+            "config": {"workload": w.name, "frames_per_step": frames, "tokens_per_step": tok // args.steps},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                              "sample": f"{frames} of {w.batch} frames per step, full T={w.T} stack "
                                        f"forward and Jacobi inverse"},

@@ -1,0 +1,95 @@
+"""The deep frame-causal flow f_D at full size (24 layers, d 2048, 16 heads of 128,
+8190 and 46800 tokens, block-Jacobi B = 390 with KV cache and warm start).
+
+The GPU runs the full-size workload in the configuration the bench times; the
+CPU oracle computes the causal prefix of the same inputs, which the full
+result must reproduce exactly up to rounding because later tokens never reach
+earlier ones ("STARFlow-V ... paper notes", key design 3: causal blocks, KV
+cache of finished blocks).  The rest of the sequence is checked by properties
+that hold at any size: the inverse's round trip through the forward, and the
+iteration cap.  bf16 tolerances as in test_gpu_parity.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synthetic as syn
+from oracle import af_oracle as O
+from tests.gpu_util import rel, to_dev, to_np
+
+pytestmark = pytest.mark.gpu
+
+BF_X_TOL, BF_PART_TOL, BF_RT_TOL = 2e-2, 3e-2, 2e-2
+
+
+@pytest.fixture(scope="module")
+def fd():
+    from video_generation_b200 import build
+    build.build()
+    from video_generation_b200 import flow
+    assert torch.cuda.is_available()
+    shape = syn.WORKLOADS[4].shape          # configs 4 and 5 share the model
+    W = syn.make_weights(shape)
+    model = flow.AFModel(shape, W)
+    blk = O.Block(shape, W)
+    del W
+    return flow, model, blk
+
+
+@pytest.mark.parametrize("cid", [4, 5])
+def test_fd_forward_full_size_prefix_matches_oracle(fd, cid):
+    flow, model, blk = fd
+    w = syn.WORKLOADS[cid]
+    x = syn.workload_latents(w, "x")
+    z, ld = flow.af_forward(model, to_dev(x), O.L2R)
+    torch.cuda.synchronize()
+    assert model.device_error() == 0
+    n = w.B                                  # first frame: exact by causality
+    z_ref, _ = O.af_forward(blk, x[:, :n], O.L2R)
+    zn = to_np(z)[:, :n]
+    assert rel(zn, z_ref) <= BF_X_TOL
+    assert rel(zn - x[:, :n], z_ref - x[:, :n]) <= BF_PART_TOL
+    assert np.isfinite(to_np(z)).all() and np.isfinite(to_np(ld)).all()
+
+
+def test_fd_5s_inverse_full_size_prefix_matches_oracle(fd):
+    flow, model, blk = fd
+    w = syn.WORKLOADS[4]
+    z = syn.workload_latents(w, "z")
+    ws = model.workspace(w.batch, w.L, w.B)
+    x, it = flow.af_inverse_jacobi(model, to_dev(z), O.L2R, w.B, w.tau, w.max_iter, w.warm_start, ws=ws)
+    nonconv = flow.last_convergence(ws)
+    assert model.device_error() == 0
+    # the first two blocks (warm start and one KV-cache commit) against the oracle
+    n = 2 * w.B
+    x_ref, it_ref, conv_ref = O.af_inverse_jacobi(blk, z[:, :n], O.L2R, w.B, w.tau, w.max_iter, True)
+    xn = to_np(x)
+    assert rel(xn[:, :n], x_ref) <= BF_X_TOL
+    assert rel(xn[:, :n] - z[:, :n], x_ref - z[:, :n]) <= BF_PART_TOL
+    itn = it.cpu().numpy()
+    assert np.abs(itn[:, :2] - it_ref).max() <= 1
+    assert (itn >= 1).all() and (itn <= w.max_iter).all()
+    assert 0 <= nonconv <= int((itn == w.max_iter).sum())
+    # the whole 21-frame result: forward(inverse(z)) returns z
+    zz, _ = flow.af_forward(model, x, O.L2R)
+    assert rel(to_np(zz), z) <= BF_RT_TOL
+
+
+def test_fd_30s_inverse_full_size(fd):
+    flow, model, blk = fd
+    w = syn.WORKLOADS[5]
+    z = syn.workload_latents(w, "z")
+    ws = model.workspace(w.batch, w.L, w.B)
+    x, it = flow.af_inverse_jacobi(model, to_dev(z), O.L2R, w.B, w.tau, w.max_iter, w.warm_start, ws=ws)
+    flow.last_convergence(ws)
+    assert model.device_error() == 0
+    n = w.B
+    x_ref, it_ref, _ = O.af_inverse_jacobi(blk, z[:, :n], O.L2R, w.B, w.tau, w.max_iter, True)
+    xn = to_np(x)
+    assert rel(xn[:, :n], x_ref) <= BF_X_TOL
+    assert np.abs(it.cpu().numpy()[:, :1] - it_ref).max() <= 1
+    # 120 frames: the round trip through the forward holds everywhere, late frames included
+    zz, _ = flow.af_forward(model, x, O.L2R)
+    zn = to_np(zz)
+    assert rel(zn, z) <= BF_RT_TOL
+    assert rel(zn[:, -w.B:], z[:, -w.B:]) <= BF_RT_TOL

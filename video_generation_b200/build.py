@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libaf.so")
-SOURCES = ["af_api.cu", "af_kernels.cu", "af_gemm_tc.cu", "af_attn.cu", "af_noalloc.cu"]
+SOURCES = ["af_api.cu", "af_kernels.cu", "af_gemm_tc.cu", "af_attn_tc.cu", "af_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I" + INCLUDE, "-I" + CSRC]
 

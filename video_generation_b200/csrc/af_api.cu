@@ -90,7 +90,11 @@ struct Bufs {
   void* q;
   void* u;
   void* kv;
+  size_t kv_bytes;
   float* tmp;
+  float* opart;   // split-attention partials (bf16 path)
+  float* mlpart;
+  int nsplit;
   size_t total;
 };
 
@@ -117,8 +121,14 @@ Bufs carve(const af_model* m, void* ws, int batch, int L, int B) {
   b.a = take(es * mmax * c.d);
   b.q = take(es * mmax * c.d);
   b.u = take(es * mmax * m->fd);
-  b.kv = take(es * (size_t)c.layers * 2 * batch * L * c.d);
+  b.kv_bytes = es * (size_t)c.layers * 2 * batch * L * c.d;
+  b.kv = take(b.kv_bytes);
   b.tmp = (float*)take(sizeof(float) * (size_t)batch * L * c.C);
+  b.nsplit = m->bf ? attn_tc_splits(batch, c.heads, rows_per_sample(L, B), L, m->num_sms) : 1;
+  if (b.nsplit > 1) {
+    b.opart = (float*)take(sizeof(float) * (size_t)b.nsplit * mmax * c.d);
+    b.mlpart = (float*)take(sizeof(float) * (size_t)b.nsplit * mmax * c.heads * 2);
+  }
   b.total = off;
   return b;
 }
@@ -226,7 +236,11 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
       eq.kc = kvl;
       eq.vc = kvl + kv_layer;
       if (!gemm(EPI_QKV, tA_a, w.w_qkv, 3 * d, d, eq)) { set_err("GEMM plan failed (qkv)"); return AF_ERR_CUDA; }
-      launch_attn_tc(b.ctl, q, (const bf16*)kvl, (const bf16*)(kvl + kv_layer), a, batch, L, d, c.heads, r_max, st);
+      if (!launch_attn_tc2(b.ctl, q, (const bf16*)kvl, (const bf16*)(kvl + kv_layer), a, b.opart, b.mlpart, b.nsplit,
+                           batch, L, d, c.heads, r_max, m_max, m->d_err, st)) {
+        set_err("attention plan failed");
+        return AF_ERR_CUDA;
+      }
       EpiArgs eo = e;
       eo.bias = w.b_o;
       if (!gemm(EPI_RESID, tA_a, w.w_o, d, d, eo)) { set_err("GEMM plan failed (out)"); return AF_ERR_CUDA; }
@@ -423,6 +437,8 @@ af_status build_forward(void* vctx, cudaStream_t cs) {
   FwdCtx* c = static_cast<FwdCtx*>(vctx);
   const int G = (2 * c->blocks[0]->cfg.C) / 16;
   const int m_max = c->batch * c->L;
+  // keys past a tile's last needed position are masked, but must be finite
+  if (c->blocks[0]->bf) CK(cudaMemsetAsync(c->b.kv, 0, c->b.kv_bytes, cs));
   for (int t = 0; t < c->T; ++t) {
     // block t writes z when T-1-t is even, else tmp; block t reads what t-1 wrote
     const float* in = t == 0 ? c->x : (((c->T - t) % 2 == 0) ? c->z : c->b.tmp);
@@ -451,6 +467,7 @@ struct InvCtx {
 af_status build_inverse(void* vctx, cudaStream_t cs) {
   InvCtx* c = static_cast<InvCtx*>(vctx);
   const int nb = c->L / c->B;
+  if (c->blocks[0]->bf) CK(cudaMemsetAsync(c->b.kv, 0, c->b.kv_bytes, cs));
   for (int t = c->T - 1; t >= 0; --t) {
     float* out = (t % 2 == 0) ? c->x : c->b.tmp;
     const float* in = (t == c->T - 1) ? c->z : ((((t + 1) % 2) == 0) ? c->x : c->b.tmp);

@@ -411,7 +411,8 @@ __global__ void __launch_bounds__(384, 1)
         }
       };
       if (EPI == EPI_RESID || EPI == EPI_INPROJ) load_rows(0, pre[0], pre2[0]);
-      if (!mbar_wait(tfull0 + 8 * acc, use & 1u, abort_flag)) break;
+      // the wait's outcome is made warp-uniform before the .aligned TMEM loads
+      if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * acc, use & 1u, abort_flag))) break;
       tc_fence_after();
       float vb[2][16];
       tmem_ld16(taddr, vb[0]);

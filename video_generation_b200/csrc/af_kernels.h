@@ -48,8 +48,13 @@ void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, int
                     int m_max, const EpiArgs& e, int* err, int num_sms, cudaStream_t st);
 int gemm_tc_pick(int N, int m_max, int num_sms, int unit, int max_bn);
 
-// Causal attention over the KV cache, bf16 tensor cores (af_attn.cu).
-void launch_attn_tc(const Ctl* ctl, const bf16* q, const bf16* kc, const bf16* vc, bf16* o,
-                    int batch, int Lc, int d, int heads, int r_max, cudaStream_t st);
+// Causal attention over the KV cache on tcgen05 (af_attn_tc.cu).  nsplit key
+// splits (attn_tc_splits); with nsplit > 1, opart [nsplit, m_max, d] and
+// mlpart [nsplit, m_max, heads, 2] hold the partials.  False if a tensor map
+// cannot be encoded.
+int attn_tc_splits(int batch, int heads, int r_max, int Lc, int num_sms);
+bool launch_attn_tc2(const Ctl* ctl, const bf16* q, const bf16* kc, const bf16* vc, bf16* o, float* opart,
+                     float* mlpart, int nsplit, int batch, int Lc, int d, int heads, int r_max, int m_max, int* err,
+                     cudaStream_t st);
 
 }  // namespace af
