@@ -7,8 +7,10 @@
 // and the current block's rows attend causally among themselves ("STARFlow-V
 // ... paper notes", key design 3: finished blocks feed a KV cache).
 //
-// One CTA: 128 query rows of one (sample, head) against the key tiles of one
-// split of the key range, 128 keys per tile.
+// Persistent CTAs (one per SM) walk a static list of work items: 128 query rows
+// of one (sample, head) against the key tiles of one split of the key range,
+// 128 keys per tile.  Q and the O accumulator are double-buffered across items
+// so the next item's loads and MMAs overlap the current item's softmax.
 //   warp 0      TMA: Q once (128 x hd), then K and V tiles (128 keys x hd)
 //               into a 2-3 stage ring; 128-byte swizzle.
 //   warp 1      one thread issues S_j = Q K_j^T (M=128, N=128, K=hd) into one
@@ -40,9 +42,11 @@ template <int HD> struct AttnCfg {
   static constexpr uint32_t Q_BYTES = KCH * BOX;
   static constexpr uint32_t KV_BYTES = KCH * BOX;         // K or V tile
   static constexpr int STAGES = HD == 64 ? 3 : 2;
-  static constexpr uint32_t P_BYTES = 2 * BOX;            // 128 rows x 128 keys
-  static constexpr size_t SMEM = 1024 + Q_BYTES + (size_t)STAGES * 2 * KV_BYTES + P_BYTES + 3 * 2 * 128 * 4 +
-                                 (2 * STAGES + 8 + 12) * 8 + 64;
+  static constexpr int QBUF = HD == 64 ? 2 : 1;            // Q buffers across work items
+  static constexpr int PB = HD == 64 ? 2 : 1;              // P tiles (softmax j+1 overlaps P_j V_j)
+  static constexpr uint32_t P_BYTES = 2 * BOX;            // one P tile: 128 rows x 128 keys
+  static constexpr size_t SMEM = 1024 + QBUF * Q_BYTES + (size_t)STAGES * 2 * KV_BYTES + PB * P_BYTES +
+                                 3 * 2 * 128 * 4 + (2 * STAGES + 27) * 8 + 64;
   // S = Q K^T: M 128, N 128, both K-major
   static constexpr uint32_t IDESC_S = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BKV >> 3) << 17) |
                                       ((uint32_t)(BQ >> 4) << 24);
@@ -134,6 +138,12 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// 2^x on the special-function unit (flush-to-zero; 2^-inf = +0)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -144,7 +154,7 @@ struct AttnArgs {
   bf16* o;           // [Mmax, d] output (nsplit == 1)
   float* opart;      // [nsplit, Mmax, d] unnormalised partial outputs (nsplit > 1)
   float* mlpart;     // [nsplit, Mmax, heads, 2] running max (log2 units) and row sum
-  int Lc, d, heads, nsplit, tiles_per_split, m_max;
+  int Lc, d, heads, nsplit, tiles_per_split, m_max, batch;
 };
 
 template <int HD>
@@ -155,14 +165,16 @@ __global__ void __launch_bounds__(384, 1)
   constexpr int S = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + Cfg::Q_BYTES;
+  constexpr int QB = Cfg::QBUF;
+  uint8_t* sQ = smem;                                         // QB buffers
+  uint8_t* sK = sQ + QB * Cfg::Q_BYTES;
   uint8_t* sV = sK + S * Cfg::KV_BYTES;
-  uint8_t* sP = sV + S * Cfg::KV_BYTES;
-  float* red = reinterpret_cast<float*>(sP + Cfg::P_BYTES);  // [2 tiles][2 halves][128], then [2 halves][128]
+  constexpr int PB = Cfg::PB;
+  uint8_t* sP = sV + S * Cfg::KV_BYTES;                       // PB tiles
+  float* red = reinterpret_cast<float*>(sP + PB * Cfg::P_BYTES);  // [2 tiles][2 halves][128], then [2 halves][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(red + 3 * 2 * 128);
-  // bars: kv_full[S], kv_empty[S], q_full, s_full[2], s_free[2], p_full, o_done, drain,
-  //       pair[4 quarters][2 tiles] (row-max exchange), fin[4] (row-sum exchange)
+  // bars: kv_full[S], kv_empty[S], q_full[2], q_empty[2], s_full[2], s_free[2], p_full[2], o_done[2],
+  //       o_free[2], drain, pair[4 quarters][2 tiles], fin[4]
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   volatile int* abort_flag = &s_abort;
@@ -170,37 +182,15 @@ __global__ void __launch_bounds__(384, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Ctl* ctl = g.ctl;
   const int R = ctl->R, p0 = ctl->p0;
-  const int qt = blockIdx.x, hh = blockIdx.y;
-  const int s = (int)blockIdx.z / g.nsplit, split = (int)blockIdx.z % g.nsplit;
-  const int q_begin = qt * BQ;
-  if (q_begin >= R) return;                                   // uniform over the CTA
-  const int q_end = min(q_begin + BQ, R);
-  const int kmax = p0 + q_end - 1;                            // last key any row needs
-  const int ntiles = kmax / BKV + 1;
-  const int t0 = split * g.tiles_per_split;
-  const int t1 = min(ntiles, t0 + g.tiles_per_split);
-  const int nt = t1 - t0;                                     // may be <= 0 for a split past the end
-  const int qpos_min = p0 + q_begin;
+  const int q_tiles = (R + BQ - 1) / BQ;
+  const int n_items = q_tiles * g.heads * g.batch * g.nsplit;
 
-  const uint32_t kvf0 = smem_u32(bars), kve0 = smem_u32(bars + S), q_full = smem_u32(bars + 2 * S);
-  const uint32_t sfull0 = smem_u32(bars + 2 * S + 1), sfree0 = smem_u32(bars + 2 * S + 3);
-  const uint32_t p_full = smem_u32(bars + 2 * S + 5), o_done = smem_u32(bars + 2 * S + 6);
-  const uint32_t drain = smem_u32(bars + 2 * S + 7);
-  const uint32_t pair0 = smem_u32(bars + 2 * S + 8), fin0 = smem_u32(bars + 2 * S + 16);
-
-  if (nt <= 0) {
-    // nothing to attend in this split: an empty partial (m = -inf, l = 0)
-    if (threadIdx.x < 128) {
-      const int r = q_begin + threadIdx.x;
-      if (r < R) {
-        const size_t row = (size_t)s * R + r;
-        float* ml = g.mlpart + (((size_t)split * g.m_max + row) * g.heads + hh) * 2;
-        ml[0] = -INFINITY;
-        ml[1] = 0.f;
-      }
-    }
-    return;
-  }
+  const uint32_t kvf0 = smem_u32(bars), kve0 = smem_u32(bars + S);
+  const uint32_t qf0 = smem_u32(bars + 2 * S), qe0 = smem_u32(bars + 2 * S + 2);
+  const uint32_t sfull0 = smem_u32(bars + 2 * S + 4), sfree0 = smem_u32(bars + 2 * S + 6);
+  const uint32_t pfull0 = smem_u32(bars + 2 * S + 8), odone0 = smem_u32(bars + 2 * S + 10);
+  const uint32_t ofree0 = smem_u32(bars + 2 * S + 12), drain = smem_u32(bars + 2 * S + 14);
+  const uint32_t pair0 = smem_u32(bars + 2 * S + 15), fin0 = smem_u32(bars + 2 * S + 23);
 
   if (threadIdx.x == 0) {
     s_abort = 0;
@@ -208,13 +198,15 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(kvf0 + 8 * i, 1);
       mbar_init(kve0 + 8 * i, 1);
     }
-    mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
+      mbar_init(qf0 + 8 * i, 1);
+      mbar_init(qe0 + 8 * i, 1);
       mbar_init(sfull0 + 8 * i, 1);
       mbar_init(sfree0 + 8 * i, 256);
+      mbar_init(ofree0 + 8 * i, 256);
+      mbar_init(pfull0 + 8 * i, 256);
+      mbar_init(odone0 + 8 * i, 1);
     }
-    mbar_init(p_full, 256);
-    mbar_init(o_done, 1);
     mbar_init(drain, 1);
     for (int i = 0; i < 8; ++i) mbar_init(pair0 + 8 * i, 64);
     for (int i = 0; i < 4; ++i) mbar_init(fin0 + 8 * i, 64);
@@ -228,69 +220,110 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  const uint32_t tS = tmem, tO = tmem + 2 * BKV;             // S buffers at 0 and 128, O at 256
+  const uint32_t tS = tmem, tO = tmem + 2 * BKV;              // S buffers at 0 and 128, O buffers at 256, 256 + hd
+
+  // Work item -> (query tile, head, sample, key split) and its key-tile range.
+  struct Item { int qt, hh, s, split, q_begin, t0, nt; };
+  auto item_of = [&](int it) {
+    Item x;
+    x.qt = it % q_tiles;
+    int r = it / q_tiles;
+    x.hh = r % g.heads;
+    r /= g.heads;
+    x.split = r % g.nsplit;
+    x.s = r / g.nsplit;
+    x.q_begin = x.qt * BQ;
+    const int q_end = min(x.q_begin + BQ, R);
+    const int ntiles = (p0 + q_end - 1) / BKV + 1;          // key tiles up to the last needed key
+    x.t0 = x.split * g.tiles_per_split;
+    x.nt = min(ntiles, x.t0 + g.tiles_per_split) - x.t0;
+    return x;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------------ TMA producer
-      mbar_expect_tx(q_full, Cfg::Q_BYTES);
-#pragma unroll
-      for (int kc = 0; kc < Cfg::KCH; ++kc)
-        tma_load_2d(smem_u32(sQ + kc * Cfg::BOX), &tmQ, q_full, hh * HD + kc * 64, s * R + q_begin);
       int stage = 0;
       uint32_t phase = 0;
-      for (int j = 0; j < nt; ++j) {
-        if (!mbar_wait(kve0 + 8 * stage, phase ^ 1u, abort_flag)) break;
-        mbar_expect_tx(kvf0 + 8 * stage, 2 * Cfg::KV_BYTES);
-        const int key0 = (t0 + j) * BKV;
+      int gi = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+        const Item x = item_of(it);
+        if (x.nt <= 0) continue;
+        const int qb = gi % QB;
+        if (gi >= QB && !mbar_wait(qe0 + 8 * qb, (uint32_t)(((gi - QB) / QB) & 1), abort_flag)) break;
+        mbar_expect_tx(qf0 + 8 * qb, Cfg::Q_BYTES);
 #pragma unroll
-        for (int kc = 0; kc < Cfg::KCH; ++kc) {
-          tma_load_2d(smem_u32(sK + stage * Cfg::KV_BYTES + kc * Cfg::BOX), &tmK, kvf0 + 8 * stage,
-                      hh * HD + kc * 64, s * g.Lc + key0);
-          tma_load_2d(smem_u32(sV + stage * Cfg::KV_BYTES + kc * Cfg::BOX), &tmV, kvf0 + 8 * stage,
-                      hh * HD + kc * 64, s * g.Lc + key0);
+        for (int kc = 0; kc < Cfg::KCH; ++kc)
+          tma_load_2d(smem_u32(sQ + qb * Cfg::Q_BYTES + kc * Cfg::BOX), &tmQ, qf0 + 8 * qb, x.hh * HD + kc * 64,
+                      x.s * R + x.q_begin);
+        for (int j = 0; j < x.nt; ++j) {
+          if (!mbar_wait(kve0 + 8 * stage, phase ^ 1u, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(kvf0 + 8 * stage, 2 * Cfg::KV_BYTES);
+          const int key0 = (x.t0 + j) * BKV;
+#pragma unroll
+          for (int kc = 0; kc < Cfg::KCH; ++kc) {
+            tma_load_2d(smem_u32(sK + stage * Cfg::KV_BYTES + kc * Cfg::BOX), &tmK, kvf0 + 8 * stage,
+                        x.hh * HD + kc * 64, x.s * g.Lc + key0);
+            tma_load_2d(smem_u32(sV + stage * Cfg::KV_BYTES + kc * Cfg::BOX), &tmV, kvf0 + 8 * stage,
+                        x.hh * HD + kc * 64, x.s * g.Lc + key0);
+          }
+          if (++stage == S) { stage = 0; phase ^= 1u; }
         }
-        if (++stage == S) { stage = 0; phase ^= 1u; }
+        ++gi;
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------------ MMA issuer
-      bool ok = mbar_wait(q_full, 0, abort_flag);
-      tc_fence_after();
       int stage = 0, pstage = 0;
-      uint32_t phase = 0, pphase = 0;
-      auto issue_pv = [&](int j) -> bool {       // O += P_j V_j
-        if (!mbar_wait(p_full, (uint32_t)(j & 1), abort_flag)) return false;
+      uint32_t phase = 0;
+      int gt = 0, gi = 0;                                     // global tile and item counters
+      bool ok = true;
+      for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+        const Item x = item_of(it);
+        if (x.nt <= 0) continue;
+        const int qb = gi % QB, ob = gi & 1;
+        if (!mbar_wait(qf0 + 8 * qb, (uint32_t)((gi / QB) & 1), abort_flag)) break;
+        if (gi >= 2 && !mbar_wait(ofree0 + 8 * ob, (uint32_t)(((gi - 2) >> 1) & 1), abort_flag)) break;
         tc_fence_after();
+        const uint32_t dO = tO + ob * HD;
+        auto issue_pv = [&](int j, int gtile) -> bool {       // O += P_j V_j
+          const int pb = gtile % PB;
+          if (!mbar_wait(pfull0 + 8 * pb, (uint32_t)((gtile / PB) & 1), abort_flag)) return false;
+          tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < BKV / 16; ++ks) {
-          const uint64_t da = desc_k(smem_u32(sP + (ks >> 2) * Cfg::BOX + (ks & 3) * 32));
-          const uint64_t db = desc_mn(smem_u32(sV + pstage * Cfg::KV_BYTES + ks * 16 * 128), Cfg::BOX);
-          umma(tO, da, db, Cfg::IDESC_O, (j > 0 || ks > 0) ? 1u : 0u);
-        }
-        umma_commit(o_done);
-        umma_commit(kve0 + 8 * pstage);
-        if (++pstage == S) { pstage = 0; pphase ^= 1u; }
-        return true;
-      };
-      for (int j = 0; ok && j < nt; ++j) {
-        if (!mbar_wait(kvf0 + 8 * stage, phase, abort_flag)) { ok = false; break; }
-        const int b = j & 1;
-        if (j >= 2 && !mbar_wait(sfree0 + 8 * b, (uint32_t)(((j - 2) >> 1) & 1), abort_flag)) { ok = false; break; }
-        tc_fence_after();
+          for (int ks = 0; ks < BKV / 16; ++ks) {
+            const uint64_t da = desc_k(smem_u32(sP + pb * Cfg::P_BYTES + (ks >> 2) * Cfg::BOX + (ks & 3) * 32));
+            const uint64_t db = desc_mn(smem_u32(sV + pstage * Cfg::KV_BYTES + ks * 16 * 128), Cfg::BOX);
+            umma(dO, da, db, Cfg::IDESC_O, (j > 0 || ks > 0) ? 1u : 0u);
+          }
+          umma_commit(odone0 + 8 * pb);
+          umma_commit(kve0 + 8 * pstage);
+          if (++pstage == S) pstage = 0;
+          return true;
+        };
+        for (int j = 0; j < x.nt; ++j) {
+          const int gtile = gt + j;
+          if (!mbar_wait(kvf0 + 8 * stage, phase, abort_flag)) { ok = false; break; }
+          const int b = gtile & 1;
+          if (gtile >= 2 && !mbar_wait(sfree0 + 8 * b, (uint32_t)(((gtile - 2) >> 1) & 1), abort_flag)) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < HD / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * Cfg::BOX + (ks & 3) * 32;
-          umma(tS + b * BKV, desc_k(smem_u32(sQ + off)), desc_k(smem_u32(sK + stage * Cfg::KV_BYTES + off)),
-               Cfg::IDESC_S, ks > 0 ? 1u : 0u);
+          for (int ks = 0; ks < HD / 16; ++ks) {
+            const uint32_t off = (ks >> 2) * Cfg::BOX + (ks & 3) * 32;
+            umma(tS + b * BKV, desc_k(smem_u32(sQ + qb * Cfg::Q_BYTES + off)),
+                 desc_k(smem_u32(sK + stage * Cfg::KV_BYTES + off)), Cfg::IDESC_S, ks > 0 ? 1u : 0u);
+          }
+          umma_commit(sfull0 + 8 * b);
+          if (j == x.nt - 1) umma_commit(qe0 + 8 * qb);       // the item's Q is no longer read
+          if (++stage == S) { stage = 0; phase ^= 1u; }
+          if (j >= 1 && !issue_pv(j - 1, gtile - 1)) { ok = false; break; }
         }
-        umma_commit(sfull0 + 8 * b);
-        if (++stage == S) { stage = 0; phase ^= 1u; }
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        if (!ok || !issue_pv(x.nt - 1, gt + x.nt - 1)) break;
+        gt += x.nt;
+        ++gi;
       }
-      if (ok) issue_pv(nt - 1);
-      (void)pphase;
       umma_commit(drain);
       const uint64_t tw = globaltimer_ns();
       while (!mbar_try(drain, 0)) {
@@ -301,125 +334,160 @@ __global__ void __launch_bounds__(384, 1)
     // -------------------------------------------------------------------- softmax
     const int ew = warp - 4;
     const int q = ew & 3, hf = ew >> 2;
-    const int row = q * 32 + lane;                            // 0..127 within the tile
-    const int qpos = p0 + q_begin + row;
+    const int row = q * 32 + lane;                            // 0..127 within the query tile
     const float sl2 = 1.4426950408889634f / sqrtf((float)HD);
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    float m_use = -INFINITY, l = 0.f;
-    int j = 0;
-    for (; j < nt; ++j) {
-      const int b = j & 1;
-      // every wait's outcome is made warp-uniform before any .aligned TMEM access
-      if (!__all_sync(0xffffffffu, mbar_wait(sfull0 + 8 * b, (uint32_t)((j >> 1) & 1), abort_flag))) break;
-      tc_fence_after();
-      const int key0 = (t0 + j) * BKV + hf * 64;
-      const bool need_mask = (t0 + j) * BKV + BKV - 1 > qpos_min;
-      const uint32_t sa = tS + b * BKV + hf * 64 + lane_off;
-      // pass 1: row max of the scaled scores t = s * log2(e) / sqrt(hd)
-      float mx = -INFINITY;
+    int gt = 0, gi = 0;
+    bool alive = true;
+    for (int it = blockIdx.x; alive && it < n_items; it += gridDim.x) {
+      const Item x = item_of(it);
+      const int rloc = x.q_begin + row;
+      const size_t mrow = (size_t)x.s * R + rloc;
+      if (x.nt <= 0) {
+        // nothing to attend in this split: an empty partial (m = -inf, l = 0)
+        if (hf == 0 && rloc < R) {
+          float* ml = g.mlpart + (((size_t)x.split * g.m_max + mrow) * g.heads + x.hh) * 2;
+          ml[0] = -INFINITY;
+          ml[1] = 0.f;
+        }
+        continue;
+      }
+      const int qpos = p0 + rloc;
+      const int qpos_min = p0 + x.q_begin;
+      const int ob = gi & 1;
+      float m_use = -INFINITY, l = 0.f;
+      int j = 0;
+      for (; j < x.nt; ++j) {
+        const int gtile = gt + j;
+        const int b = gtile & 1;
+        // every wait's outcome is made warp-uniform before any .aligned TMEM access
+        if (!__all_sync(0xffffffffu, mbar_wait(sfull0 + 8 * b, (uint32_t)((gtile >> 1) & 1), abort_flag))) break;
+        tc_fence_after();
+        const int key0 = (x.t0 + j) * BKV + hf * 64;
+        const bool need_mask = (x.t0 + j) * BKV + BKV - 1 > qpos_min;
+        const uint32_t sa = tS + b * BKV + hf * 64 + lane_off;
+        // pass 1: row max.  The scores stay in registers for pass 2; the max is
+        // taken on raw scores and scaled once (the scale is positive).
+        float v[64];
 #pragma unroll
-      for (int c = 0; c < 64; c += 16) {
-        float v[16];
-        tmem_ld16(sa + c, v);
+        for (int c = 0; c < 64; c += 16) tmem_ld16(sa + c, v + c);
         tmem_wait_ld();
+        float mraw = -INFINITY;
+        if (need_mask) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float t = (need_mask && key0 + c + i > qpos) ? -INFINITY : v[i] * sl2;
-          mx = fmaxf(mx, t);
+          for (int i = 0; i < 64; ++i)
+            if (key0 + i <= qpos) mraw = fmaxf(mraw, v[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) mraw = fmaxf(mraw, v[i]);
         }
+        float mx = mraw * sl2;
+        float* rd = red + (b * 2) * 128;
+        rd[hf * 128 + row] = mx;
+        mbar_arrive(pair0 + 8 * (q * 2 + b));
+        if (!__all_sync(0xffffffffu, mbar_wait(pair0 + 8 * (q * 2 + b), (uint32_t)((gtile >> 1) & 1), abort_flag))) break;
+        mx = fmaxf(mx, rd[(1 - hf) * 128 + row]);
+        const float m_new = fmaxf(m_use, mx);
+        // raise the running max lazily; rows decide alone, the TMEM rescale of O
+        // runs for the whole warp when any of its rows needs it (factor 1 for the rest)
+        float corr = 1.f;
+        if (m_new > m_use + kRescaleLog2 || m_use == -INFINITY) {
+          if (m_use != -INFINITY) corr = exp2f(m_use - m_new);
+          l *= corr;
+          m_use = m_new;
+        }
+        if (j >= 1 && __any_sync(0xffffffffu, corr != 1.f)) {
+          // O holds tiles 0..j-1: wait for P_{j-1} V_{j-1}
+          const int gp = gtile - 1;
+          if (!__all_sync(0xffffffffu, mbar_wait(odone0 + 8 * (gp % PB), (uint32_t)((gp / PB) & 1), abort_flag))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < HD / 2; c += 16) {
+            float v[16];
+            const uint32_t oa = tO + ob * HD + hf * (HD / 2) + c + lane_off;
+            tmem_ld16(oa, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] *= corr;
+            tmem_st16(oa, v);
+          }
+          tmem_wait_st();
+        }
+        // the P tile this tile writes was last read by tile gtile - PB
+        const int pb = gtile % PB;
+        if (gtile >= PB &&
+            !__all_sync(0xffffffffu, mbar_wait(odone0 + 8 * pb, (uint32_t)(((gtile - PB) / PB) & 1), abort_flag)))
+          break;
+        // pass 2: P = 2^(s * scale - m) in bf16 into the swizzled P tile, row sums;
+        // masked keys are exactly 0
+        const float nmb = (m_use == -INFINITY) ? 0.f : -m_use;
+        uint8_t* prow = sP + pb * Cfg::P_BYTES + hf * Cfg::BOX + row * 128;
+#pragma unroll
+        for (int c = 0; c < 64; c += 16) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int i = 0; i < 16; i += 2) {
+            float e0 = ex2_approx(fmaf(v[c + i], sl2, nmb));
+            float e1 = ex2_approx(fmaf(v[c + i + 1], sl2, nmb));
+            if (need_mask) {
+              if (key0 + c + i > qpos) e0 = 0.f;
+              if (key0 + c + i + 1 > qpos) e1 = 0.f;
+            }
+            l += e0 + e1;
+            pk[i >> 1] = pack_bf16(e0, e1);
+          }
+          const int u0 = c >> 3;                             // 16-byte units u0, u0+1 of this row
+          *reinterpret_cast<uint4*>(prow + (((u0) ^ (row & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(prow + (((u0 + 1) ^ (row & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc_fence_before();
+        mbar_arrive(pfull0 + 8 * pb);
+        mbar_arrive(sfree0 + 8 * b);
       }
-      float* rd = red + (b * 2) * 128;
-      rd[hf * 128 + row] = mx;
-      mbar_arrive(pair0 + 8 * (q * 2 + b));
-      if (!__all_sync(0xffffffffu, mbar_wait(pair0 + 8 * (q * 2 + b), (uint32_t)((j >> 1) & 1), abort_flag))) break;
-      mx = fmaxf(mx, rd[(1 - hf) * 128 + row]);
-      const float m_new = fmaxf(m_use, mx);
-      // O_{j-1} complete: the P tile is free and O may be rescaled
-      if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait(o_done, (uint32_t)((j - 1) & 1), abort_flag))) break;
+      // item epilogue: wait for its last O, combine the halves' row sums, write out
+      const int glast = gt + x.nt - 1;
+      const bool ok = __all_sync(0xffffffffu, (j == x.nt) && mbar_wait(odone0 + 8 * (glast % PB),
+                                                                        (uint32_t)((glast / PB) & 1), abort_flag));
       tc_fence_after();
-      // raise the running max lazily; rows decide alone, the TMEM rescale of O
-      // runs for the whole warp when any of its rows needs it (factor 1 for the rest)
-      float corr = 1.f;
-      if (m_new > m_use + kRescaleLog2 || m_use == -INFINITY) {
-        if (m_use != -INFINITY) corr = exp2f(m_use - m_new);
-        l *= corr;
-        m_use = m_new;
-      }
-      if (j >= 1 && __any_sync(0xffffffffu, corr != 1.f)) {
+      float* rl = red + 4 * 128;                               // past both row-max slots
+      rl[hf * 128 + row] = l;
+      mbar_arrive(fin0 + 8 * q);
+      const bool ok2 = __all_sync(0xffffffffu, mbar_wait(fin0 + 8 * q, (uint32_t)(gi & 1), abort_flag));
+      const float lt = l + rl[(1 - hf) * 128 + row];
+      const bool valid = ok && ok2 && rloc < R;
 #pragma unroll
-        for (int c = 0; c < HD / 2; c += 16) {
-          float v[16];
-          const uint32_t oa = tO + hf * (HD / 2) + c + lane_off;
-          tmem_ld16(oa, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] *= corr;
-          tmem_st16(oa, v);
-        }
-        tmem_wait_st();
-      }
-      // pass 2: P = exp2(t - m) in bf16 into the swizzled P tile, row sums
-      const float mb = (m_use == -INFINITY) ? 0.f : m_use;
-      uint8_t* prow = sP + hf * Cfg::BOX + row * 128;
-#pragma unroll
-      for (int c = 0; c < 64; c += 16) {
+      for (int c = 0; c < HD / 2; c += 16) {
         float v[16];
-        tmem_ld16(sa + c, v);
+        tmem_ld16(tO + ob * HD + hf * (HD / 2) + c + lane_off, v);
         tmem_wait_ld();
-        uint32_t pk[8];
+        const int col = x.hh * HD + hf * (HD / 2) + c;
+        if (!valid) continue;
+        if (g.nsplit == 1) {
+          const float inv = 1.f / lt;
+          uint32_t pk[8];
 #pragma unroll
-        for (int i = 0; i < 16; i += 2) {
-          const float t0v = (need_mask && key0 + c + i > qpos) ? -INFINITY : v[i] * sl2;
-          const float t1v = (need_mask && key0 + c + i + 1 > qpos) ? -INFINITY : v[i + 1] * sl2;
-          const float e0 = exp2f(t0v - mb), e1 = exp2f(t1v - mb);
-          l += e0 + e1;
-          pk[i >> 1] = pack_bf16(e0, e1);
+          for (int i = 0; i < 16; i += 2) pk[i >> 1] = pack_bf16(v[i] * inv, v[i + 1] * inv);
+          uint4* dst = reinterpret_cast<uint4*>(g.o + mrow * g.d + col);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        } else {
+          float4* dst = reinterpret_cast<float4*>(g.opart + ((size_t)x.split * g.m_max + mrow) * g.d + col);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
         }
-        const int u0 = c >> 3;                               // 16-byte units u0, u0+1 of this row
-        *reinterpret_cast<uint4*>(prow + (((u0) ^ (row & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        *reinterpret_cast<uint4*>(prow + (((u0 + 1) ^ (row & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      if (valid && g.nsplit > 1 && hf == 0) {
+        float* ml = g.mlpart + (((size_t)x.split * g.m_max + mrow) * g.heads + x.hh) * 2;
+        ml[0] = m_use;
+        ml[1] = lt;
+      }
+      // the O buffer and the row-sum slots are free for the item after next
       tc_fence_before();
-      mbar_arrive(p_full);
-      mbar_arrive(sfree0 + 8 * b);
-    }
-    // epilogue: wait for the last O, combine the halves' row sums, write out
-    const bool ok = __all_sync(0xffffffffu, (j == nt) && mbar_wait(o_done, (uint32_t)((nt - 1) & 1), abort_flag));
-    tc_fence_after();
-    float* rl = red + 4 * 128;                               // past both row-max slots
-    rl[hf * 128 + row] = l;
-    mbar_arrive(fin0 + 8 * q);
-    const bool ok2 = __all_sync(0xffffffffu, mbar_wait(fin0 + 8 * q, 0, abort_flag));
-    const float lt = l + rl[(1 - hf) * 128 + row];
-    const int rloc = q_begin + row;
-    const bool valid = ok && ok2 && rloc < R;
-    const size_t mrow = (size_t)s * R + rloc;
-#pragma unroll
-    for (int c = 0; c < HD / 2; c += 16) {
-      float v[16];
-      tmem_ld16(tO + hf * (HD / 2) + c + lane_off, v);
-      tmem_wait_ld();
-      const int col = hh * HD + hf * (HD / 2) + c;
-      if (!valid) continue;
-      if (g.nsplit == 1) {
-        const float inv = 1.f / lt;
-        uint32_t pk[8];
-#pragma unroll
-        for (int i = 0; i < 16; i += 2) pk[i >> 1] = pack_bf16(v[i] * inv, v[i + 1] * inv);
-        uint4* dst = reinterpret_cast<uint4*>(g.o + mrow * g.d + col);
-        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-      } else {
-        float4* dst = reinterpret_cast<float4*>(g.opart + ((size_t)split * g.m_max + mrow) * g.d + col);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-      }
-    }
-    if (valid && g.nsplit > 1 && hf == 0) {
-      float* ml = g.mlpart + (((size_t)split * g.m_max + mrow) * g.heads + hh) * 2;
-      ml[0] = m_use;
-      ml[1] = lt;
+      mbar_arrive(ofree0 + 8 * ob);
+      alive = ok && ok2;
+      gt += x.nt;
+      ++gi;
     }
   }
   tc_fence_before();
@@ -468,7 +536,14 @@ void launch_hd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
     cudaFuncSetAttribute(k_attn_tc<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM);
     attr = true;
   }
-  dim3 grid((r_max + BQ - 1) / BQ, g.heads, batch * g.nsplit);
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  const long long items = (long long)((r_max + BQ - 1) / BQ) * g.heads * batch * g.nsplit;
+  const int grid = (int)(items < sms ? items : sms);
   k_attn_tc<HD><<<grid, 384, Cfg::SMEM, st>>>(tq, tk, tv, g, err);
   if (g.nsplit > 1) {
     const long long warps = (long long)g.m_max * g.heads;
@@ -508,6 +583,7 @@ bool launch_attn_tc2(const Ctl* ctl, const bf16* q, const bf16* kc, const bf16* 
   const int key_tiles = (Lc + BKV - 1) / BKV;
   g.tiles_per_split = (key_tiles + nsplit - 1) / nsplit;
   g.m_max = m_max;
+  g.batch = batch;
   if (d / heads == 64) launch_hd<64>(tq, tk, tv, g, batch, r_max, err, st);
   else launch_hd<128>(tq, tk, tv, g, batch, r_max, err, st);
   return true;

@@ -28,6 +28,7 @@ struct Ctl {
   int iter;       // updates computed so far in this block
   int n_active;   // samples still iterating in this block
   int nonconv;    // (sample, block) pairs that stopped at max_iter unconverged
+  int done;       // CTAs of the current Jacobi step that finished their sample
 };
 
 // Error codes written to the model's device error word.

@@ -166,19 +166,57 @@ __device__ __forceinline__ void umma_commit_pair_local(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
-// GELU with erf from Abramowitz & Stegun, Handbook of Mathematical Functions,
-// formula 7.1.26 (Hastings): erf(u) = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5))))
-// exp(-u^2), t = 1 / (1 + p u), u >= 0, |error| <= 1.5e-7 -- far below the bf16
-// rounding of the MLP activations it feeds.  The fp32 SIMT path keeps erff.
-__device__ __forceinline__ float gelu_as7126(float v) {
-  const float u = fabsf(v) * 0.70710678118654752f;
-  const float t = __fdividef(1.0f, fmaf(0.3275911f, u, 1.0f));
-  float q = fmaf(t, 1.061405429f, -1.453152027f);
-  q = fmaf(t, q, 1.421413741f);
-  q = fmaf(t, q, -0.284496736f);
-  q = fmaf(t, q, 0.254829592f);
-  const float erf_abs = 1.0f - q * t * __expf(-u * u);
-  return 0.5f * v * (1.0f + copysignf(erf_abs, v));
+// Packed fp32x2 arithmetic of sm_100 (two lanes of one 64-bit register).
+__device__ __forceinline__ uint64_t u64_of(float2 v) { return *reinterpret_cast<uint64_t*>(&v); }
+__device__ __forceinline__ float2 f2_of(uint64_t v) { return *reinterpret_cast<float2*>(&v); }
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(u64_of(a)), "l"(u64_of(b)), "l"(u64_of(c)));
+  return f2_of(d);
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(u64_of(a)), "l"(u64_of(b)));
+  return f2_of(d);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(u64_of(a)), "l"(u64_of(b)));
+  return f2_of(d);
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float2 splat(float a) { return make_float2(a, a); }
+
+// GELU of two values, with erf from Abramowitz & Stegun, Handbook of
+// Mathematical Functions, formula 7.1.26 (Hastings):
+// erf(u) = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-u^2), t = 1 / (1 + p u),
+// u >= 0, |error| <= 1.5e-7 -- far below the bf16 rounding of the MLP
+// activations it feeds.  GELU(v) = v/2 + (v/2) sign(v) erf(|v| / sqrt 2).
+// The fp32 SIMT path keeps erff.
+__device__ __forceinline__ float2 gelu2_as7126(float2 v) {
+  const float2 u = fmul2(make_float2(fabsf(v.x), fabsf(v.y)), splat(0.70710678118654752f));
+  const float2 den = ffma2(u, splat(0.3275911f), splat(1.0f));
+  const float2 t = make_float2(rcp_approx(den.x), rcp_approx(den.y));
+  float2 q = ffma2(t, splat(1.061405429f), splat(-1.453152027f));
+  q = ffma2(t, q, splat(1.421413741f));
+  q = ffma2(t, q, splat(-0.284496736f));
+  q = ffma2(t, q, splat(0.254829592f));
+  q = fmul2(q, t);
+  const float2 w = fmul2(fmul2(u, u), splat(-1.4426950408889634f));   // -u^2 log2(e)
+  const float2 e = make_float2(ex2_approx(w.x), ex2_approx(w.y));
+  const float2 erf_abs = ffma2(fmul2(q, e), splat(-1.0f), splat(1.0f));
+  const float2 erf_s = make_float2(copysignf(erf_abs.x, v.x), copysignf(erf_abs.y, v.y));
+  const float2 hv = fmul2(v, splat(0.5f));
+  return ffma2(hv, erf_s, hv);
 }
 
 __device__ __forceinline__ void st_bf16x4(bf16* dst, float a, float b, float c, float d) {
@@ -388,6 +426,22 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
+      // head: one row per thread, hoisted (sample, position, token) and row pointers
+      bool head_out = false, head_act = false;
+      const float* hin = nullptr;
+      float* hout = nullptr;
+      float* hpart = nullptr;
+      if (EPI == EPI_HEAD) {
+        const int r = row0 + lane;
+        const int sm = r / R;
+        const int p = p0 + (r - sm * R);
+        head_out = r < M && p >= ctl->P;
+        const size_t base = ((size_t)sm * e.L + tok_of(p, e.L, e.dir)) * e.C;
+        hin = e.xin_f + base;
+        hout = e.xout_f + base;
+        hpart = e.part + (size_t)r * ((2 * e.C) >> 4) * 2;
+        head_act = head_out && (e.head_mode == 0 || e.active[sm]);
+      }
       // Loads that do not depend on the accumulator are issued before waiting
       // for it (bias, and the first chunk's residual / position rows), and
       // every chunk's TMEM load and global loads are in flight while the
@@ -398,6 +452,18 @@ __global__ void __launch_bounds__(384, 1)
       for (int k = 0; k < NCH; ++k) bias4[k] = *reinterpret_cast<const float4*>(e.bias + n0 + k * 16 + cq * 4);
       float4 pre[2][4], pre2[2][4];
       auto load_rows = [&](int k, float4* dst, float4* dst2) {
+        if (EPI == EPI_HEAD) {
+          if (head_act) {
+            const int c0 = (n0 + k * 16) >> 1;
+            dst[0] = *reinterpret_cast<const float4*>(hin + c0);
+            dst[1] = *reinterpret_cast<const float4*>(hin + c0 + 4);
+            if (e.head_mode == 1) {
+              dst2[0] = *reinterpret_cast<const float4*>(hout + c0);
+              dst2[1] = *reinterpret_cast<const float4*>(hout + c0 + 4);
+            }
+          }
+          return;
+        }
         const int col = n0 + k * 16 + cq * 4;
 #pragma unroll
         for (int it = 0; it < 4; ++it) {
@@ -410,7 +476,7 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       };
-      if (EPI == EPI_RESID || EPI == EPI_INPROJ) load_rows(0, pre[0], pre2[0]);
+      if (EPI == EPI_RESID || EPI == EPI_INPROJ || EPI == EPI_HEAD) load_rows(0, pre[0], pre2[0]);
       // the wait's outcome is made warp-uniform before the .aligned TMEM loads
       if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * acc, use & 1u, abort_flag))) break;
       tc_fence_after();
@@ -422,11 +488,36 @@ __global__ void __launch_bounds__(384, 1)
         tmem_wait_ld();
         if (k + 1 < NCH) {
           tmem_ld16(taddr + c + 16, vb[(k + 1) & 1]);
-          if (EPI == EPI_RESID || EPI == EPI_INPROJ) load_rows(k + 1, pre[(k + 1) & 1], pre2[(k + 1) & 1]);
+          if (EPI == EPI_RESID || EPI == EPI_INPROJ || EPI == EPI_HEAD) load_rows(k + 1, pre[(k + 1) & 1], pre2[(k + 1) & 1]);
         }
         const float* v = vb[k & 1];
         if (EPI == EPI_HEAD) {
-          if (row0 + lane < M) head_group(e, row0 + lane, n0 + c, v);
+          // 8 channels whose (mu_c, s_c) sit at columns (2c, 2c+1)
+          const int col0 = n0 + c;
+          float2* part = reinterpret_cast<float2*>(hpart) + (col0 >> 4);
+          if (!head_out) continue;
+          if (!head_act) { *part = make_float2(0.f, 0.f); continue; }
+          const float* xi = reinterpret_cast<const float*>(pre[k & 1]);
+          float r8[8];
+          float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            const float mu = v[2 * jj] + e.bias[col0 + 2 * jj];
+            const float sl = v[2 * jj + 1] + e.bias[col0 + 2 * jj + 1];
+            if (e.head_mode == 0) {
+              r8[jj] = (xi[jj] - mu) * expf(-sl);            // z = (x - mu) exp(-s)
+              a0 += sl;
+            } else {
+              r8[jj] = fmaf(expf(sl), xi[jj], mu);           // x_new = mu + exp(s) z
+              const float dx = r8[jj] - reinterpret_cast<const float*>(pre2[k & 1])[jj];
+              a0 = fmaf(dx, dx, a0);
+              a1 = fmaf(r8[jj], r8[jj], a1);
+            }
+          }
+          const int c0 = col0 >> 1;
+          *reinterpret_cast<float4*>(hout + c0) = make_float4(r8[0], r8[1], r8[2], r8[3]);
+          *reinterpret_cast<float4*>(hout + c0 + 4) = make_float4(r8[4], r8[5], r8[6], r8[7]);
+          *part = make_float2(a0, a1);
           continue;
         }
         float4* srow = reinterpret_cast<float4*>(stg + lane * 16);
@@ -461,10 +552,13 @@ __global__ void __launch_bounds__(384, 1)
           }
         } else if (EPI == EPI_GELU) {
 #pragma unroll
-          for (int it = 0; it < 4; ++it)
-            if (row0 + it * 8 + rl < M)
-              st_bf16x4(reinterpret_cast<bf16*>(rowp[it]) + col, gelu_as7126(a[it].x + bb.x),
-                        gelu_as7126(a[it].y + bb.y), gelu_as7126(a[it].z + bb.z), gelu_as7126(a[it].w + bb.w));
+          for (int it = 0; it < 4; ++it) {
+            if (row0 + it * 8 + rl < M) {
+              const float2 g0 = gelu2_as7126(fadd2(make_float2(a[it].x, a[it].y), make_float2(bb.x, bb.y)));
+              const float2 g1 = gelu2_as7126(fadd2(make_float2(a[it].z, a[it].w), make_float2(bb.z, bb.w)));
+              st_bf16x4(reinterpret_cast<bf16*>(rowp[it]) + col, g0.x, g0.y, g1.x, g1.y);
+            }
+          }
         } else if (EPI == EPI_QKV) {
 #pragma unroll
           for (int it = 0; it < 4; ++it)

@@ -96,42 +96,49 @@ __global__ void k_block_init(Ctl* ctl, int* active, const float* __restrict__ z,
       ctl->M = batch * (P + B - p0);
       ctl->iter = 0;
       ctl->n_active = batch;
+      ctl->done = 0;
       cudaGraphSetConditional(inner, 1u);
     }
   }
 }
 
 // End of one Jacobi update: per-sample residual from the head's partial sums
-// (fixed summation order), the stopping test, the iteration counters and the
-// inner loop condition.  One block of 1024 threads; one warp per sample.
-__global__ void __launch_bounds__(1024) k_jacobi_step(Ctl* ctl, int* active, const float* __restrict__ part,
-                                                      int batch, int B, int G, float tau, int max_iter,
-                                                      int32_t* iters, int nblocks,
-                                                      cudaGraphConditionalHandle inner) {
+// (one CTA per sample, fixed summation order), the stopping test, the
+// iteration counters; the last CTA to finish sets the inner loop condition.
+__global__ void __launch_bounds__(512) k_jacobi_step(Ctl* ctl, int* active, const float* __restrict__ part,
+                                                     int batch, int B, int G, float tau, int max_iter,
+                                                     int32_t* iters, int nblocks,
+                                                     cudaGraphConditionalHandle inner) {
+  __shared__ int s_last;
+  const int s = blockIdx.x;
   const int R = ctl->R, p0 = ctl->p0, P = ctl->P, iter = ctl->iter, blk = ctl->block;
-  const int skip = P - p0;
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  for (int s = w; s < batch; s += nw) {
-    if (!active[s]) continue;
-    const float* p = part + ((size_t)s * R + skip) * G * 2;
+  if (active[s]) {                                     // uniform over the CTA
+    const float2* p = reinterpret_cast<const float2*>(part + ((size_t)s * R + (P - p0)) * G * 2);
     const int n = B * G;
     float num = 0.f, den = 0.f;
-    for (int i = lane; i < n; i += 32) {
-      num += p[2 * i];
-      den += p[2 * i + 1];
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const float2 v = p[i];
+      num += v.x;
+      den += v.y;
     }
-    num = warp_sum(num);
-    den = warp_sum(den);
-    if (lane == 0) {
+    num = block_sum(num);
+    den = block_sum(den);
+    if (threadIdx.x == 0) {
       iters[(size_t)s * nblocks + blk] = iter + 1;
       const bool conv = (den == 0.f) ? (num == 0.f) : (num / den < tau);
       if (conv) active[s] = 0;
     }
   }
-  __syncthreads();
   if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(&ctl->done, 1) == batch - 1;
+  }
+  __syncthreads();
+  if (s_last && threadIdx.x == 0) {
+    __threadfence();
     int na = 0;
-    for (int s = 0; s < batch; ++s) na += active[s];
+    for (int i = 0; i < batch; ++i) na += *((volatile int*)active + i);
+    ctl->done = 0;
     ctl->iter = iter + 1;
     ctl->n_active = na;
     const bool cont = na > 0 && iter + 1 < max_iter;
@@ -170,37 +177,48 @@ __global__ void k_gather(const Ctl* ctl, const float* __restrict__ x, int L, int
   }
 }
 
-// LayerNorm (eps 1e-5), one warp per row, fp32 statistics (two passes over
-// registers: mean, then the centred variance).  NV = d / 128 float4 per lane.
+// LayerNorm (eps 1e-5), one warp per two rows, fp32 statistics (two passes
+// over registers: mean, then the centred variance).  NV = d / 128 float4 per
+// lane and row; both rows' loads are issued before any arithmetic.
 template <typename T, int NV>
-__global__ void k_layernorm_reg(const Ctl* ctl, const float* __restrict__ h, const float* __restrict__ g,
-                                const float* __restrict__ b, T* out, int d) {
-  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (row >= ctl->M) return;
-  const float4* hr = reinterpret_cast<const float4*>(h + (size_t)row * d);
-  float4 v[NV];
-  float sum = 0.f;
+__global__ void __launch_bounds__(256) k_layernorm_reg(const Ctl* ctl, const float* __restrict__ h,
+                                                       const float* __restrict__ g, const float* __restrict__ b,
+                                                       T* out, int d) {
+  const int wg = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  const int M = ctl->M;
+  const int r0 = 2 * wg;
+  if (r0 >= M) return;
+  const bool two = r0 + 1 < M;
+  float4 v[2][NV];
 #pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    v[i] = hr[lane + 32 * i];
-    sum += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+  for (int k = 0; k < 2; ++k) {
+    const float4* hr = reinterpret_cast<const float4*>(h + (size_t)(two ? r0 + k : r0) * d);
+#pragma unroll
+    for (int i = 0; i < NV; ++i) v[k][i] = hr[lane + 32 * i];
   }
-  const float mean = warp_sum(sum) / d;
-  float sq = 0.f;
 #pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const float a = v[i].x - mean, bb = v[i].y - mean, c = v[i].z - mean, e = v[i].w - mean;
-    sq += (a * a + bb * bb) + (c * c + e * e);
-  }
-  const float rstd = 1.0f / sqrtf(warp_sum(sq) / d + 1e-5f);
+  for (int k = 0; k < 2; ++k) {
+    if (k == 1 && !two) break;
+    float sum = 0.f;
 #pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int c = (lane + 32 * i) * 4;
-    const float4 gg = *reinterpret_cast<const float4*>(g + c);
-    const float4 bv = *reinterpret_cast<const float4*>(b + c);
-    store4(out + (size_t)row * d + c, (v[i].x - mean) * rstd * gg.x + bv.x,
-           (v[i].y - mean) * rstd * gg.y + bv.y, (v[i].z - mean) * rstd * gg.z + bv.z,
-           (v[i].w - mean) * rstd * gg.w + bv.w);
+    for (int i = 0; i < NV; ++i) sum += (v[k][i].x + v[k][i].y) + (v[k][i].z + v[k][i].w);
+    const float mean = warp_sum(sum) / d;
+    float sq = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const float a = v[k][i].x - mean, bb = v[k][i].y - mean, c = v[k][i].z - mean, e = v[k][i].w - mean;
+      sq += (a * a + bb * bb) + (c * c + e * e);
+    }
+    const float rstd = 1.0f / sqrtf(warp_sum(sq) / d + 1e-5f);
+    T* orow = out + (size_t)(r0 + k) * d;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int c = (lane + 32 * i) * 4;
+      const float4 gg = *reinterpret_cast<const float4*>(g + c);
+      const float4 bv = *reinterpret_cast<const float4*>(b + c);
+      store4(orow + c, (v[k][i].x - mean) * rstd * gg.x + bv.x, (v[k][i].y - mean) * rstd * gg.y + bv.y,
+             (v[k][i].z - mean) * rstd * gg.z + bv.z, (v[k][i].w - mean) * rstd * gg.w + bv.w);
+    }
   }
 }
 
@@ -223,12 +241,20 @@ __global__ void k_layernorm_gen(const Ctl* ctl, const float* __restrict__ h, con
 }
 
 // logdet[s] = -sum of s over the sample's rows and head groups (fixed order).
-__global__ void k_logdet_finalize(const float* __restrict__ part, int L, int G, float* logdet,
-                                  int accumulate) {
+__global__ void __launch_bounds__(512) k_logdet_finalize(const float* __restrict__ part, int L, int G,
+                                                         float* logdet, int accumulate) {
   const int s = blockIdx.x;
-  const float* p = part + (size_t)s * L * G * 2;
+  const float4* p = reinterpret_cast<const float4*>(part + (size_t)s * L * G * 2);
+  const int n = L * G / 2;                     // float4 = two (sum, unused) pairs
   float acc = 0.f;
-  for (int i = threadIdx.x; i < L * G; i += blockDim.x) acc += p[2 * i];
+#pragma unroll 4
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const float4 v = p[i];
+    acc += v.x + v.z;
+  }
+  if ((L * G) & 1) {
+    if (threadIdx.x == 0) acc += part[((size_t)s * L * G + L * G - 1) * 2];
+  }
   acc = block_sum(acc);
   if (threadIdx.x == 0) logdet[s] = accumulate ? logdet[s] - acc : -acc;
 }
@@ -358,13 +384,13 @@ template void launch_gather<bf16>(const Ctl*, const float*, int, int, int, bf16*
 template <typename T>
 void launch_layernorm(const Ctl* ctl, const float* h, const float* g, const float* b, T* out, int d,
                       int m_max, cudaStream_t st) {
-  const int grid = (m_max + 7) / 8;
+  const int grid = (m_max + 7) / 8, grid2 = (m_max + 15) / 16;
   switch (d % 128 == 0 ? d / 128 : 0) {
-    case 2: k_layernorm_reg<T, 2><<<grid, 256, 0, st>>>(ctl, h, g, b, out, d); break;
-    case 4: k_layernorm_reg<T, 4><<<grid, 256, 0, st>>>(ctl, h, g, b, out, d); break;
-    case 6: k_layernorm_reg<T, 6><<<grid, 256, 0, st>>>(ctl, h, g, b, out, d); break;
-    case 8: k_layernorm_reg<T, 8><<<grid, 256, 0, st>>>(ctl, h, g, b, out, d); break;
-    case 16: k_layernorm_reg<T, 16><<<grid, 256, 0, st>>>(ctl, h, g, b, out, d); break;
+    case 2: k_layernorm_reg<T, 2><<<grid2, 256, 0, st>>>(ctl, h, g, b, out, d); break;
+    case 4: k_layernorm_reg<T, 4><<<grid2, 256, 0, st>>>(ctl, h, g, b, out, d); break;
+    case 6: k_layernorm_reg<T, 6><<<grid2, 256, 0, st>>>(ctl, h, g, b, out, d); break;
+    case 8: k_layernorm_reg<T, 8><<<grid2, 256, 0, st>>>(ctl, h, g, b, out, d); break;
+    case 16: k_layernorm_reg<T, 16><<<grid2, 256, 0, st>>>(ctl, h, g, b, out, d); break;
     default: k_layernorm_gen<T><<<grid, 256, 0, st>>>(ctl, h, g, b, out, d); break;
   }
 }
@@ -373,7 +399,7 @@ template void launch_layernorm<bf16>(const Ctl*, const float*, const float*, con
 
 void launch_logdet_finalize(const float* part, int batch, int L, int G, float* logdet, int accumulate,
                             cudaStream_t st) {
-  k_logdet_finalize<<<batch, 256, 0, st>>>(part, L, G, logdet, accumulate);
+  k_logdet_finalize<<<batch, 512, 0, st>>>(part, L, G, logdet, accumulate);
 }
 
 void launch_block_init(Ctl* ctl, int* active, const float* z, float* x, int batch, int L, int C, int B,
@@ -385,7 +411,7 @@ void launch_block_init(Ctl* ctl, int* active, const float* z, float* x, int batc
 void launch_jacobi_step(Ctl* ctl, int* active, const float* part, int batch, int B, int G, float tau,
                         int max_iter, int32_t* iters, int nblocks, cudaGraphConditionalHandle inner,
                         cudaStream_t st) {
-  k_jacobi_step<<<1, 1024, 0, st>>>(ctl, active, part, batch, B, G, tau, max_iter, iters, nblocks, inner);
+  k_jacobi_step<<<batch, 512, 0, st>>>(ctl, active, part, batch, B, G, tau, max_iter, iters, nblocks, inner);
 }
 
 void launch_block_advance(Ctl* ctl, int nblocks, cudaGraphConditionalHandle outer, cudaStream_t st) {
