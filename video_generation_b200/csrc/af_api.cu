@@ -10,6 +10,7 @@
 #include <cuda_runtime.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <map>
@@ -20,6 +21,10 @@
 #include "af_kernels.h"
 
 using namespace af;
+
+namespace af {
+int g_pdl = 1;
+}
 
 namespace {
 
@@ -368,18 +373,27 @@ af_status graph_run(const af_model* mc, const std::string& key, cudaStream_t st,
   af_model* m = const_cast<af_model*>(mc);
   auto it = m->graphs.find(key);
   if (it == m->graphs.end()) {
-    cudaGraph_t g;
-    CK(cudaGraphCreate(&g, 0));
-    CK(cudaStreamBeginCaptureToGraph(m->cap, g, nullptr, nullptr, 0, cudaStreamCaptureModeRelaxed));
-    af_status s = build(ctx, m->cap);
-    cudaGraph_t g2;
-    cudaError_t ee = cudaStreamEndCapture(m->cap, &g2);
-    if (s) { cudaGraphDestroy(g); return s; }
-    if (ee != cudaSuccess) { cudaGraphDestroy(g); set_err("graph capture failed: %s", cudaGetErrorString(ee)); return AF_ERR_CUDA; }
     cudaGraphExec_t ex;
-    cudaError_t ie = cudaGraphInstantiate(&ex, g, 0);
-    cudaGraphDestroy(g);
-    if (ie != cudaSuccess) { set_err("graph instantiation failed: %s", cudaGetErrorString(ie)); return AF_ERR_CUDA; }
+    for (int attempt = 0;; ++attempt) {
+      cudaGraph_t g;
+      CK(cudaGraphCreate(&g, 0));
+      CK(cudaStreamBeginCaptureToGraph(m->cap, g, nullptr, nullptr, 0, cudaStreamCaptureModeRelaxed));
+      af_status s = build(ctx, m->cap);
+      cudaGraph_t g2;
+      cudaError_t ee = cudaStreamEndCapture(m->cap, &g2);
+      cudaError_t ie = cudaErrorUnknown;
+      if (!s && ee == cudaSuccess) ie = cudaGraphInstantiate(&ex, g, 0);
+      cudaGraphDestroy(g);
+      if (!s && ee == cudaSuccess && ie == cudaSuccess) break;
+      cudaGetLastError();
+      if (attempt == 0 && g_pdl) {   // programmatic edges refused here: plain edges instead
+        g_pdl = 0;
+        continue;
+      }
+      if (s) return s;
+      set_err("graph capture/instantiation failed: %s", cudaGetErrorString(ee != cudaSuccess ? ee : ie));
+      return AF_ERR_CUDA;
+    }
     if (m->graph_order.size() >= 16) {
       cudaGraphExecDestroy(m->graphs[m->graph_order.front()]);
       m->graphs.erase(m->graph_order.front());
@@ -541,6 +555,7 @@ af_status af_model_create(const af_config* cfg, const float* const* tensors, int
   for (int i = 0; i < n_tensors; ++i)
     if (!tensors[i]) { set_err("null tensor %d", i); return AF_ERR_ARG; }
 
+  if (const char* v = getenv("AF_PDL")) g_pdl = atoi(v) != 0;
   af_model* m = new af_model();
   m->cfg = c;
   m->fd = c.mlp_ratio * c.d;

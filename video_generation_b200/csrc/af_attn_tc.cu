@@ -180,10 +180,7 @@ __global__ void __launch_bounds__(384, 1)
   volatile int* abort_flag = &s_abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const Ctl* ctl = g.ctl;
-  const int R = ctl->R, p0 = ctl->p0;
-  const int q_tiles = (R + BQ - 1) / BQ;
-  const int n_items = q_tiles * g.heads * g.batch * g.nsplit;
+  pdl_trigger();
 
   const uint32_t kvf0 = smem_u32(bars), kve0 = smem_u32(bars + S);
   const uint32_t qf0 = smem_u32(bars + 2 * S), qe0 = smem_u32(bars + 2 * S + 2);
@@ -221,13 +218,21 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = s_tmem;
   const uint32_t tS = tmem, tO = tmem + 2 * BKV;              // S buffers at 0 and 128, O buffers at 256, 256 + hd
+  pdl_wait();                                                 // q, the cache and the row layout come from upstream
+  const Ctl* ctl = g.ctl;
+  const int R = ctl->R, p0 = ctl->p0;
+  const int q_tiles = (R + BQ - 1) / BQ;
+  const int n_items = q_tiles * g.heads * g.batch * g.nsplit;
 
   // Work item -> (query tile, head, sample, key split) and its key-tile range.
+  // The query tile varies slowest and the last (causally heaviest) tiles come
+  // first, so CTAs taking items round-robin get a balanced mix of work.
   struct Item { int qt, hh, s, split, q_begin, t0, nt; };
+  const int per_qt = g.heads * g.batch * g.nsplit;
   auto item_of = [&](int it) {
     Item x;
-    x.qt = it % q_tiles;
-    int r = it / q_tiles;
+    x.qt = q_tiles - 1 - it / per_qt;
+    int r = it % per_qt;
     x.hh = r % g.heads;
     r /= g.heads;
     x.split = r % g.nsplit;
@@ -502,6 +507,8 @@ __global__ void __launch_bounds__(384, 1)
 // Merge the splits' partials: o = sum_i 2^(m_i - m) o_i / sum_i 2^(m_i - m) l_i.
 template <int HD>
 __global__ void __launch_bounds__(256) k_attn_combine(AttnArgs g) {
+  pdl_trigger();
+  pdl_wait();
   const int wg = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int M = g.ctl->M;
   if (wg >= M * g.heads) return;
@@ -544,10 +551,10 @@ void launch_hd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
   }
   const long long items = (long long)((r_max + BQ - 1) / BQ) * g.heads * batch * g.nsplit;
   const int grid = (int)(items < sms ? items : sms);
-  k_attn_tc<HD><<<grid, 384, Cfg::SMEM, st>>>(tq, tk, tv, g, err);
+  launch_k(k_attn_tc<HD>, dim3(grid), dim3(384), Cfg::SMEM, st, tq, tk, tv, g, err);
   if (g.nsplit > 1) {
     const long long warps = (long long)g.m_max * g.heads;
-    k_attn_combine<HD><<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(g);
+    launch_k(k_attn_combine<HD>, dim3((unsigned)((warps * 32 + 255) / 256)), dim3(256), 0, st, g);
   }
 }
 

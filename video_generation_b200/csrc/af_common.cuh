@@ -185,6 +185,13 @@ __device__ __forceinline__ void epi4(const EpiArgs& e, int row, int col, float a
   }
 }
 
+// Programmatic dependent launch: every kernel lets its dependents launch as
+// soon as all of its CTAs are running, and waits for its predecessors'
+// results (griddepcontrol.wait) before reading anything they wrote.  Both are
+// no-ops for a kernel launched without a programmatic dependency.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Bounded wait helper: true while `t0` + limit_ns has not passed.
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;

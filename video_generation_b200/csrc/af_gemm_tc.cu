@@ -246,12 +246,11 @@ __global__ void __launch_bounds__(384, 1)
   volatile int* abort_flag = &s_abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_trigger();
   const uint32_t rank = CG == 2 ? cluster_rank() : 0u;   // 0 = the pair's leader (issues the MMAs)
   const int unit = CG == 2 ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int nunits = CG == 2 ? (int)(gridDim.x >> 1) : (int)gridDim.x;
-  const int M = e.ctl->M;
-  const int tiles_m = (M + TM - 1) / TM, tiles_n = N / BN;
-  const int ntiles = tiles_m * tiles_n;
+  const int tiles_n = N / BN;
   const int kbn = K / BK;
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S);
   const uint32_t tfull0 = smem_u32(bars + 2 * S), tempty0 = smem_u32(bars + 2 * S + 2);
@@ -290,6 +289,10 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t tmem = s_tmem;
   const uint32_t full_lead = CG == 2 ? map_to_rank(full0, 0) : full0;
   const uint32_t tempty_lead = CG == 2 ? map_to_rank(tempty0, 0) : tempty0;
+  pdl_wait();                      // the A operand and the row count come from upstream
+  const int M = e.ctl->M;
+  const int tiles_m = (M + TM - 1) / TM;
+  const int ntiles = tiles_m * tiles_n;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -610,18 +613,20 @@ void launch_bn_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, int N, int K,
   const int tiles = ((m_max + BM * CG - 1) / (BM * CG)) * (N / BN);
   const int units = tiles < max_units ? tiles : max_units;
   if (CG == 1) {
-    k_gemm_tc<BN, EPI, 1><<<units, 384, Cfg::SMEM, st>>>(tmA, tmB, N, K, e, err);
+    launch_k(k_gemm_tc<BN, EPI, 1>, dim3(units), dim3(384), Cfg::SMEM, st, tmA, tmB, N, K, e, err);
   } else {
     cudaLaunchConfig_t c = {};
     c.gridDim = dim3(2 * units);
     c.blockDim = dim3(384);
     c.dynamicSmemBytes = Cfg::SMEM;
     c.stream = st;
-    cudaLaunchAttribute a[1];
+    cudaLaunchAttribute a[2];
     a[0].id = cudaLaunchAttributeClusterDimension;
     a[0].val.clusterDim.x = 2; a[0].val.clusterDim.y = 1; a[0].val.clusterDim.z = 1;
+    a[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a[1].val.programmaticStreamSerializationAllowed = g_pdl;
     c.attrs = a;
-    c.numAttrs = 1;
+    c.numAttrs = 2;
     cudaLaunchKernelEx(&c, k_gemm_tc<BN, EPI, CG>, tmA, tmB, N, K, e, err);
   }
 }

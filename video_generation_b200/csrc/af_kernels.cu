@@ -53,11 +53,15 @@ int grid_for(long long work, int per_block) {
 // ------------------------------------------------------------------ control
 
 __global__ void k_ctl_forward(Ctl* ctl, int batch, int L) {
+  pdl_trigger();
+  pdl_wait();
   ctl->P = 0; ctl->p0 = 0; ctl->R = L; ctl->M = batch * L;
   ctl->block = 0; ctl->iter = 0; ctl->n_active = 0;
 }
 
 __global__ void k_call_init(Ctl* ctl, int reset_nonconv) {
+  pdl_trigger();
+  pdl_wait();
   ctl->block = 0;
   if (reset_nonconv) ctl->nonconv = 0;
 }
@@ -68,6 +72,8 @@ __global__ void k_call_init(Ctl* ctl, int reset_nonconv) {
 __global__ void k_block_init(Ctl* ctl, int* active, const float* __restrict__ z, float* x, int batch,
                              int L, int C, int B, int dir, int warm,
                              cudaGraphConditionalHandle inner) {
+  pdl_trigger();
+  pdl_wait();
   const int b = ctl->block;
   const int P = b * B;
   const int nvec = C >> 2;
@@ -109,6 +115,8 @@ __global__ void __launch_bounds__(512) k_jacobi_step(Ctl* ctl, int* active, cons
                                                      int batch, int B, int G, float tau, int max_iter,
                                                      int32_t* iters, int nblocks,
                                                      cudaGraphConditionalHandle inner) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int s_last;
   const int s = blockIdx.x;
   const int R = ctl->R, p0 = ctl->p0, P = ctl->P, iter = ctl->iter, blk = ctl->block;
@@ -151,6 +159,8 @@ __global__ void __launch_bounds__(512) k_jacobi_step(Ctl* ctl, int* active, cons
 }
 
 __global__ void k_block_advance(Ctl* ctl, int nblocks, cudaGraphConditionalHandle outer) {
+  pdl_trigger();
+  pdl_wait();
   const int b = ctl->block + 1;
   ctl->block = b;
   cudaGraphSetConditional(outer, b < nblocks ? 1u : 0u);
@@ -162,6 +172,8 @@ __global__ void k_block_advance(Ctl* ctl, int nblocks, cudaGraphConditionalHandl
 // x_{p-1} (zero at p = 0), read through the direction flip.
 template <typename T>
 __global__ void k_gather(const Ctl* ctl, const float* __restrict__ x, int L, int C, int dir, T* xin) {
+  pdl_trigger();
+  pdl_wait();
   const int M = ctl->M, R = ctl->R, p0 = ctl->p0;
   const int nvec = C >> 2;
   const long long n = (long long)M * nvec;
@@ -184,6 +196,8 @@ template <typename T, int NV>
 __global__ void __launch_bounds__(256) k_layernorm_reg(const Ctl* ctl, const float* __restrict__ h,
                                                        const float* __restrict__ g, const float* __restrict__ b,
                                                        T* out, int d) {
+  pdl_trigger();
+  pdl_wait();
   const int wg = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int M = ctl->M;
   const int r0 = 2 * wg;
@@ -225,6 +239,8 @@ __global__ void __launch_bounds__(256) k_layernorm_reg(const Ctl* ctl, const flo
 template <typename T>
 __global__ void k_layernorm_gen(const Ctl* ctl, const float* __restrict__ h, const float* __restrict__ g,
                                 const float* __restrict__ b, T* out, int d) {
+  pdl_trigger();
+  pdl_wait();
   const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (row >= ctl->M) return;
   const float* hr = h + (size_t)row * d;
@@ -243,6 +259,8 @@ __global__ void k_layernorm_gen(const Ctl* ctl, const float* __restrict__ h, con
 // logdet[s] = -sum of s over the sample's rows and head groups (fixed order).
 __global__ void __launch_bounds__(512) k_logdet_finalize(const float* __restrict__ part, int L, int G,
                                                          float* logdet, int accumulate) {
+  pdl_trigger();
+  pdl_wait();
   const int s = blockIdx.x;
   const float4* p = reinterpret_cast<const float4*>(part + (size_t)s * L * G * 2);
   const int n = L * G / 2;                     // float4 = two (sum, unused) pairs
@@ -265,6 +283,8 @@ __global__ void __launch_bounds__(512) k_logdet_finalize(const float* __restrict
 template <int EPI>
 __global__ void __launch_bounds__(256) k_gemm_simt(const float* __restrict__ A, const float* __restrict__ W,
                                                    int N, int K, EpiArgs e) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float As[16][64 + 4];
   __shared__ float Ws[16][64 + 4];
   const int M = e.ctl->M;
@@ -302,6 +322,8 @@ __global__ void __launch_bounds__(256) k_gemm_simt(const float* __restrict__ A, 
 
 // Head in fp32: one thread per (row, 16-column group), then the shared affine epilogue.
 __global__ void k_head_simt(const float* __restrict__ A, const float* __restrict__ W, int N, int K, EpiArgs e) {
+  pdl_trigger();
+  pdl_wait();
   const int G = N >> 4;
   const int M = e.ctl->M;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -325,6 +347,8 @@ template <int HD>
 __global__ void __launch_bounds__(256) k_attn_simt(const Ctl* ctl, const float* __restrict__ q,
                                                    const float* __restrict__ kc, const float* __restrict__ vc,
                                                    float* o, int Lc, int d, int heads) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float qs[8][HD];
   const int wib = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gw = blockIdx.x * 8 + wib;
@@ -367,16 +391,16 @@ __global__ void __launch_bounds__(256) k_attn_simt(const Ctl* ctl, const float* 
 // ------------------------------------------------------------------ launchers
 
 void launch_ctl_forward(Ctl* ctl, int batch, int L, cudaStream_t st) {
-  k_ctl_forward<<<1, 1, 0, st>>>(ctl, batch, L);
+  launch_k(k_ctl_forward, dim3(1), dim3(1), 0, st, ctl, batch, L);
 }
 void launch_call_init(Ctl* ctl, int reset_nonconv, cudaStream_t st) {
-  k_call_init<<<1, 1, 0, st>>>(ctl, reset_nonconv);
+  launch_k(k_call_init, dim3(1), dim3(1), 0, st, ctl, reset_nonconv);
 }
 
 template <typename T>
 void launch_gather(const Ctl* ctl, const float* x, int L, int C, int dir, T* xin, int m_max,
                    cudaStream_t st) {
-  k_gather<T><<<grid_for((long long)m_max * (C / 4), kThreads), kThreads, 0, st>>>(ctl, x, L, C, dir, xin);
+  launch_k(k_gather<T>, dim3(grid_for((long long)m_max * (C / 4), kThreads)), dim3(kThreads), 0, st, ctl, x, L, C, dir, xin);
 }
 template void launch_gather<float>(const Ctl*, const float*, int, int, int, float*, int, cudaStream_t);
 template void launch_gather<bf16>(const Ctl*, const float*, int, int, int, bf16*, int, cudaStream_t);
@@ -386,12 +410,12 @@ void launch_layernorm(const Ctl* ctl, const float* h, const float* g, const floa
                       int m_max, cudaStream_t st) {
   const int grid = (m_max + 7) / 8, grid2 = (m_max + 15) / 16;
   switch (d % 128 == 0 ? d / 128 : 0) {
-    case 2: k_layernorm_reg<T, 2><<<grid2, 256, 0, st>>>(ctl, h, g, b, out, d); break;
-    case 4: k_layernorm_reg<T, 4><<<grid2, 256, 0, st>>>(ctl, h, g, b, out, d); break;
-    case 6: k_layernorm_reg<T, 6><<<grid2, 256, 0, st>>>(ctl, h, g, b, out, d); break;
-    case 8: k_layernorm_reg<T, 8><<<grid2, 256, 0, st>>>(ctl, h, g, b, out, d); break;
-    case 16: k_layernorm_reg<T, 16><<<grid2, 256, 0, st>>>(ctl, h, g, b, out, d); break;
-    default: k_layernorm_gen<T><<<grid, 256, 0, st>>>(ctl, h, g, b, out, d); break;
+    case 2: launch_k(k_layernorm_reg<T, 2>, dim3(grid2), dim3(256), 0, st, ctl, h, g, b, out, d); break;
+    case 4: launch_k(k_layernorm_reg<T, 4>, dim3(grid2), dim3(256), 0, st, ctl, h, g, b, out, d); break;
+    case 6: launch_k(k_layernorm_reg<T, 6>, dim3(grid2), dim3(256), 0, st, ctl, h, g, b, out, d); break;
+    case 8: launch_k(k_layernorm_reg<T, 8>, dim3(grid2), dim3(256), 0, st, ctl, h, g, b, out, d); break;
+    case 16: launch_k(k_layernorm_reg<T, 16>, dim3(grid2), dim3(256), 0, st, ctl, h, g, b, out, d); break;
+    default: launch_k(k_layernorm_gen<T>, dim3(grid), dim3(256), 0, st, ctl, h, g, b, out, d); break;
   }
 }
 template void launch_layernorm<float>(const Ctl*, const float*, const float*, const float*, float*, int, int, cudaStream_t);
@@ -399,41 +423,41 @@ template void launch_layernorm<bf16>(const Ctl*, const float*, const float*, con
 
 void launch_logdet_finalize(const float* part, int batch, int L, int G, float* logdet, int accumulate,
                             cudaStream_t st) {
-  k_logdet_finalize<<<batch, 512, 0, st>>>(part, L, G, logdet, accumulate);
+  launch_k(k_logdet_finalize, dim3(batch), dim3(512), 0, st, part, L, G, logdet, accumulate);
 }
 
 void launch_block_init(Ctl* ctl, int* active, const float* z, float* x, int batch, int L, int C, int B,
                        int dir, int warm, cudaGraphConditionalHandle inner, cudaStream_t st) {
-  k_block_init<<<grid_for((long long)batch * B * (C / 4), kThreads), kThreads, 0, st>>>(
+  launch_k(k_block_init, dim3(grid_for((long long)batch * B * (C / 4), kThreads)), dim3(kThreads), 0, st, 
       ctl, active, z, x, batch, L, C, B, dir, warm, inner);
 }
 
 void launch_jacobi_step(Ctl* ctl, int* active, const float* part, int batch, int B, int G, float tau,
                         int max_iter, int32_t* iters, int nblocks, cudaGraphConditionalHandle inner,
                         cudaStream_t st) {
-  k_jacobi_step<<<batch, 512, 0, st>>>(ctl, active, part, batch, B, G, tau, max_iter, iters, nblocks, inner);
+  launch_k(k_jacobi_step, dim3(batch), dim3(512), 0, st, ctl, active, part, batch, B, G, tau, max_iter, iters, nblocks, inner);
 }
 
 void launch_block_advance(Ctl* ctl, int nblocks, cudaGraphConditionalHandle outer, cudaStream_t st) {
-  k_block_advance<<<1, 1, 0, st>>>(ctl, nblocks, outer);
+  launch_k(k_block_advance, dim3(1), dim3(1), 0, st, ctl, nblocks, outer);
 }
 
 void launch_gemm_simt(int epi, const float* A, const float* W, int N, int K, int m_max, const EpiArgs& e,
                       cudaStream_t st) {
   dim3 grid((N + 63) / 64, (m_max + 63) / 64);
   switch (epi) {
-    case EPI_INPROJ: k_gemm_simt<EPI_INPROJ><<<grid, 256, 0, st>>>(A, W, N, K, e); break;
-    case EPI_QKV: k_gemm_simt<EPI_QKV><<<grid, 256, 0, st>>>(A, W, N, K, e); break;
-    case EPI_RESID: k_gemm_simt<EPI_RESID><<<grid, 256, 0, st>>>(A, W, N, K, e); break;
-    case EPI_GELU: k_gemm_simt<EPI_GELU><<<grid, 256, 0, st>>>(A, W, N, K, e); break;
-    default: k_gemm_simt<EPI_RAW><<<grid, 256, 0, st>>>(A, W, N, K, e); break;
+    case EPI_INPROJ: launch_k(k_gemm_simt<EPI_INPROJ>, dim3(grid), dim3(256), 0, st, A, W, N, K, e); break;
+    case EPI_QKV: launch_k(k_gemm_simt<EPI_QKV>, dim3(grid), dim3(256), 0, st, A, W, N, K, e); break;
+    case EPI_RESID: launch_k(k_gemm_simt<EPI_RESID>, dim3(grid), dim3(256), 0, st, A, W, N, K, e); break;
+    case EPI_GELU: launch_k(k_gemm_simt<EPI_GELU>, dim3(grid), dim3(256), 0, st, A, W, N, K, e); break;
+    default: launch_k(k_gemm_simt<EPI_RAW>, dim3(grid), dim3(256), 0, st, A, W, N, K, e); break;
   }
 }
 
 void launch_head_simt(const float* A, const float* W, int N, int K, int m_max, const EpiArgs& e,
                       cudaStream_t st) {
   const long long n = (long long)m_max * (N / 16);
-  k_head_simt<<<(int)((n + 127) / 128), 128, 0, st>>>(A, W, N, K, e);
+  launch_k(k_head_simt, dim3((int)((n + 127) / 128)), dim3(128), 0, st, A, W, N, K, e);
 }
 
 void launch_attn_simt(const Ctl* ctl, const float* q, const float* kc, const float* vc, float* o, int batch,
@@ -441,10 +465,10 @@ void launch_attn_simt(const Ctl* ctl, const float* q, const float* kc, const flo
   (void)batch;
   const int grid = (int)(((long long)m_max * heads + 7) / 8);
   switch (d / heads) {
-    case 16: k_attn_simt<16><<<grid, 256, 0, st>>>(ctl, q, kc, vc, o, Lc, d, heads); break;
-    case 32: k_attn_simt<32><<<grid, 256, 0, st>>>(ctl, q, kc, vc, o, Lc, d, heads); break;
-    case 64: k_attn_simt<64><<<grid, 256, 0, st>>>(ctl, q, kc, vc, o, Lc, d, heads); break;
-    default: k_attn_simt<128><<<grid, 256, 0, st>>>(ctl, q, kc, vc, o, Lc, d, heads); break;
+    case 16: launch_k(k_attn_simt<16>, dim3(grid), dim3(256), 0, st, ctl, q, kc, vc, o, Lc, d, heads); break;
+    case 32: launch_k(k_attn_simt<32>, dim3(grid), dim3(256), 0, st, ctl, q, kc, vc, o, Lc, d, heads); break;
+    case 64: launch_k(k_attn_simt<64>, dim3(grid), dim3(256), 0, st, ctl, q, kc, vc, o, Lc, d, heads); break;
+    default: launch_k(k_attn_simt<128>, dim3(grid), dim3(256), 0, st, ctl, q, kc, vc, o, Lc, d, heads); break;
   }
 }
 

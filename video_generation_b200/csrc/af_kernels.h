@@ -7,6 +7,26 @@
 
 namespace af {
 
+// Launches with programmatic stream serialization when g_pdl is set (the
+// default; AF_PDL=0 in the environment turns it off), so that a kernel's
+// launch and set-up overlap the tail of the kernel before it.
+extern int g_pdl;
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                            Args&&... args) {
+  cudaLaunchConfig_t c = {};
+  c.gridDim = grid;
+  c.blockDim = block;
+  c.dynamicSmemBytes = smem;
+  c.stream = st;
+  cudaLaunchAttribute a[1];
+  a[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a[0].val.programmaticStreamSerializationAllowed = g_pdl;
+  c.attrs = a;
+  c.numAttrs = 1;
+  return cudaLaunchKernelEx(&c, kern, static_cast<KArgs>(args)...);
+}
+
 // ---- small kernels (af_kernels.cu) -----------------------------------------
 // All row-wise kernels read the live row count from ctl->M and are launched
 // for `m_max` rows.
