@@ -7,14 +7,14 @@
 // block's causal Transformer: input projection, QKV, attention output
 // projection, the two MLP matrices and the (mu, log-sigma) head.
 //
-// Design (one persistent CTA per SM, 384 threads):
+// Design (one persistent CTA per SM, 384 or 640 threads):
 //   warp 0      TMA producer: 128x64 A tile + BNx64 W tile per stage,
 //               128-byte swizzle, mbarrier transaction counts.
 //   warp 1      owns 512 TMEM columns; one thread issues tcgen05.mma
 //               (M=128, N=BN, K=16) into one of two accumulators and commits
 //               to the stage's "empty" barrier and the accumulator's "full".
-//   warps 4..11 epilogue, two warps per TMEM lane quarter (each takes half
-//               of the tile's columns): tcgen05.ld 32 lanes x 16 columns,
+//   warps 4..   epilogue, two or four warps per TMEM lane quarter (each takes
+//               a column group of the tile): tcgen05.ld 32 lanes x 16 columns,
 //               transpose through shared memory, apply the fused epilogue
 //               with row-coalesced stores, release the accumulator.
 // With two accumulators the epilogue of tile i overlaps the MMAs of tile i+1.
@@ -28,18 +28,29 @@ namespace af {
 namespace {
 
 constexpr int BM = 128, BK = 64;
+// Epilogue warps: 16 (4 per TMEM lane quarter) for the store-only epilogues,
+// 8 for those that also read a row of the residual stream or the positions
+// (more registers per thread).  Block = producer, MMA, 2 spare, epilogue.
+template <int EPI> struct EpiShape {
+  static constexpr int WARPS = (EPI == EPI_RESID || EPI == EPI_INPROJ) ? 8 : 16;
+  static constexpr int THREADS = (4 + WARPS) * 32;
+};
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-template <int BN, int CG> struct TcCfg {
+template <int BN, int CG, int EPI> struct TcCfg {
   // CG = CTAs per MMA: 1, or 2 for the SM-pair MMA (tile of 256 rows, each CTA
   // holding 128 rows of A and BN/2 rows of W).
-  static constexpr int STAGES = CG == 2 ? (BN >= 256 ? 6 : (BN >= 192 ? 6 : 7)) : (BN >= 256 ? 4 : (BN >= 192 ? 5 : 6));
+  static constexpr int EPI_WARPS = EpiShape<EPI>::WARPS;
+  static constexpr int STAGES = EPI_WARPS == 16
+      ? (CG == 2 ? (BN >= 256 ? 6 : (BN >= 192 ? 6 : 8)) : (BN >= 256 ? 3 : (BN >= 192 ? 4 : 6)))
+      : (CG == 2 ? (BN >= 256 ? 6 : (BN >= 192 ? 6 : 7)) : (BN >= 256 ? 4 : (BN >= 192 ? 5 : 6)));
   static constexpr uint32_t A_BYTES = BM * BK * 2;
   static constexpr uint32_t B_BYTES = (BN / CG) * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t NBARS = 2 * STAGES + 5;
-  // per epilogue warp (8 of them): a 32 x 16 fp32 staging tile, 16-byte chunks XOR-swizzled
-  static constexpr uint32_t EPI_BYTES = 8 * 32 * 16 * 4;
+  // per epilogue warp: a 32 x 16 fp32 staging tile, 16-byte chunks XOR-swizzled
+  static constexpr uint32_t EPI_BYTES = EPI_WARPS * 32 * 16 * 4;
+  static constexpr int THREADS = EpiShape<EPI>::THREADS;
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + NBARS * 8 + 16;
   // instruction descriptor: F32 accumulate, BF16 A and B, both K-major, N>>3, M>>4
   static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
@@ -228,10 +239,10 @@ __device__ __forceinline__ void st_bf16x4(bf16* dst, float a, float b, float c, 
 }
 
 template <int BN, int EPI, int CG>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int N, int K,
               EpiArgs e, int* err) {
-  using Cfg = TcCfg<BN, CG>;
+  using Cfg = TcCfg<BN, CG, EPI>;
   constexpr int S = Cfg::STAGES;
   constexpr int TM = BM * CG;               // accumulator rows per tile (both CTAs)
   extern __shared__ uint8_t smem_raw[];
@@ -264,7 +275,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(tfull0 + 8 * i, 1);
-      mbar_init(tempty0 + 8 * i, 256 * CG);
+      mbar_init(tempty0 + 8 * i, Cfg::EPI_WARPS * 32 * CG);
     }
     mbar_init(drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -380,14 +391,14 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp >= 4) {
       // ---------------------------------------------------------------- epilogue
     // Warp 4+ew owns TMEM lane quarter q = ew % 4 (rows 32q..32q+31 of the
-    // tile) and column half ew / 4.  A 16-column chunk is read from TMEM
+    // tile) and column quarter ew / 4.  A 16-column chunk is read from TMEM
     // (thread = row), transposed through a swizzled 32x16 staging tile, and
     // applied with lane l on row 8*it + l/4, columns 4*(l%4)..+3: each store
     // covers eight 64-byte row segments.  Row -> (sample, position) and the
     // destination row pointers are computed once per tile.
     const int ew = warp - 4;
-    const int q = ew & 3, hf = ew >> 2;
-    constexpr int HALF = BN / 2;
+    const int q = ew & 3, hf = ew >> 2;                 // lane quarter, column group
+    constexpr int HALF = BN / (Cfg::EPI_WARPS / 4);     // columns per warp
     float* stg = sEpi + ew * 32 * 16;
     const int rl = lane >> 2, cq = lane & 3;
     const int sw_w = (lane >> 1) & 3;            // swizzle of the row this lane writes
@@ -589,7 +600,7 @@ __global__ void __launch_bounds__(384, 1)
 template <int BN, int EPI, int CG>
 void launch_bn_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, int N, int K, int m_max, const EpiArgs& e,
                    int* err, int num_sms, cudaStream_t st) {
-  using Cfg = TcCfg<BN, CG>;
+  using Cfg = TcCfg<BN, CG, EPI>;
   static int max_units = 0;
   if (!max_units) {
     cudaFuncSetAttribute(k_gemm_tc<BN, EPI, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM);
@@ -597,7 +608,7 @@ void launch_bn_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, int N, int K,
     if (CG == 2) {
       cudaLaunchConfig_t q = {};
       q.gridDim = dim3(2 * max_units);
-      q.blockDim = dim3(384);
+      q.blockDim = dim3(Cfg::THREADS);
       q.dynamicSmemBytes = Cfg::SMEM;
       cudaLaunchAttribute a[1];
       a[0].id = cudaLaunchAttributeClusterDimension;
@@ -613,11 +624,11 @@ void launch_bn_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, int N, int K,
   const int tiles = ((m_max + BM * CG - 1) / (BM * CG)) * (N / BN);
   const int units = tiles < max_units ? tiles : max_units;
   if (CG == 1) {
-    launch_k(k_gemm_tc<BN, EPI, 1>, dim3(units), dim3(384), Cfg::SMEM, st, tmA, tmB, N, K, e, err);
+    launch_k(k_gemm_tc<BN, EPI, 1>, dim3(units), dim3(Cfg::THREADS), Cfg::SMEM, st, tmA, tmB, N, K, e, err);
   } else {
     cudaLaunchConfig_t c = {};
     c.gridDim = dim3(2 * units);
-    c.blockDim = dim3(384);
+    c.blockDim = dim3(Cfg::THREADS);
     c.dynamicSmemBytes = Cfg::SMEM;
     c.stream = st;
     cudaLaunchAttribute a[2];
