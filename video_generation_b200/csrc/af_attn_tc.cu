@@ -8,22 +8,30 @@
 // ... paper notes", key design 3: finished blocks feed a KV cache).
 //
 // Persistent CTAs (one per SM) walk a static list of work items: 128 query rows
-// of one (sample, head) against the key tiles of one split of the key range,
-// 128 keys per tile.  Q and the O accumulator are double-buffered across items
-// so the next item's loads and MMAs overlap the current item's softmax.
-//   warp 0      TMA: Q once (128 x hd), then K and V tiles (128 keys x hd)
-//               into a 2-3 stage ring; 128-byte swizzle.
-//   warp 1      one thread issues S_j = Q K_j^T (M=128, N=128, K=hd) into one
-//               of two TMEM buffers, and O += P_j V_j (M=128, N=hd, K=128)
-//               into the TMEM accumulator; V is consumed in its natural
-//               [key][hd] layout as an MN-major operand.
-//   warps 4-11  softmax, two warps per TMEM lane quarter, each owning half of
-//               a row's 128 scores and half of its hd outputs: pass 1 takes
-//               the row max (halves exchanged through shared memory), pass 2
-//               writes P = exp2(t - m) as bf16 into a swizzled shared tile.
-//               The running max is raised lazily: O (in TMEM) and the row sum
-//               are rescaled only when the max grows by more than 2^8, which
-//               keeps every P below 256 and the result exact.
+// of one (sample, head) against the 64-key tiles of one split of the key
+// range.  A CTA's items alternate between two groups, each a complete pipeline
+// with its own producer, MMA issuer, softmax warps and shared-memory buffers;
+// the groups share only the tensor core, the exponential units and (disjoint
+// columns of) TMEM, so one group's exponentials overlap the other's loads,
+// row maxima, MMA waits and output.  Per group:
+//   warp 0 / 2  TMA: the item's Q (128 x hd; the next item's Q is prefetched
+//               when two buffers fit), then per tile K into a short ring (read
+//               only by S = Q K^T) and V into its own ring; 128-byte swizzle.
+//   warp 1 / 3  one thread issues S_t = Q K_t^T (M=128, N=64, K=hd) into the
+//               group's TMEM S as soon as the softmax has taken S_{t-1} into
+//               registers, and O += P_{t-1} V_{t-1} (M=128, N=hd, K=64) into
+//               its TMEM O once that P is written; V is consumed in its
+//               natural [key][hd] layout (MN-major).
+//   warps 4-7 / 8-11  softmax: one thread per query row holds the tile's 64
+//               scores in registers, takes the row max, and writes P =
+//               exp2(t - m) as bf16 into one of the group's two swizzled P
+//               tiles with the row sum kept in fp32.  Warps whose 32 rows are
+//               all outside the sample, and 16-key chunks that the causal mask
+//               removes for all of a warp's rows, skip the arithmetic (masked
+//               chunks are written as zeros).  The running max is raised
+//               lazily: O (in TMEM) and the row sum are rescaled only when the
+//               max grows by more than 2^8, which keeps every P below 256 and
+//               the result exact.
 // With several splits, each writes an unnormalised (o, m, l) partial and
 // k_attn_combine merges them.  Every wait is bounded (2 s); on expiry the CTA
 // drains, frees TMEM and reports ERR_ATTN_WAIT.
@@ -32,28 +40,36 @@
 namespace af {
 namespace {
 
-constexpr int BQ = 128, BKV = 128;
+constexpr int BQ = 128;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kAttnThreads = 384;
 
 template <int HD> struct AttnCfg {
-  static constexpr int KCH = HD / 64;                     // 64-wide column boxes per row
-  static constexpr uint32_t BOX = 128 * 64 * 2;           // one 128-row x 64-col bf16 box: 16 KB
-  static constexpr uint32_t Q_BYTES = KCH * BOX;
-  static constexpr uint32_t KV_BYTES = KCH * BOX;         // K or V tile
-  static constexpr int STAGES = HD == 64 ? 3 : 2;
-  static constexpr int QBUF = HD == 64 ? 2 : 1;            // Q buffers across work items
-  static constexpr int PB = HD == 64 ? 2 : 1;              // P tiles (softmax j+1 overlaps P_j V_j)
-  static constexpr uint32_t P_BYTES = 2 * BOX;            // one P tile: 128 rows x 128 keys
-  static constexpr size_t SMEM = 1024 + QBUF * Q_BYTES + (size_t)STAGES * 2 * KV_BYTES + PB * P_BYTES +
-                                 3 * 2 * 128 * 4 + (2 * STAGES + 27) * 8 + 64;
-  // S = Q K^T: M 128, N 128, both K-major
+  static constexpr int BKV = 64;                          // keys per tile
+  static constexpr int KCH = HD / 64;                     // 64-column boxes per q / k / v row
+  static constexpr uint32_t QBOX = BQ * 128;              // 128 rows x 64 bf16: 16 KB
+  static constexpr uint32_t KVBOX = BKV * 128;            // BKV rows x 64 bf16
+  static constexpr uint32_t Q_BYTES = KCH * QBOX;
+  static constexpr uint32_t KV_BYTES = KCH * KVBOX;       // one K or one V tile
+  // Per group: QB Q buffers (the next item's Q prefetched when two fit), a K
+  // ring (a K tile is read only by its S = Q K^T), a V ring (held until P V)
+  // and two P tiles.
+  static constexpr int QB = HD == 64 ? 2 : 1;
+  static constexpr int SK = 2, SV = HD == 64 ? 4 : 1;
+  static constexpr uint32_t P_BYTES = QBOX;               // 128 rows x 64 keys
+  static constexpr uint32_t GROUP_BYTES = QB * Q_BYTES + (SK + SV) * KV_BYTES + 2 * P_BYTES;
+  // barriers per group: QF[QB] QE[QB] KF[SK] KE[SK] VF[SV] VE[SV] SF SR PF[2] OD[2] OR DRAIN
+  static constexpr int GBARS = 2 * QB + 2 * SK + 2 * SV + 8;
+  static constexpr size_t SMEM = 1024 + 2 * (size_t)GROUP_BYTES + 2 * GBARS * 8;
+  // S = Q K^T: M 128, N BKV, both K-major
   static constexpr uint32_t IDESC_S = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BKV >> 3) << 17) |
                                       ((uint32_t)(BQ >> 4) << 24);
   // O += P V: M 128, N hd, A (P) K-major, B (V) MN-major
   static constexpr uint32_t IDESC_O = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
                                       ((uint32_t)(HD >> 3) << 17) | ((uint32_t)(BQ >> 4) << 24);
 };
+static_assert(AttnCfg<64>::SMEM <= 232448 && AttnCfg<128>::SMEM <= 232448, "attention shared memory");
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -88,6 +104,9 @@ __device__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_fla
       }
     }
   }
+}
+__device__ __forceinline__ bool wait_fast(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  return mbar_try(bar, parity) || mbar_wait(bar, parity, abort_flag);
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1) {
   asm volatile(
@@ -158,55 +177,43 @@ struct AttnArgs {
 };
 
 template <int HD>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(kAttnThreads, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, AttnArgs g, int* err) {
   using Cfg = AttnCfg<HD>;
-  constexpr int S = Cfg::STAGES;
+  constexpr int BKV = Cfg::BKV, QB = Cfg::QB, SK = Cfg::SK, SV = Cfg::SV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  constexpr int QB = Cfg::QBUF;
-  uint8_t* sQ = smem;                                         // QB buffers
-  uint8_t* sK = sQ + QB * Cfg::Q_BYTES;
-  uint8_t* sV = sK + S * Cfg::KV_BYTES;
-  constexpr int PB = Cfg::PB;
-  uint8_t* sP = sV + S * Cfg::KV_BYTES;                       // PB tiles
-  float* red = reinterpret_cast<float*>(sP + PB * Cfg::P_BYTES);  // [2 tiles][2 halves][128], then [2 halves][128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 3 * 2 * 128);
-  // bars: kv_full[S], kv_empty[S], q_full[2], q_empty[2], s_full[2], s_free[2], p_full[2], o_done[2],
-  //       o_free[2], drain, pair[4 quarters][2 tiles], fin[4]
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   volatile int* abort_flag = &s_abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // group of this warp: warps 0, 1 and 4-7 serve group 0; warps 2, 3 and 8-11 group 1
+  const int grp = warp < 4 ? (warp >> 1) : ((warp - 4) >> 2);
   pdl_trigger();
 
-  const uint32_t kvf0 = smem_u32(bars), kve0 = smem_u32(bars + S);
-  const uint32_t qf0 = smem_u32(bars + 2 * S), qe0 = smem_u32(bars + 2 * S + 2);
-  const uint32_t sfull0 = smem_u32(bars + 2 * S + 4), sfree0 = smem_u32(bars + 2 * S + 6);
-  const uint32_t pfull0 = smem_u32(bars + 2 * S + 8), odone0 = smem_u32(bars + 2 * S + 10);
-  const uint32_t ofree0 = smem_u32(bars + 2 * S + 12), drain = smem_u32(bars + 2 * S + 14);
-  const uint32_t pair0 = smem_u32(bars + 2 * S + 15), fin0 = smem_u32(bars + 2 * S + 23);
+  // this group's shared memory: [Q buffers][K ring][V ring][2 P tiles]
+  uint8_t* gs = smem + grp * Cfg::GROUP_BYTES;
+  uint8_t* sQ = gs;
+  uint8_t* sK = sQ + QB * Cfg::Q_BYTES;
+  uint8_t* sV = sK + SK * Cfg::KV_BYTES;
+  uint8_t* sP = sV + SV * Cfg::KV_BYTES;
+  const uint32_t bars0 = smem_u32(smem + 2 * Cfg::GROUP_BYTES);
+  const uint32_t gb = bars0 + 8u * (uint32_t)(grp * Cfg::GBARS);
+  const uint32_t QF = gb, QE = QF + 8 * QB, KF = QE + 8 * QB, KE = KF + 8 * SK, VF = KE + 8 * SK,
+                 VE = VF + 8 * SV, SF = VE + 8 * SV, SR = SF + 8, PF = SR + 8, OD = PF + 16, OR = OD + 16,
+                 DRAIN = OR + 8;
 
   if (threadIdx.x == 0) {
     s_abort = 0;
-    for (int i = 0; i < S; ++i) {
-      mbar_init(kvf0 + 8 * i, 1);
-      mbar_init(kve0 + 8 * i, 1);
+    for (int i = 0; i < 2 * Cfg::GBARS; ++i) {
+      // arrival counts: SR, PF and OR take one arrival per softmax thread of the group
+      const int k = i % Cfg::GBARS;
+      const int sr = 2 * QB + 2 * SK + 2 * SV + 1;
+      const bool many = k == sr || k == sr + 1 || k == sr + 2 || k == sr + 5;
+      mbar_init(bars0 + 8 * i, many ? 128 : 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(qf0 + 8 * i, 1);
-      mbar_init(qe0 + 8 * i, 1);
-      mbar_init(sfull0 + 8 * i, 1);
-      mbar_init(sfree0 + 8 * i, 256);
-      mbar_init(ofree0 + 8 * i, 256);
-      mbar_init(pfull0 + 8 * i, 256);
-      mbar_init(odone0 + 8 * i, 1);
-    }
-    mbar_init(drain, 1);
-    for (int i = 0; i < 8; ++i) mbar_init(pair0 + 8 * i, 64);
-    for (int i = 0; i < 4; ++i) mbar_init(fin0 + 8 * i, 64);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -217,7 +224,8 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  const uint32_t tS = tmem, tO = tmem + 2 * BKV;              // S buffers at 0 and 128, O buffers at 256, 256 + hd
+  // TMEM columns: S of groups 0 and 1 at 0 and BKV, O of groups 0 and 1 at 2 BKV and 2 BKV + hd
+  const uint32_t tS = tmem + grp * BKV, tO = tmem + 2 * BKV + grp * HD;
   pdl_wait();                                                 // q, the cache and the row layout come from upstream
   const Ctl* ctl = g.ctl;
   const int R = ctl->R, p0 = ctl->p0;
@@ -225,10 +233,13 @@ __global__ void __launch_bounds__(384, 1)
   const int n_items = q_tiles * g.heads * g.batch * g.nsplit;
 
   // Work item -> (query tile, head, sample, key split) and its key-tile range.
-  // The query tile varies slowest and the last (causally heaviest) tiles come
+  // Query tiles end at R, R - 128, ...: the ragged tile is the first one, whose
+  // few rows need only the first keys (its rows before 0 are padding).  The
+  // query tile varies slowest and the last (causally heaviest) tiles come
   // first, so CTAs taking items round-robin get a balanced mix of work.
   struct Item { int qt, hh, s, split, q_begin, t0, nt; };
   const int per_qt = g.heads * g.batch * g.nsplit;
+  const int pad = q_tiles * BQ - R;
   auto item_of = [&](int it) {
     Item x;
     x.qt = q_tiles - 1 - it / per_qt;
@@ -237,120 +248,154 @@ __global__ void __launch_bounds__(384, 1)
     r /= g.heads;
     x.split = r % g.nsplit;
     x.s = r / g.nsplit;
-    x.q_begin = x.qt * BQ;
-    const int q_end = min(x.q_begin + BQ, R);
+    x.q_begin = x.qt * BQ - pad;
+    const int q_end = x.q_begin + BQ;
     const int ntiles = (p0 + q_end - 1) / BKV + 1;          // key tiles up to the last needed key
     x.t0 = x.split * g.tiles_per_split;
     x.nt = min(ntiles, x.t0 + g.tiles_per_split) - x.t0;
     return x;
   };
+  // The CTA's k-th item (k = 0, 1, ...) is global item blockIdx.x + k * gridDim.x
+  // and belongs to group k % 2; every role of a group walks the same items.
+  auto global_item = [&](int k) { return (int)blockIdx.x + k * (int)gridDim.x; };
 
-  if (warp == 0) {
+  if (warp < 4 && (warp & 1) == 0) {
     if (lane == 0) {
-      // ------------------------------------------------------------------ TMA producer
-      int stage = 0;
-      uint32_t phase = 0;
-      int gi = 0;
+      // ------------------------------------------------------------------ TMA producer of the group
+      int iw = 0, kst = 0, vst = 0;
+      uint32_t kph = 0, vph = 0;
       bool ok = true;
-      for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+      for (int k = grp; ok; k += 2) {
+        const int it = global_item(k);
+        if (it >= n_items) break;
         const Item x = item_of(it);
         if (x.nt <= 0) continue;
-        const int qb = gi % QB;
-        if (gi >= QB && !mbar_wait(qe0 + 8 * qb, (uint32_t)(((gi - QB) / QB) & 1), abort_flag)) break;
-        mbar_expect_tx(qf0 + 8 * qb, Cfg::Q_BYTES);
+        // Q buffer iw % QB is free once item iw - QB's last S has been computed.
+        // 32-row quarters; group 1 stores them in reverse order, so that on the
+        // diagonal its light quarters share a sub-partition with group 0's
+        // heavy ones (a softmax warp serves TMEM lanes 32 (warp % 4) ..).
+        const int qb = iw % QB;
+        if (iw >= QB && !mbar_wait(QE + 8 * qb, (uint32_t)(((iw / QB) - 1) & 1), abort_flag)) break;
+        mbar_expect_tx(QF + 8 * qb, Cfg::Q_BYTES);
 #pragma unroll
         for (int kc = 0; kc < Cfg::KCH; ++kc)
-          tma_load_2d(smem_u32(sQ + qb * Cfg::Q_BYTES + kc * Cfg::BOX), &tmQ, qf0 + 8 * qb, x.hh * HD + kc * 64,
-                      x.s * R + x.q_begin);
-        for (int j = 0; j < x.nt; ++j) {
-          if (!mbar_wait(kve0 + 8 * stage, phase ^ 1u, abort_flag)) { ok = false; break; }
-          mbar_expect_tx(kvf0 + 8 * stage, 2 * Cfg::KV_BYTES);
-          const int key0 = (x.t0 + j) * BKV;
 #pragma unroll
-          for (int kc = 0; kc < Cfg::KCH; ++kc) {
-            tma_load_2d(smem_u32(sK + stage * Cfg::KV_BYTES + kc * Cfg::BOX), &tmK, kvf0 + 8 * stage,
-                        x.hh * HD + kc * 64, x.s * g.Lc + key0);
-            tma_load_2d(smem_u32(sV + stage * Cfg::KV_BYTES + kc * Cfg::BOX), &tmV, kvf0 + 8 * stage,
-                        x.hh * HD + kc * 64, x.s * g.Lc + key0);
-          }
-          if (++stage == S) { stage = 0; phase ^= 1u; }
+          for (int qq = 0; qq < 4; ++qq)
+            tma_load_2d(smem_u32(sQ + qb * Cfg::Q_BYTES + kc * Cfg::QBOX + (grp ? 3 - qq : qq) * 4096), &tmQ,
+                        QF + 8 * qb, x.hh * HD + kc * 64, x.s * R + x.q_begin + 32 * qq);
+        for (int j = 0; j < x.nt; ++j) {
+          const int krow = x.s * g.Lc + (x.t0 + j) * BKV;
+          if (!mbar_wait(KE + 8 * kst, kph ^ 1u, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(KF + 8 * kst, Cfg::KV_BYTES);
+#pragma unroll
+          for (int kc = 0; kc < Cfg::KCH; ++kc)
+            tma_load_2d(smem_u32(sK + kst * Cfg::KV_BYTES + kc * Cfg::KVBOX), &tmK, KF + 8 * kst, x.hh * HD + kc * 64,
+                        krow);
+          if (++kst == SK) { kst = 0; kph ^= 1u; }
+          if (!mbar_wait(VE + 8 * vst, vph ^ 1u, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(VF + 8 * vst, Cfg::KV_BYTES);
+#pragma unroll
+          for (int kc = 0; kc < Cfg::KCH; ++kc)
+            tma_load_2d(smem_u32(sV + vst * Cfg::KV_BYTES + kc * Cfg::KVBOX), &tmV, VF + 8 * vst, x.hh * HD + kc * 64,
+                        krow);
+          if (++vst == SV) { vst = 0; vph ^= 1u; }
         }
-        ++gi;
+        ++iw;
       }
     }
-  } else if (warp == 1) {
+  } else if (warp < 4) {
     if (lane == 0) {
-      // ------------------------------------------------------------------ MMA issuer
-      int stage = 0, pstage = 0;
-      uint32_t phase = 0;
-      int gt = 0, gi = 0;                                     // global tile and item counters
+      // ------------------------------------------------------------------ MMA issuer of the group
+      // Per tile t: S_t = Q K_t^T as soon as the group has taken S_{t-1} into
+      // registers, then O += P_{t-1} V_{t-1} once that P is written.
+      // Descriptors are formed once; a step adds its offset (16-byte units).
+      const uint64_t dq = desc_k(smem_u32(sQ)), dk = desc_k(smem_u32(sK)), dp = desc_k(smem_u32(sP));
+      const uint64_t dv = desc_mn(smem_u32(sV), Cfg::KVBOX);
+      int iw = 0, kst = 0, vst = 0, t = 0;
+      uint32_t kph = 0, vph = 0;
+      // the tile whose P*V is pending: V stage and phase, tile within its item, item
+      bool pend = false;
+      int p_vst = 0, p_vph = 0, p_j = 0, p_iw = 0;
       bool ok = true;
-      for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+      auto issue_pv = [&]() -> bool {
+        const int u = t - 1, pb = u & 1;
+        // an item's first P*V overwrites O: the group has read the previous item's O
+        if (p_j == 0 && p_iw >= 1 && !wait_fast(OR, (uint32_t)((p_iw - 1) & 1), abort_flag)) return false;
+        if (!wait_fast(PF + 8 * pb, (uint32_t)((u >> 1) & 1), abort_flag)) return false;
+        if (!wait_fast(VF + 8 * p_vst, (uint32_t)p_vph, abort_flag)) return false;
+        tc_fence_after();
+        const uint64_t a0 = dp + (uint64_t)(pb * (Cfg::P_BYTES >> 4));
+        const uint64_t b0 = dv + (uint64_t)(p_vst * (Cfg::KV_BYTES >> 4));
+#pragma unroll
+        for (int ks = 0; ks < BKV / 16; ++ks)
+          umma(tO, a0 + (uint64_t)(ks * 2), b0 + (uint64_t)(ks * (2048 >> 4)), Cfg::IDESC_O, (p_j > 0 || ks > 0) ? 1u : 0u);
+        umma_commit(OD + 8 * pb);
+        umma_commit(VE + 8 * p_vst);                         // V tile no longer read
+        return true;
+      };
+      for (int k = grp; ok; k += 2) {
+        const int it = global_item(k);
+        if (it >= n_items) break;
         const Item x = item_of(it);
         if (x.nt <= 0) continue;
-        const int qb = gi % QB, ob = gi & 1;
-        if (!mbar_wait(qf0 + 8 * qb, (uint32_t)((gi / QB) & 1), abort_flag)) break;
-        if (gi >= 2 && !mbar_wait(ofree0 + 8 * ob, (uint32_t)(((gi - 2) >> 1) & 1), abort_flag)) break;
-        tc_fence_after();
-        const uint32_t dO = tO + ob * HD;
-        auto issue_pv = [&](int j, int gtile) -> bool {       // O += P_j V_j
-          const int pb = gtile % PB;
-          if (!mbar_wait(pfull0 + 8 * pb, (uint32_t)((gtile / PB) & 1), abort_flag)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < BKV / 16; ++ks) {
-            const uint64_t da = desc_k(smem_u32(sP + pb * Cfg::P_BYTES + (ks >> 2) * Cfg::BOX + (ks & 3) * 32));
-            const uint64_t db = desc_mn(smem_u32(sV + pstage * Cfg::KV_BYTES + ks * 16 * 128), Cfg::BOX);
-            umma(dO, da, db, Cfg::IDESC_O, (j > 0 || ks > 0) ? 1u : 0u);
-          }
-          umma_commit(odone0 + 8 * pb);
-          umma_commit(kve0 + 8 * pstage);
-          if (++pstage == S) pstage = 0;
-          return true;
-        };
+        const int qb = iw % QB;
+        if (!wait_fast(QF + 8 * qb, (uint32_t)((iw / QB) & 1), abort_flag)) { ok = false; break; }
+        const uint64_t aq = dq + (uint64_t)(qb * (Cfg::Q_BYTES >> 4));
         for (int j = 0; j < x.nt; ++j) {
-          const int gtile = gt + j;
-          if (!mbar_wait(kvf0 + 8 * stage, phase, abort_flag)) { ok = false; break; }
-          const int b = gtile & 1;
-          if (gtile >= 2 && !mbar_wait(sfree0 + 8 * b, (uint32_t)(((gtile - 2) >> 1) & 1), abort_flag)) { ok = false; break; }
+          if (!wait_fast(KF + 8 * kst, kph, abort_flag)) { ok = false; break; }
+          if (t >= 1 && !wait_fast(SR, (uint32_t)((t - 1) & 1), abort_flag)) { ok = false; break; }
           tc_fence_after();
+          const uint64_t bk = dk + (uint64_t)(kst * (Cfg::KV_BYTES >> 4));
 #pragma unroll
           for (int ks = 0; ks < HD / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * Cfg::BOX + (ks & 3) * 32;
-            umma(tS + b * BKV, desc_k(smem_u32(sQ + qb * Cfg::Q_BYTES + off)),
-                 desc_k(smem_u32(sK + stage * Cfg::KV_BYTES + off)), Cfg::IDESC_S, ks > 0 ? 1u : 0u);
+            const uint64_t off = (uint64_t)((ks >> 2) * (Cfg::QBOX >> 4) + (ks & 3) * 2);
+            const uint64_t offk = (uint64_t)((ks >> 2) * (Cfg::KVBOX >> 4) + (ks & 3) * 2);
+            umma(tS, aq + off, bk + offk, Cfg::IDESC_S, ks > 0 ? 1u : 0u);
           }
-          umma_commit(sfull0 + 8 * b);
-          if (j == x.nt - 1) umma_commit(qe0 + 8 * qb);       // the item's Q is no longer read
-          if (++stage == S) { stage = 0; phase ^= 1u; }
-          if (j >= 1 && !issue_pv(j - 1, gtile - 1)) { ok = false; break; }
+          umma_commit(SF);
+          umma_commit(KE + 8 * kst);                         // K tile no longer read
+          if (j == x.nt - 1) umma_commit(QE + 8 * qb);       // the item's Q is no longer read
+          if (++kst == SK) { kst = 0; kph ^= 1u; }
+          if (pend && !issue_pv()) { ok = false; break; }
+          pend = true;
+          p_vst = vst;
+          p_vph = (int)vph;
+          p_j = j;
+          p_iw = iw;
+          if (++vst == SV) { vst = 0; vph ^= 1u; }
+          ++t;
         }
-        if (!ok || !issue_pv(x.nt - 1, gt + x.nt - 1)) break;
-        gt += x.nt;
-        ++gi;
+        ++iw;
       }
-      umma_commit(drain);
-      const uint64_t tw = globaltimer_ns();
-      while (!mbar_try(drain, 0)) {
-        if (globaltimer_ns() - tw > kWaitLimitNs) { atomicExch(err, ERR_ATTN_WAIT); break; }
+      if (ok && pend && !issue_pv()) ok = false;
+      umma_commit(DRAIN);
+      const uint64_t tw0 = globaltimer_ns();
+      while (!mbar_try(DRAIN, 0)) {
+        if (globaltimer_ns() - tw0 > kWaitLimitNs) { atomicExch(err, ERR_ATTN_WAIT); break; }
       }
     }
-  } else if (warp >= 4) {
-    // -------------------------------------------------------------------- softmax
-    const int ew = warp - 4;
-    const int q = ew & 3, hf = ew >> 2;
-    const int row = q * 32 + lane;                            // 0..127 within the query tile
+  } else {
+    // -------------------------------------------------------------------- softmax of the group
+    const int w = grp;
+    const int q = warp & 3;                                   // TMEM lane quarter (warp % 4)
+    const int quarter = w ? 3 - q : q;                        // the query rows it holds
+    const int row = quarter * 32 + lane;                      // 0..127 within the query tile
     const float sl2 = 1.4426950408889634f / sqrtf((float)HD);
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    int gt = 0, gi = 0;
+    const uint32_t tSw = tS + lane_off, tOw = tO + lane_off;
+    uint8_t* prow0 = sP + (q * 32 + lane) * 128;             // P row = TMEM lane
+    const int sw = lane & 7;                                  // 128-byte swizzle of this row
+    int tw = 0;                                               // tiles this group has consumed
     bool alive = true;
-    for (int it = blockIdx.x; alive && it < n_items; it += gridDim.x) {
+    for (int k = w; alive; k += 2) {
+      const int it = global_item(k);
+      if (it >= n_items) break;
       const Item x = item_of(it);
       const int rloc = x.q_begin + row;
-      const size_t mrow = (size_t)x.s * R + rloc;
       if (x.nt <= 0) {
         // nothing to attend in this split: an empty partial (m = -inf, l = 0)
-        if (hf == 0 && rloc < R) {
+        if (rloc >= 0 && rloc < R) {
+          const size_t mrow = (size_t)x.s * R + rloc;
           float* ml = g.mlpart + (((size_t)x.split * g.m_max + mrow) * g.heads + x.hh) * 2;
           ml[0] = -INFINITY;
           ml[1] = 0.f;
@@ -358,141 +403,160 @@ __global__ void __launch_bounds__(384, 1)
         continue;
       }
       const int qpos = p0 + rloc;
-      const int qpos_min = p0 + x.q_begin;
-      const int ob = gi & 1;
-      float m_use = -INFINITY, l = 0.f;
+      const int wrow0 = x.q_begin + quarter * 32;             // the warp's first row
+      const bool wvalid = wrow0 + 31 >= 0 && wrow0 < R;       // warp-uniform
+      const int qlo = p0 + max(wrow0, 0), qhi = p0 + min(wrow0 + 31, R - 1);
+      float m_use = -INFINITY;
+      float2 l2 = make_float2(0.f, 0.f);
       int j = 0;
       for (; j < x.nt; ++j) {
-        const int gtile = gt + j;
-        const int b = gtile & 1;
         // every wait's outcome is made warp-uniform before any .aligned TMEM access
-        if (!__all_sync(0xffffffffu, mbar_wait(sfull0 + 8 * b, (uint32_t)((gtile >> 1) & 1), abort_flag))) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(SF, (uint32_t)(tw & 1), abort_flag))) break;
         tc_fence_after();
-        const int key0 = (x.t0 + j) * BKV + hf * 64;
-        const bool need_mask = (x.t0 + j) * BKV + BKV - 1 > qpos_min;
-        const uint32_t sa = tS + b * BKV + hf * 64 + lane_off;
-        // pass 1: row max.  The scores stay in registers for pass 2; the max is
-        // taken on raw scores and scaled once (the scale is positive).
-        float v[64];
+        const int key0 = (x.t0 + j) * BKV;
+        // the row's scores move to registers and S is released at once, so the
+        // next tile's S = Q K^T overlaps this tile's exponentials
+        float v[BKV];
+        if (wvalid) {
 #pragma unroll
-        for (int c = 0; c < 64; c += 16) tmem_ld16(sa + c, v + c);
-        tmem_wait_ld();
-        float mraw = -INFINITY;
-        if (need_mask) {
-#pragma unroll
-          for (int i = 0; i < 64; ++i)
-            if (key0 + i <= qpos) mraw = fmaxf(mraw, v[i]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 64; ++i) mraw = fmaxf(mraw, v[i]);
+          for (int c = 0; c < BKV; c += 16) tmem_ld16(tSw + c, v + c);
+          tmem_wait_ld();
         }
-        float mx = mraw * sl2;
-        float* rd = red + (b * 2) * 128;
-        rd[hf * 128 + row] = mx;
-        mbar_arrive(pair0 + 8 * (q * 2 + b));
-        if (!__all_sync(0xffffffffu, mbar_wait(pair0 + 8 * (q * 2 + b), (uint32_t)((gtile >> 1) & 1), abort_flag))) break;
-        mx = fmaxf(mx, rd[(1 - hf) * 128 + row]);
-        const float m_new = fmaxf(m_use, mx);
-        // raise the running max lazily; rows decide alone, the TMEM rescale of O
-        // runs for the whole warp when any of its rows needs it (factor 1 for the rest)
+        tc_fence_before();
+        mbar_arrive(SR);
         float corr = 1.f;
-        if (m_new > m_use + kRescaleLog2 || m_use == -INFINITY) {
-          if (m_use != -INFINITY) corr = exp2f(m_use - m_new);
-          l *= corr;
-          m_use = m_new;
+        if (wvalid) {
+          // row max on raw scores (the scale is positive), causal keys only
+          float mraw = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < BKV; c += 16) {
+            const int kc0 = key0 + c;
+            if (kc0 > qhi) continue;                          // masked for every row of the warp
+            if (kc0 + 15 <= qlo) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) mraw = fmaxf(mraw, v[c + i]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                if (kc0 + i <= qpos) mraw = fmaxf(mraw, v[c + i]);
+            }
+          }
+          const float m_new = fmaxf(m_use, mraw * sl2);
+          // raise the running max lazily; rows decide alone, the TMEM rescale of O
+          // runs for the whole warp when any of its rows needs it (factor 1 for the rest)
+          if (m_new > m_use + kRescaleLog2 || m_use == -INFINITY) {
+            if (m_use != -INFINITY) corr = exp2f(m_use - m_new);
+            l2 = fmul2(l2, splat(corr));
+            m_use = m_new;
+          }
+        }
+        // P tile tw % 2 is free once the group's P*V of tile tw - 2 has completed
+        const int pb = tw & 1;
+        if (tw >= 2 &&
+            !__all_sync(0xffffffffu, mbar_wait(OD + 8 * pb, (uint32_t)(((tw >> 1) - 1) & 1), abort_flag)))
+          break;
+        uint8_t* prow = prow0 + pb * Cfg::P_BYTES;
+        if (wvalid) {
+          // P = 2^(s * scale - m) in bf16, masked keys exactly 0
+          const float2 nmb = splat((m_use == -INFINITY) ? 0.f : -m_use);
+#pragma unroll
+          for (int c = 0; c < BKV; c += 16) {
+            const int kc0 = key0 + c;
+            uint32_t pk[8];
+            if (kc0 > qhi) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) pk[i] = 0u;
+            } else {
+              const bool partial = kc0 + 15 > qlo;
+#pragma unroll
+              for (int i = 0; i < 16; i += 2) {
+                float2 t = ffma2(make_float2(v[c + i], v[c + i + 1]), splat(sl2), nmb);
+                if (partial) {
+                  if (kc0 + i > qpos) t.x = -INFINITY;           // 2^-inf = +0
+                  if (kc0 + i + 1 > qpos) t.y = -INFINITY;
+                }
+                const float2 e = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+                l2 = fadd2(l2, e);
+                pk[i >> 1] = pack_bf16(e.x, e.y);
+              }
+            }
+            const int u0 = c >> 3;                            // 16-byte units u0, u0 + 1 of this row
+            *reinterpret_cast<uint4*>(prow + ((u0 ^ sw) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(prow + (((u0 + 1) ^ sw) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
         }
         if (j >= 1 && __any_sync(0xffffffffu, corr != 1.f)) {
-          // O holds tiles 0..j-1: wait for P_{j-1} V_{j-1}
-          const int gp = gtile - 1;
-          if (!__all_sync(0xffffffffu, mbar_wait(odone0 + 8 * (gp % PB), (uint32_t)((gp / PB) & 1), abort_flag))) break;
+          // the max grew: rescale O, which must hold tiles 0..j-1, before this
+          // tile's P*V is issued
+          const int tl = tw - 1;
+          if (!__all_sync(0xffffffffu, mbar_wait(OD + 8 * (tl & 1), (uint32_t)((tl >> 1) & 1), abort_flag)))
+            break;
           tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < HD / 2; c += 16) {
-            float v[16];
-            const uint32_t oa = tO + ob * HD + hf * (HD / 2) + c + lane_off;
-            tmem_ld16(oa, v);
+          for (int c = 0; c < HD; c += 16) {
+            float o[16];
+            tmem_ld16(tOw + c, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] *= corr;
-            tmem_st16(oa, v);
+            for (int i = 0; i < 16; i += 2) {
+              const float2 r2 = fmul2(make_float2(o[i], o[i + 1]), splat(corr));
+              o[i] = r2.x;
+              o[i + 1] = r2.y;
+            }
+            tmem_st16(tOw + c, o);
           }
           tmem_wait_st();
         }
-        // the P tile this tile writes was last read by tile gtile - PB
-        const int pb = gtile % PB;
-        if (gtile >= PB &&
-            !__all_sync(0xffffffffu, mbar_wait(odone0 + 8 * pb, (uint32_t)(((gtile - PB) / PB) & 1), abort_flag)))
-          break;
-        // pass 2: P = 2^(s * scale - m) in bf16 into the swizzled P tile, row sums;
-        // masked keys are exactly 0
-        const float nmb = (m_use == -INFINITY) ? 0.f : -m_use;
-        uint8_t* prow = sP + pb * Cfg::P_BYTES + hf * Cfg::BOX + row * 128;
-#pragma unroll
-        for (int c = 0; c < 64; c += 16) {
-          uint32_t pk[8];
-#pragma unroll
-          for (int i = 0; i < 16; i += 2) {
-            float e0 = ex2_approx(fmaf(v[c + i], sl2, nmb));
-            float e1 = ex2_approx(fmaf(v[c + i + 1], sl2, nmb));
-            if (need_mask) {
-              if (key0 + c + i > qpos) e0 = 0.f;
-              if (key0 + c + i + 1 > qpos) e1 = 0.f;
-            }
-            l += e0 + e1;
-            pk[i >> 1] = pack_bf16(e0, e1);
-          }
-          const int u0 = c >> 3;                             // 16-byte units u0, u0+1 of this row
-          *reinterpret_cast<uint4*>(prow + (((u0) ^ (row & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          *reinterpret_cast<uint4*>(prow + (((u0 + 1) ^ (row & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tc_fence_before();
-        mbar_arrive(pfull0 + 8 * pb);
-        mbar_arrive(sfree0 + 8 * b);
+        mbar_arrive(PF + 8 * pb);
+        ++tw;
       }
-      // item epilogue: wait for its last O, combine the halves' row sums, write out
-      const int glast = gt + x.nt - 1;
-      const bool ok = __all_sync(0xffffffffu, (j == x.nt) && mbar_wait(odone0 + 8 * (glast % PB),
-                                                                        (uint32_t)((glast / PB) & 1), abort_flag));
+      // item epilogue: wait for the last P*V, read O, release it, normalise and store
+      // (the item's sample, head and split are looked up again here rather than
+      // kept in registers through the tile loop)
+      const Item xe = item_of(it);
+      const size_t mrow = (size_t)xe.s * R + rloc;
+      const int tl = tw - 1;
+      const bool ok = __all_sync(
+          0xffffffffu, (j == x.nt) && mbar_wait(OD + 8 * (tl & 1), (uint32_t)((tl >> 1) & 1), abort_flag));
       tc_fence_after();
-      float* rl = red + 4 * 128;                               // past both row-max slots
-      rl[hf * 128 + row] = l;
-      mbar_arrive(fin0 + 8 * q);
-      const bool ok2 = __all_sync(0xffffffffu, mbar_wait(fin0 + 8 * q, (uint32_t)(gi & 1), abort_flag));
-      const float lt = l + rl[(1 - hf) * 128 + row];
-      const bool valid = ok && ok2 && rloc < R;
+      const float lt = l2.x + l2.y;
+      const bool valid = ok && rloc >= 0 && rloc < R;
+      const float inv = 1.f / lt;
+      // 32 columns at a time; O is released after the last TMEM read
 #pragma unroll
-      for (int c = 0; c < HD / 2; c += 16) {
-        float v[16];
-        tmem_ld16(tO + ob * HD + hf * (HD / 2) + c + lane_off, v);
-        tmem_wait_ld();
-        const int col = x.hh * HD + hf * (HD / 2) + c;
+      for (int h0 = 0; h0 < HD; h0 += 32) {
+        float o[32];
+        if (wvalid && ok) {
+          tmem_ld16(tOw + h0, o);
+          tmem_ld16(tOw + h0 + 16, o + 16);
+          tmem_wait_ld();
+        }
+        if (h0 + 32 == HD) {
+          tc_fence_before();
+          mbar_arrive(OR);                           // O may be overwritten by the group's next item
+        }
         if (!valid) continue;
         if (g.nsplit == 1) {
-          const float inv = 1.f / lt;
-          uint32_t pk[8];
+          uint4* dst = reinterpret_cast<uint4*>(g.o + mrow * g.d + xe.hh * HD + h0);
 #pragma unroll
-          for (int i = 0; i < 16; i += 2) pk[i >> 1] = pack_bf16(v[i] * inv, v[i + 1] * inv);
-          uint4* dst = reinterpret_cast<uint4*>(g.o + mrow * g.d + col);
-          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          for (int c = 0; c < 32; c += 8)
+            dst[c >> 3] = make_uint4(pack_bf16(o[c] * inv, o[c + 1] * inv), pack_bf16(o[c + 2] * inv, o[c + 3] * inv),
+                                     pack_bf16(o[c + 4] * inv, o[c + 5] * inv), pack_bf16(o[c + 6] * inv, o[c + 7] * inv));
         } else {
-          float4* dst = reinterpret_cast<float4*>(g.opart + ((size_t)x.split * g.m_max + mrow) * g.d + col);
+          float4* dst =
+              reinterpret_cast<float4*>(g.opart + ((size_t)xe.split * g.m_max + mrow) * g.d + xe.hh * HD + h0);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          for (int c = 0; c < 32; c += 4) dst[c >> 2] = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
         }
       }
-      if (valid && g.nsplit > 1 && hf == 0) {
-        float* ml = g.mlpart + (((size_t)x.split * g.m_max + mrow) * g.heads + x.hh) * 2;
+      if (valid && g.nsplit > 1) {
+        float* ml = g.mlpart + (((size_t)xe.split * g.m_max + mrow) * g.heads + xe.hh) * 2;
         ml[0] = m_use;
         ml[1] = lt;
       }
-      // the O buffer and the row-sum slots are free for the item after next
-      tc_fence_before();
-      mbar_arrive(ofree0 + 8 * ob);
-      alive = ok && ok2;
-      gt += x.nt;
-      ++gi;
+      alive = ok;
     }
   }
   tc_fence_before();
@@ -535,7 +599,7 @@ __global__ void __launch_bounds__(256) k_attn_combine(AttnArgs g) {
 }
 
 template <int HD>
-void launch_hd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& g, int batch,
+bool launch_hd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& g, int batch,
                int r_max, int* err, cudaStream_t st) {
   using Cfg = AttnCfg<HD>;
   static bool attr = false;
@@ -551,11 +615,12 @@ void launch_hd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
   }
   const long long items = (long long)((r_max + BQ - 1) / BQ) * g.heads * batch * g.nsplit;
   const int grid = (int)(items < sms ? items : sms);
-  launch_k(k_attn_tc<HD>, dim3(grid), dim3(384), Cfg::SMEM, st, tq, tk, tv, g, err);
+  launch_k(k_attn_tc<HD>, dim3(grid), dim3(kAttnThreads), Cfg::SMEM, st, tq, tk, tv, g, err);
   if (g.nsplit > 1) {
     const long long warps = (long long)g.m_max * g.heads;
     launch_k(k_attn_combine<HD>, dim3((unsigned)((warps * 32 + 255) / 256)), dim3(256), 0, st, g);
   }
+  return true;
 }
 
 }  // namespace
@@ -564,7 +629,7 @@ int attn_tc_splits(int batch, int heads, int r_max, int Lc, int num_sms) {
   const int q_tiles = (r_max + BQ - 1) / BQ;
   const long long ctas = (long long)q_tiles * heads * batch;
   if (ctas >= 2LL * num_sms) return 1;
-  const int key_tiles = (Lc + BKV - 1) / BKV;
+  const int key_tiles = (Lc + 127) / 128;                   // in 128-key units
   int n = (key_tiles + 15) / 16;
   if (n < 1) n = 1;
   if (n > 64) n = 64;
@@ -574,9 +639,11 @@ int attn_tc_splits(int batch, int heads, int r_max, int Lc, int num_sms) {
 bool launch_attn_tc2(const Ctl* ctl, const bf16* q, const bf16* kc, const bf16* vc, bf16* o, float* opart,
                      float* mlpart, int nsplit, int batch, int Lc, int d, int heads, int r_max, int m_max, int* err,
                      cudaStream_t st) {
+  const int hd = d / heads;
+  const int bkv = hd == 64 ? AttnCfg<64>::BKV : AttnCfg<128>::BKV;
   CUtensorMap tq, tk, tv;
-  if (!make_tmap_bf16(&tq, q, m_max, d, 128) || !make_tmap_bf16(&tk, kc, batch * Lc, d, 128) ||
-      !make_tmap_bf16(&tv, vc, batch * Lc, d, 128))
+  if (!make_tmap_bf16(&tq, q, m_max, d, 32) || !make_tmap_bf16(&tk, kc, batch * Lc, d, bkv) ||
+      !make_tmap_bf16(&tv, vc, batch * Lc, d, bkv))
     return false;
   AttnArgs g;
   g.ctl = ctl;
@@ -587,13 +654,12 @@ bool launch_attn_tc2(const Ctl* ctl, const bf16* q, const bf16* kc, const bf16* 
   g.d = d;
   g.heads = heads;
   g.nsplit = nsplit;
-  const int key_tiles = (Lc + BKV - 1) / BKV;
+  const int key_tiles = (Lc + bkv - 1) / bkv;
   g.tiles_per_split = (key_tiles + nsplit - 1) / nsplit;
   g.m_max = m_max;
   g.batch = batch;
-  if (d / heads == 64) launch_hd<64>(tq, tk, tv, g, batch, r_max, err, st);
-  else launch_hd<128>(tq, tk, tv, g, batch, r_max, err, st);
-  return true;
+  return hd == 64 ? launch_hd<64>(tq, tk, tv, g, batch, r_max, err, st)
+                  : launch_hd<128>(tq, tk, tv, g, batch, r_max, err, st);
 }
 
 }  // namespace af
