@@ -216,16 +216,18 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
     bf16* q = (bf16*)b.q;
     bf16* u = (bf16*)b.u;
     const int ns = m->num_sms;
-    CUtensorMap tA_x, tA_a, tA_u, tB;
+    CUtensorMap tA_x, tA_a, tA_u, tB, tC_h, tC_u;
     bool ok = make_tmap_bf16(&tA_x, xin, m_max, C, 128) && make_tmap_bf16(&tA_a, a, m_max, d, 128) &&
-              make_tmap_bf16(&tA_u, u, m_max, fd, 128);
+              make_tmap_bf16(&tA_u, u, m_max, fd, 128) && make_tmap_out(&tC_h, b.h, true, m_max, d) &&
+              make_tmap_out(&tC_u, u, false, m_max, fd);
     if (!ok) { set_err("cuTensorMapEncodeTiled failed for an activation"); return AF_ERR_CUDA; }
     auto gemm = [&](int epi, const CUtensorMap& tA, const void* W, int N, int K, const EpiArgs& ea) -> bool {
       // a QKV tile must fall inside one of q, k, v; the position-add epilogue
       // keeps two row sets in flight and stays at <= 192 columns
       const int pick = gemm_tc_pick(N, m_max, ns, epi == EPI_QKV ? d : 0, epi == EPI_INPROJ ? 192 : 256);
       if (!pick || !make_tmap_bf16(&tB, W, N, K, (pick / 10) / (pick % 10))) return false;
-      launch_gemm_tc(epi, tA, tB, pick, N, K, m_max, ea, m->d_err, ns, st);
+      const CUtensorMap* tC = epi == EPI_RESID ? &tC_h : (epi == EPI_GELU ? &tC_u : nullptr);
+      launch_gemm_tc(epi, tA, tB, tC, pick, N, K, m_max, ea, m->d_err, ns, st);
       return true;
     };
     launch_gather<bf16>(b.ctl, xsrc, L, C, dir, xin, m_max, st);

@@ -34,6 +34,11 @@ constexpr int BM = 128, BK = 64;
 template <int EPI> struct EpiShape {
   static constexpr int WARPS = (EPI == EPI_RESID || EPI == EPI_INPROJ) ? 8 : 16;
   static constexpr int THREADS = (4 + WARPS) * 32;
+  // residual add and GELU leave through TMA: each warp stages 32 rows x 16
+  // columns (two slots, alternating) in the output tensor map's swizzle and
+  // issues a bulk reduce-add (h += tile) or a bulk store (u = tile)
+  static constexpr bool TMA_OUT = EPI == EPI_RESID || EPI == EPI_GELU;
+  static constexpr uint32_t SLOT = EPI == EPI_RESID ? 32 * 16 * 4 : 32 * 16 * 2;
 };
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
@@ -41,17 +46,20 @@ template <int BN, int CG, int EPI> struct TcCfg {
   // CG = CTAs per MMA: 1, or 2 for the SM-pair MMA (tile of 256 rows, each CTA
   // holding 128 rows of A and BN/2 rows of W).
   static constexpr int EPI_WARPS = EpiShape<EPI>::WARPS;
-  static constexpr int STAGES = EPI_WARPS == 16
-      ? (CG == 2 ? (BN >= 256 ? 6 : (BN >= 192 ? 6 : 8)) : (BN >= 256 ? 3 : (BN >= 192 ? 4 : 6)))
-      : (CG == 2 ? (BN >= 256 ? 6 : (BN >= 192 ? 6 : 7)) : (BN >= 256 ? 4 : (BN >= 192 ? 5 : 6)));
   static constexpr uint32_t A_BYTES = BM * BK * 2;
   static constexpr uint32_t B_BYTES = (BN / CG) * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  // per epilogue warp: a 32 x 16 fp32 transpose tile, 16-byte chunks
+  // XOR-swizzled, or two TMA staging slots
+  static constexpr uint32_t EPI_BYTES =
+      EpiShape<EPI>::TMA_OUT ? EPI_WARPS * 2 * EpiShape<EPI>::SLOT : EPI_WARPS * 32 * 16 * 4;
+  // as many stages as the remaining shared memory holds (at most 8)
+  static constexpr int STAGES_FIT = (int)((232448u - 1024u - 512u - EPI_BYTES) / STAGE_BYTES);
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static constexpr uint32_t NBARS = 2 * STAGES + 5;
-  // per epilogue warp: a 32 x 16 fp32 staging tile, 16-byte chunks XOR-swizzled
-  static constexpr uint32_t EPI_BYTES = EPI_WARPS * 32 * 16 * 4;
   static constexpr int THREADS = EpiShape<EPI>::THREADS;
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + NBARS * 8 + 16;
+  static_assert(STAGES >= 3 && SMEM <= 232448, "GEMM shared memory");
   // instruction descriptor: F32 accumulate, BF16 A and B, both K-major, N>>3, M>>4
   static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                     ((uint32_t)((BM * CG) >> 4) << 24);
@@ -211,6 +219,24 @@ __device__ __forceinline__ float2 gelu2_as7126(float2 v) {
   return ffma2(hv, erf_s, hv);
 }
 
+// TMA bulk writes of a staged tile (one thread), tracked as bulk async-groups.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(c0), "r"(c1)
+               : "memory");
+}
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(c0), "r"(c1)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// at most one group still reading its shared-memory source
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ void st_bf16x4(bf16* dst, float a, float b, float c, float d) {
   __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
   uint2 u;
@@ -221,8 +247,8 @@ __device__ __forceinline__ void st_bf16x4(bf16* dst, float a, float b, float c, 
 
 template <int BN, int EPI, int CG>
 __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
-    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int N, int K,
-              EpiArgs e, int* err) {
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const __grid_constant__ CUtensorMap tmC, int N, int K, EpiArgs e, int* err) {
   using Cfg = TcCfg<BN, CG, EPI>;
   constexpr int S = Cfg::STAGES;
   constexpr int TM = BM * CG;               // accumulator rows per tile (both CTAs)
@@ -262,6 +288,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+    if (EpiShape<EPI>::TMA_OUT) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmC)) : "memory");
   }
   if (warp == 1) {
     if (CG == 2) {
@@ -380,191 +407,272 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
     const int ew = warp - 4;
     const int q = ew & 3, hf = ew >> 2;                 // lane quarter, column group
     constexpr int HALF = BN / (Cfg::EPI_WARPS / 4);     // columns per warp
-    float* stg = sEpi + ew * 32 * 16;
-    const int rl = lane >> 2, cq = lane & 3;
-    const int sw_w = (lane >> 1) & 3;            // swizzle of the row this lane writes
-    const int sw_r = (rl >> 1) & 3;              // swizzle of the rows this lane reads
-    const Ctl* ctl = e.ctl;
-    const int R = ctl->R, p0 = ctl->p0;
-    int i = 0;
-    for (int t = unit; t < ntiles; t += nunits, ++i) {
-      const int acc = i & 1;
-      const uint32_t use = (uint32_t)(i >> 1);
-      const int mb = t % tiles_m, nb = t / tiles_m;
-      const int row0 = mb * TM + (int)rank * BM + q * 32;
-      const int n0 = nb * BN + hf * HALF;
-      const uint32_t taddr = tmem + (uint32_t)(acc * BN + hf * HALF) + ((uint32_t)(q * 32) << 16);
-      // per-tile row info for the 4 rows this lane stores
-      char* rowp[4];
-      const float* pos_s[4];
-      const float* pos_t[4];
-      int colbase = 0;
+    if constexpr (EpiShape<EPI>::TMA_OUT) {
+      // Thread = row: each 16-column chunk read from TMEM gets its bias (and
+      // GELU) and is written, in the output tensor map's swizzle, to one of the
+      // warp's two staging slots; lane 0 then sends the 32 x 16 tile with a TMA
+      // bulk reduce-add into h (each element gets exactly one add, so the result
+      // is deterministic) or a bulk store into u.  Rows past the last real row
+      // land in workspace rows no kernel reads; rows past the buffer are clipped.
+      constexpr uint32_t SLOT = EpiShape<EPI>::SLOT;
+      constexpr int NCH = HALF / 16;
+      uint8_t* stg0 = reinterpret_cast<uint8_t*>(sEpi) + ew * 2 * SLOT;
+      int cc = 0;                                       // chunks sent by this warp
+      int i = 0;
+      for (int t = unit; t < ntiles; t += nunits, ++i) {
+        const int acc = i & 1;
+        const uint32_t use = (uint32_t)(i >> 1);
+        const int mb = t % tiles_m, nb = t / tiles_m;
+        const int row0 = mb * TM + (int)rank * BM + q * 32;
+        const int n0 = nb * BN + hf * HALF;
+        const uint32_t taddr = tmem + (uint32_t)(acc * BN + hf * HALF) + ((uint32_t)(q * 32) << 16);
+        // the wait's outcome is made warp-uniform before the .aligned TMEM loads
+        if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * acc, use & 1u, abort_flag))) break;
+        tc_fence_after();
+        float vb[2][16];
+        tmem_ld16(taddr, vb[0]);
 #pragma unroll
-      for (int it = 0; it < 4; ++it) {
-        const int r = row0 + it * 8 + rl;
-        if (EPI == EPI_RESID) rowp[it] = reinterpret_cast<char*>(e.h + (size_t)r * e.d);
-        if (EPI == EPI_GELU) rowp[it] = reinterpret_cast<char*>(reinterpret_cast<bf16*>(e.out) + (size_t)r * e.ldo);
-        if (EPI == EPI_INPROJ || EPI == EPI_QKV) {
+        for (int k = 0; k < NCH; ++k) {
+          tmem_wait_ld();
+          if (k + 1 < NCH) {
+            tmem_ld16(taddr + (k + 1) * 16, vb[(k + 1) & 1]);
+          } else {
+            // every TMEM read of this tile is done: release the accumulator
+            tc_fence_before();
+            if (CG == 2) mbar_arrive_cluster(tempty_lead + 8 * acc);
+            else mbar_arrive(tempty0 + 8 * acc);
+          }
+          const float* v = vb[k & 1];
+          const int col = n0 + k * 16;
+          const float4* b4 = reinterpret_cast<const float4*>(e.bias + col);
+          uint8_t* slot = stg0 + (cc & 1) * SLOT;
+          if (lane == 0) bulk_wait_read1();             // the slot's previous tile has been read
+          __syncwarp();
+          if (EPI == EPI_RESID) {
+            // fp32 rows of 64 B, 64-byte swizzle: 16-byte unit j of row r at j ^ ((r >> 1) & 3)
+            uint8_t* rp = slot + lane * 64;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              const float4 bb = b4[jj];
+              *reinterpret_cast<float4*>(rp + ((jj ^ ((lane >> 1) & 3)) << 4)) =
+                  make_float4(v[4 * jj] + bb.x, v[4 * jj + 1] + bb.y, v[4 * jj + 2] + bb.z, v[4 * jj + 3] + bb.w);
+            }
+          } else {
+            // bf16 rows of 32 B, 32-byte swizzle: 16-byte unit j of row r at j ^ ((r >> 2) & 1)
+            uint32_t pk[8];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              const float4 bb = b4[jj];
+              const float2 g0 = gelu2_as7126(fadd2(make_float2(v[4 * jj], v[4 * jj + 1]), make_float2(bb.x, bb.y)));
+              const float2 g1 = gelu2_as7126(fadd2(make_float2(v[4 * jj + 2], v[4 * jj + 3]), make_float2(bb.z, bb.w)));
+              __nv_bfloat162 lo = __floats2bfloat162_rn(g0.x, g0.y), hi = __floats2bfloat162_rn(g1.x, g1.y);
+              pk[2 * jj] = *reinterpret_cast<uint32_t*>(&lo);
+              pk[2 * jj + 1] = *reinterpret_cast<uint32_t*>(&hi);
+            }
+            uint8_t* rp = slot + lane * 32;
+            const int sw = (lane >> 2) & 1;
+            *reinterpret_cast<uint4*>(rp + (sw << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(rp + ((1 ^ sw) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) {
+            if (EPI == EPI_RESID) tma_reduce_add_2d(&tmC, smem_u32(slot), col, row0);
+            else tma_store_2d(&tmC, smem_u32(slot), col, row0);
+            bulk_commit();
+          }
+          ++cc;
+        }
+      }
+      if (lane == 0) bulk_wait_all();                   // the bulk writes are complete before the CTA exits
+      __syncwarp();
+    } else {
+      float* stg = sEpi + ew * 32 * 16;
+      const int rl = lane >> 2, cq = lane & 3;
+      const int sw_w = (lane >> 1) & 3;            // swizzle of the row this lane writes
+      const int sw_r = (rl >> 1) & 3;              // swizzle of the rows this lane reads
+      const Ctl* ctl = e.ctl;
+      const int R = ctl->R, p0 = ctl->p0;
+      int i = 0;
+      for (int t = unit; t < ntiles; t += nunits, ++i) {
+        const int acc = i & 1;
+        const uint32_t use = (uint32_t)(i >> 1);
+        const int mb = t % tiles_m, nb = t / tiles_m;
+        const int row0 = mb * TM + (int)rank * BM + q * 32;
+        const int n0 = nb * BN + hf * HALF;
+        const uint32_t taddr = tmem + (uint32_t)(acc * BN + hf * HALF) + ((uint32_t)(q * 32) << 16);
+        // per-tile row info for the 4 rows this lane stores
+        char* rowp[4];
+        const float* pos_s[4];
+        const float* pos_t[4];
+        int colbase = 0;
+  #pragma unroll
+        for (int it = 0; it < 4; ++it) {
+          const int r = row0 + it * 8 + rl;
+          if (EPI == EPI_RESID) rowp[it] = reinterpret_cast<char*>(e.h + (size_t)r * e.d);
+          if (EPI == EPI_GELU) rowp[it] = reinterpret_cast<char*>(reinterpret_cast<bf16*>(e.out) + (size_t)r * e.ldo);
+          if (EPI == EPI_INPROJ || EPI == EPI_QKV) {
+            const int sm = r / R;
+            const int p = p0 + (r - sm * R);
+            if (EPI == EPI_INPROJ) {
+              rowp[it] = reinterpret_cast<char*>(e.h + (size_t)r * e.d);
+              pos_s[it] = e.pos_space + (size_t)(p % e.frame_len) * e.d;
+              pos_t[it] = e.pos_time + (size_t)(p / e.frame_len) * e.d;
+            } else {
+              const int which = (nb * BN) / e.d;            // the whole tile is q, k or v
+              if (which == 0) rowp[it] = reinterpret_cast<char*>(reinterpret_cast<bf16*>(e.out) + (size_t)r * e.d);
+              else
+                rowp[it] = reinterpret_cast<char*>(reinterpret_cast<bf16*>(which == 1 ? e.kc : e.vc) +
+                                                   ((size_t)sm * e.Lc + p) * e.d);
+              colbase = which * e.d;
+            }
+          }
+        }
+        // head: one row per thread, hoisted (sample, position, token) and row pointers
+        bool head_out = false, head_act = false;
+        const float* hin = nullptr;
+        float* hout = nullptr;
+        float* hpart = nullptr;
+        if (EPI == EPI_HEAD) {
+          const int r = row0 + lane;
           const int sm = r / R;
           const int p = p0 + (r - sm * R);
-          if (EPI == EPI_INPROJ) {
-            rowp[it] = reinterpret_cast<char*>(e.h + (size_t)r * e.d);
-            pos_s[it] = e.pos_space + (size_t)(p % e.frame_len) * e.d;
-            pos_t[it] = e.pos_time + (size_t)(p / e.frame_len) * e.d;
-          } else {
-            const int which = (nb * BN) / e.d;            // the whole tile is q, k or v
-            if (which == 0) rowp[it] = reinterpret_cast<char*>(reinterpret_cast<bf16*>(e.out) + (size_t)r * e.d);
-            else
-              rowp[it] = reinterpret_cast<char*>(reinterpret_cast<bf16*>(which == 1 ? e.kc : e.vc) +
-                                                 ((size_t)sm * e.Lc + p) * e.d);
-            colbase = which * e.d;
-          }
+          head_out = r < M && p >= ctl->P;
+          const size_t base = ((size_t)sm * e.L + tok_of(p, e.L, e.dir)) * e.C;
+          hin = e.xin_f + base;
+          hout = e.xout_f + base;
+          hpart = e.part + (size_t)r * ((2 * e.C) >> 4) * 2;
+          head_act = head_out && (e.head_mode == 0 || e.active[sm]);
         }
-      }
-      // head: one row per thread, hoisted (sample, position, token) and row pointers
-      bool head_out = false, head_act = false;
-      const float* hin = nullptr;
-      float* hout = nullptr;
-      float* hpart = nullptr;
-      if (EPI == EPI_HEAD) {
-        const int r = row0 + lane;
-        const int sm = r / R;
-        const int p = p0 + (r - sm * R);
-        head_out = r < M && p >= ctl->P;
-        const size_t base = ((size_t)sm * e.L + tok_of(p, e.L, e.dir)) * e.C;
-        hin = e.xin_f + base;
-        hout = e.xout_f + base;
-        hpart = e.part + (size_t)r * ((2 * e.C) >> 4) * 2;
-        head_act = head_out && (e.head_mode == 0 || e.active[sm]);
-      }
-      // Loads that do not depend on the accumulator are issued before waiting
-      // for it (bias, and the first chunk's residual / position rows), and
-      // every chunk's TMEM load and global loads are in flight while the
-      // previous chunk is transposed and stored.
-      constexpr int NCH = HALF / 16;
-      float4 bias4[NCH];
-#pragma unroll
-      for (int k = 0; k < NCH; ++k) bias4[k] = *reinterpret_cast<const float4*>(e.bias + n0 + k * 16 + cq * 4);
-      float4 pre[2][4], pre2[2][4];
-      auto load_rows = [&](int k, float4* dst, float4* dst2) {
-        if (EPI == EPI_HEAD) {
-          if (head_act) {
-            const int c0 = (n0 + k * 16) >> 1;
-            dst[0] = *reinterpret_cast<const float4*>(hin + c0);
-            dst[1] = *reinterpret_cast<const float4*>(hin + c0 + 4);
-            if (e.head_mode == 1) {
-              dst2[0] = *reinterpret_cast<const float4*>(hout + c0);
-              dst2[1] = *reinterpret_cast<const float4*>(hout + c0 + 4);
+        // Loads that do not depend on the accumulator are issued before waiting
+        // for it (bias, and the first chunk's residual / position rows), and
+        // every chunk's TMEM load and global loads are in flight while the
+        // previous chunk is transposed and stored.
+        constexpr int NCH = HALF / 16;
+        float4 bias4[NCH];
+  #pragma unroll
+        for (int k = 0; k < NCH; ++k) bias4[k] = *reinterpret_cast<const float4*>(e.bias + n0 + k * 16 + cq * 4);
+        float4 pre[2][4], pre2[2][4];
+        auto load_rows = [&](int k, float4* dst, float4* dst2) {
+          if (EPI == EPI_HEAD) {
+            if (head_act) {
+              const int c0 = (n0 + k * 16) >> 1;
+              dst[0] = *reinterpret_cast<const float4*>(hin + c0);
+              dst[1] = *reinterpret_cast<const float4*>(hin + c0 + 4);
+              if (e.head_mode == 1) {
+                dst2[0] = *reinterpret_cast<const float4*>(hout + c0);
+                dst2[1] = *reinterpret_cast<const float4*>(hout + c0 + 4);
+              }
             }
+            return;
           }
-          return;
-        }
-        const int col = n0 + k * 16 + cq * 4;
-#pragma unroll
-        for (int it = 0; it < 4; ++it) {
-          if (row0 + it * 8 + rl < M) {
-            if (EPI == EPI_RESID) dst[it] = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(rowp[it]) + col);
-            if (EPI == EPI_INPROJ) {
-              dst[it] = *reinterpret_cast<const float4*>(pos_s[it] + col);
-              dst2[it] = *reinterpret_cast<const float4*>(pos_t[it] + col);
-            }
-          }
-        }
-      };
-      if (EPI == EPI_RESID || EPI == EPI_INPROJ || EPI == EPI_HEAD) load_rows(0, pre[0], pre2[0]);
-      // the wait's outcome is made warp-uniform before the .aligned TMEM loads
-      if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * acc, use & 1u, abort_flag))) break;
-      tc_fence_after();
-      float vb[2][16];
-      tmem_ld16(taddr, vb[0]);
-#pragma unroll
-      for (int k = 0; k < NCH; ++k) {
-        const int c = k * 16;
-        tmem_wait_ld();
-        if (k + 1 < NCH) {
-          tmem_ld16(taddr + c + 16, vb[(k + 1) & 1]);
-          if (EPI == EPI_RESID || EPI == EPI_INPROJ || EPI == EPI_HEAD) load_rows(k + 1, pre[(k + 1) & 1], pre2[(k + 1) & 1]);
-        }
-        const float* v = vb[k & 1];
-        if (EPI == EPI_HEAD) {
-          // 8 channels whose (mu_c, s_c) sit at columns (2c, 2c+1)
-          const int col0 = n0 + c;
-          float2* part = reinterpret_cast<float2*>(hpart) + (col0 >> 4);
-          if (!head_out) continue;
-          if (!head_act) { *part = make_float2(0.f, 0.f); continue; }
-          const float* xi = reinterpret_cast<const float*>(pre[k & 1]);
-          float r8[8];
-          float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            const float mu = v[2 * jj] + e.bias[col0 + 2 * jj];
-            const float sl = v[2 * jj + 1] + e.bias[col0 + 2 * jj + 1];
-            if (e.head_mode == 0) {
-              r8[jj] = (xi[jj] - mu) * expf(-sl);            // z = (x - mu) exp(-s)
-              a0 += sl;
-            } else {
-              r8[jj] = fmaf(expf(sl), xi[jj], mu);           // x_new = mu + exp(s) z
-              const float dx = r8[jj] - reinterpret_cast<const float*>(pre2[k & 1])[jj];
-              a0 = fmaf(dx, dx, a0);
-              a1 = fmaf(r8[jj], r8[jj], a1);
-            }
-          }
-          const int c0 = col0 >> 1;
-          *reinterpret_cast<float4*>(hout + c0) = make_float4(r8[0], r8[1], r8[2], r8[3]);
-          *reinterpret_cast<float4*>(hout + c0 + 4) = make_float4(r8[4], r8[5], r8[6], r8[7]);
-          *part = make_float2(a0, a1);
-          continue;
-        }
-        float4* srow = reinterpret_cast<float4*>(stg + lane * 16);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) srow[j ^ sw_w] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-        __syncwarp();
-        float4 a[4];
-#pragma unroll
-        for (int it = 0; it < 4; ++it) a[it] = reinterpret_cast<const float4*>(stg + (it * 8 + rl) * 16)[cq ^ sw_r];
-        __syncwarp();
-        const int col = n0 + c + cq * 4;
-        const float4 bb = bias4[k];
-        if (EPI == EPI_RESID) {
-#pragma unroll
+          const int col = n0 + k * 16 + cq * 4;
+  #pragma unroll
           for (int it = 0; it < 4; ++it) {
             if (row0 + it * 8 + rl < M) {
-              float4 hv = pre[k & 1][it];
-              hv.x += a[it].x + bb.x; hv.y += a[it].y + bb.y;
-              hv.z += a[it].z + bb.z; hv.w += a[it].w + bb.w;
-              *reinterpret_cast<float4*>(reinterpret_cast<float*>(rowp[it]) + col) = hv;
+              if (EPI == EPI_RESID) dst[it] = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(rowp[it]) + col);
+              if (EPI == EPI_INPROJ) {
+                dst[it] = *reinterpret_cast<const float4*>(pos_s[it] + col);
+                dst2[it] = *reinterpret_cast<const float4*>(pos_t[it] + col);
+              }
             }
           }
-        } else if (EPI == EPI_INPROJ) {
-#pragma unroll
-          for (int it = 0; it < 4; ++it) {
-            if (row0 + it * 8 + rl < M) {
-              const float4 ps = pre[k & 1][it], pt = pre2[k & 1][it];
-              *reinterpret_cast<float4*>(reinterpret_cast<float*>(rowp[it]) + col) =
-                  make_float4(a[it].x + bb.x + ps.x + pt.x, a[it].y + bb.y + ps.y + pt.y,
-                              a[it].z + bb.z + ps.z + pt.z, a[it].w + bb.w + ps.w + pt.w);
-            }
+        };
+        if (EPI == EPI_RESID || EPI == EPI_INPROJ || EPI == EPI_HEAD) load_rows(0, pre[0], pre2[0]);
+        // the wait's outcome is made warp-uniform before the .aligned TMEM loads
+        if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * acc, use & 1u, abort_flag))) break;
+        tc_fence_after();
+        float vb[2][16];
+        tmem_ld16(taddr, vb[0]);
+  #pragma unroll
+        for (int k = 0; k < NCH; ++k) {
+          const int c = k * 16;
+          tmem_wait_ld();
+          if (k + 1 < NCH) {
+            tmem_ld16(taddr + c + 16, vb[(k + 1) & 1]);
+            if (EPI == EPI_RESID || EPI == EPI_INPROJ || EPI == EPI_HEAD) load_rows(k + 1, pre[(k + 1) & 1], pre2[(k + 1) & 1]);
           }
-        } else if (EPI == EPI_GELU) {
-#pragma unroll
-          for (int it = 0; it < 4; ++it) {
-            if (row0 + it * 8 + rl < M) {
-              const float2 g0 = gelu2_as7126(fadd2(make_float2(a[it].x, a[it].y), make_float2(bb.x, bb.y)));
-              const float2 g1 = gelu2_as7126(fadd2(make_float2(a[it].z, a[it].w), make_float2(bb.z, bb.w)));
-              st_bf16x4(reinterpret_cast<bf16*>(rowp[it]) + col, g0.x, g0.y, g1.x, g1.y);
+          const float* v = vb[k & 1];
+          if (EPI == EPI_HEAD) {
+            // 8 channels whose (mu_c, s_c) sit at columns (2c, 2c+1)
+            const int col0 = n0 + c;
+            float2* part = reinterpret_cast<float2*>(hpart) + (col0 >> 4);
+            if (!head_out) continue;
+            if (!head_act) { *part = make_float2(0.f, 0.f); continue; }
+            const float* xi = reinterpret_cast<const float*>(pre[k & 1]);
+            float r8[8];
+            float a0 = 0.f, a1 = 0.f;
+  #pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+              const float mu = v[2 * jj] + e.bias[col0 + 2 * jj];
+              const float sl = v[2 * jj + 1] + e.bias[col0 + 2 * jj + 1];
+              if (e.head_mode == 0) {
+                r8[jj] = (xi[jj] - mu) * expf(-sl);            // z = (x - mu) exp(-s)
+                a0 += sl;
+              } else {
+                r8[jj] = fmaf(expf(sl), xi[jj], mu);           // x_new = mu + exp(s) z
+                const float dx = r8[jj] - reinterpret_cast<const float*>(pre2[k & 1])[jj];
+                a0 = fmaf(dx, dx, a0);
+                a1 = fmaf(r8[jj], r8[jj], a1);
+              }
             }
+            const int c0 = col0 >> 1;
+            *reinterpret_cast<float4*>(hout + c0) = make_float4(r8[0], r8[1], r8[2], r8[3]);
+            *reinterpret_cast<float4*>(hout + c0 + 4) = make_float4(r8[4], r8[5], r8[6], r8[7]);
+            *part = make_float2(a0, a1);
+            continue;
           }
-        } else if (EPI == EPI_QKV) {
-#pragma unroll
-          for (int it = 0; it < 4; ++it)
-            if (row0 + it * 8 + rl < M)
-              st_bf16x4(reinterpret_cast<bf16*>(rowp[it]) + (col - colbase), a[it].x + bb.x, a[it].y + bb.y,
-                        a[it].z + bb.z, a[it].w + bb.w);
+          float4* srow = reinterpret_cast<float4*>(stg + lane * 16);
+  #pragma unroll
+          for (int j = 0; j < 4; ++j) srow[j ^ sw_w] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+          __syncwarp();
+          float4 a[4];
+  #pragma unroll
+          for (int it = 0; it < 4; ++it) a[it] = reinterpret_cast<const float4*>(stg + (it * 8 + rl) * 16)[cq ^ sw_r];
+          __syncwarp();
+          const int col = n0 + c + cq * 4;
+          const float4 bb = bias4[k];
+          if (EPI == EPI_RESID) {
+  #pragma unroll
+            for (int it = 0; it < 4; ++it) {
+              if (row0 + it * 8 + rl < M) {
+                float4 hv = pre[k & 1][it];
+                hv.x += a[it].x + bb.x; hv.y += a[it].y + bb.y;
+                hv.z += a[it].z + bb.z; hv.w += a[it].w + bb.w;
+                *reinterpret_cast<float4*>(reinterpret_cast<float*>(rowp[it]) + col) = hv;
+              }
+            }
+          } else if (EPI == EPI_INPROJ) {
+  #pragma unroll
+            for (int it = 0; it < 4; ++it) {
+              if (row0 + it * 8 + rl < M) {
+                const float4 ps = pre[k & 1][it], pt = pre2[k & 1][it];
+                *reinterpret_cast<float4*>(reinterpret_cast<float*>(rowp[it]) + col) =
+                    make_float4(a[it].x + bb.x + ps.x + pt.x, a[it].y + bb.y + ps.y + pt.y,
+                                a[it].z + bb.z + ps.z + pt.z, a[it].w + bb.w + ps.w + pt.w);
+              }
+            }
+          } else if (EPI == EPI_GELU) {
+  #pragma unroll
+            for (int it = 0; it < 4; ++it) {
+              if (row0 + it * 8 + rl < M) {
+                const float2 g0 = gelu2_as7126(fadd2(make_float2(a[it].x, a[it].y), make_float2(bb.x, bb.y)));
+                const float2 g1 = gelu2_as7126(fadd2(make_float2(a[it].z, a[it].w), make_float2(bb.z, bb.w)));
+                st_bf16x4(reinterpret_cast<bf16*>(rowp[it]) + col, g0.x, g0.y, g1.x, g1.y);
+              }
+            }
+          } else if (EPI == EPI_QKV) {
+  #pragma unroll
+            for (int it = 0; it < 4; ++it)
+              if (row0 + it * 8 + rl < M)
+                st_bf16x4(reinterpret_cast<bf16*>(rowp[it]) + (col - colbase), a[it].x + bb.x, a[it].y + bb.y,
+                          a[it].z + bb.z, a[it].w + bb.w);
+          }
         }
+        tc_fence_before();
+        if (CG == 2) mbar_arrive_cluster(tempty_lead + 8 * acc);
+        else mbar_arrive(tempty0 + 8 * acc);
       }
-      tc_fence_before();
-      if (CG == 2) mbar_arrive_cluster(tempty_lead + 8 * acc);
-      else mbar_arrive(tempty0 + 8 * acc);
     }
   }
   tc_fence_before();
@@ -579,7 +687,8 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
 }
 
 template <int BN, int EPI, int CG>
-void launch_bn_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, int N, int K, int m_max, const EpiArgs& e,
+void launch_bn_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmC, int N, int K, int m_max,
+                   const EpiArgs& e,
                    int* err, int num_sms, cudaStream_t st) {
   using Cfg = TcCfg<BN, CG, EPI>;
   static int max_units = 0;
@@ -605,7 +714,7 @@ void launch_bn_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, int N, int K,
   const int tiles = ((m_max + BM * CG - 1) / (BM * CG)) * (N / BN);
   const int units = tiles < max_units ? tiles : max_units;
   if (CG == 1) {
-    launch_k(k_gemm_tc<BN, EPI, 1>, dim3(units), dim3(Cfg::THREADS), Cfg::SMEM, st, tmA, tmB, N, K, e, err);
+    launch_k(k_gemm_tc<BN, EPI, 1>, dim3(units), dim3(Cfg::THREADS), Cfg::SMEM, st, tmA, tmB, tmC, N, K, e, err);
   } else {
     cudaLaunchConfig_t c = {};
     c.gridDim = dim3(2 * units);
@@ -619,19 +728,19 @@ void launch_bn_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, int N, int K,
     a[1].val.programmaticStreamSerializationAllowed = g_pdl;
     c.attrs = a;
     c.numAttrs = 2;
-    cudaLaunchKernelEx(&c, k_gemm_tc<BN, EPI, CG>, tmA, tmB, N, K, e, err);
+    cudaLaunchKernelEx(&c, k_gemm_tc<BN, EPI, CG>, tmA, tmB, tmC, N, K, e, err);
   }
 }
 
 template <int BN, int CG>
-void launch_bn(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, int N, int K, int m_max,
+void launch_bn(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmC, int N, int K, int m_max,
                const EpiArgs& e, int* err, int num_sms, cudaStream_t st) {
   switch (epi) {
-    case EPI_INPROJ: launch_bn_epi<BN, EPI_INPROJ, CG>(tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
-    case EPI_QKV: launch_bn_epi<BN, EPI_QKV, CG>(tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
-    case EPI_RESID: launch_bn_epi<BN, EPI_RESID, CG>(tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
-    case EPI_GELU: launch_bn_epi<BN, EPI_GELU, CG>(tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
-    default: launch_bn_epi<BN, EPI_HEAD, CG>(tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
+    case EPI_INPROJ: launch_bn_epi<BN, EPI_INPROJ, CG>(tmA, tmB, tmC, N, K, m_max, e, err, num_sms, st); break;
+    case EPI_QKV: launch_bn_epi<BN, EPI_QKV, CG>(tmA, tmB, tmC, N, K, m_max, e, err, num_sms, st); break;
+    case EPI_RESID: launch_bn_epi<BN, EPI_RESID, CG>(tmA, tmB, tmC, N, K, m_max, e, err, num_sms, st); break;
+    case EPI_GELU: launch_bn_epi<BN, EPI_GELU, CG>(tmA, tmB, tmC, N, K, m_max, e, err, num_sms, st); break;
+    default: launch_bn_epi<BN, EPI_HEAD, CG>(tmA, tmB, tmC, N, K, m_max, e, err, num_sms, st); break;
   }
 }
 
@@ -661,6 +770,20 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int rows, int cols, int 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tmap_out(CUtensorMap* map, const void* base, bool f32, int rows, int cols) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const int es = f32 ? 4 : 2;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * es};
+  cuuint32_t box[2] = {16u, 32u};
+  cuuint32_t estr[2] = {1u, 1u};
+  return fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            f32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Tile shape: SM-pair MMAs (256-row tiles) when there are at least 256 rows,
 // and the width (<= max_bn, dividing N, and `unit` when non-zero) with the fewest waves of
 // work, ceil(tiles / units) * BN; ties go to the wider tile.  Returns
@@ -680,20 +803,22 @@ int gemm_tc_pick(int N, int m_max, int num_sms, int unit, int max_bn) {
   return best ? best * 10 + cg : 0;
 }
 
-void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, int pick, int N, int K, int m_max,
+void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap* tmC, int pick, int N,
+                    int K, int m_max,
                     const EpiArgs& e, int* err, int num_sms, cudaStream_t st) {
   const int bn = pick / 10, cg = pick % 10;
+  const CUtensorMap& tmC_ = tmC ? *tmC : tmA;                // only the TMA epilogues read it
   if (cg == 2) {
     switch (bn) {
-      case 256: launch_bn<256, 2>(epi, tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
-      case 192: launch_bn<192, 2>(epi, tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
-      default: launch_bn<128, 2>(epi, tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
+      case 256: launch_bn<256, 2>(epi, tmA, tmB, tmC_, N, K, m_max, e, err, num_sms, st); break;
+      case 192: launch_bn<192, 2>(epi, tmA, tmB, tmC_, N, K, m_max, e, err, num_sms, st); break;
+      default: launch_bn<128, 2>(epi, tmA, tmB, tmC_, N, K, m_max, e, err, num_sms, st); break;
     }
   } else {
     switch (bn) {
-      case 256: launch_bn<256, 1>(epi, tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
-      case 192: launch_bn<192, 1>(epi, tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
-      default: launch_bn<128, 1>(epi, tmA, tmB, N, K, m_max, e, err, num_sms, st); break;
+      case 256: launch_bn<256, 1>(epi, tmA, tmB, tmC_, N, K, m_max, e, err, num_sms, st); break;
+      case 192: launch_bn<192, 1>(epi, tmA, tmB, tmC_, N, K, m_max, e, err, num_sms, st); break;
+      default: launch_bn<128, 1>(epi, tmA, tmB, tmC_, N, K, m_max, e, err, num_sms, st); break;
     }
   }
 }

@@ -61,11 +61,15 @@ void launch_attn_simt(const Ctl* ctl, const float* q, const float* kc, const flo
 // TMA descriptor of a row-major bf16 matrix [rows, cols] tiled as boxes of
 // [box_rows, 64 columns] with 128-byte swizzle (af_gemm_tc.cu).
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int rows, int cols, int box_rows);
+// TMA descriptor of the output of a TMA epilogue: fp32 h or bf16 u [rows, cols]
+// in boxes of 32 rows x 16 columns, 64-byte (fp32) or 32-byte (bf16) swizzle.
+bool make_tmap_out(CUtensorMap* map, const void* base, bool f32, int rows, int cols);
 // C[M, N] = A[M, K] W[N, K]^T with epilogue `epi`, K % 64 == 0.  `pick` =
 // BN * 10 + CG from gemm_tc_pick (N % BN == 0); tmA boxes are 128 rows, tmB
-// boxes BN / CG rows.
-void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, int pick, int N, int K,
-                    int m_max, const EpiArgs& e, int* err, int num_sms, cudaStream_t st);
+// boxes BN / CG rows; tmC (make_tmap_out) is the output of EPI_RESID (h) and
+// EPI_GELU (u), unused (may be null) otherwise.
+void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap* tmC, int pick,
+                    int N, int K, int m_max, const EpiArgs& e, int* err, int num_sms, cudaStream_t st);
 int gemm_tc_pick(int N, int m_max, int num_sms, int unit, int max_bn);
 
 // Causal attention over the KV cache on tcgen05 (af_attn_tc.cu).  nsplit key
