@@ -216,18 +216,19 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
     bf16* q = (bf16*)b.q;
     bf16* u = (bf16*)b.u;
     const int ns = m->num_sms;
-    CUtensorMap tA_x, tA_a, tA_u, tB, tC_h, tC_u;
+    CUtensorMap tA_x, tA_a, tA_u, tB, tC_h, tC_u, tC_q, tC_k, tC_v;
     bool ok = make_tmap_bf16(&tA_x, xin, m_max, C, 128) && make_tmap_bf16(&tA_a, a, m_max, d, 128) &&
               make_tmap_bf16(&tA_u, u, m_max, fd, 128) && make_tmap_out(&tC_h, b.h, true, m_max, d) &&
-              make_tmap_out(&tC_u, u, false, m_max, fd);
+              make_tmap_out(&tC_u, u, false, m_max, fd) && make_tmap_out(&tC_q, q, false, m_max, d);
     if (!ok) { set_err("cuTensorMapEncodeTiled failed for an activation"); return AF_ERR_CUDA; }
     auto gemm = [&](int epi, const CUtensorMap& tA, const void* W, int N, int K, const EpiArgs& ea) -> bool {
       // a QKV tile must fall inside one of q, k, v; the position-add epilogue
       // keeps two row sets in flight and stays at <= 192 columns
       const int pick = gemm_tc_pick(N, m_max, ns, epi == EPI_QKV ? d : 0, epi == EPI_INPROJ ? 192 : 256);
       if (!pick || !make_tmap_bf16(&tB, W, N, K, (pick / 10) / (pick % 10))) return false;
-      const CUtensorMap* tC = epi == EPI_RESID ? &tC_h : (epi == EPI_GELU ? &tC_u : nullptr);
-      launch_gemm_tc(epi, tA, tB, tC, pick, N, K, m_max, ea, m->d_err, ns, st);
+      const CUtensorMap* tC = epi == EPI_RESID ? &tC_h : (epi == EPI_GELU ? &tC_u : (epi == EPI_QKV ? &tC_q : nullptr));
+      launch_gemm_tc(epi, tA, tB, tC, epi == EPI_QKV ? &tC_k : nullptr, epi == EPI_QKV ? &tC_v : nullptr, pick, N, K,
+                     m_max, ea, m->d_err, ns, st);
       return true;
     };
     launch_gather<bf16>(b.ctl, xsrc, L, C, dir, xin, m_max, st);
@@ -242,6 +243,10 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
       eq.out = q;
       eq.kc = kvl;
       eq.vc = kvl + kv_layer;
+      if (!make_tmap_out(&tC_k, kvl, false, batch * L, d) || !make_tmap_out(&tC_v, kvl + kv_layer, false, batch * L, d)) {
+        set_err("cuTensorMapEncodeTiled failed for the KV cache");
+        return AF_ERR_CUDA;
+      }
       if (!gemm(EPI_QKV, tA_a, w.w_qkv, 3 * d, d, eq)) { set_err("GEMM plan failed (qkv)"); return AF_ERR_CUDA; }
       if (!launch_attn_tc2(b.ctl, q, (const bf16*)kvl, (const bf16*)(kvl + kv_layer), a, b.opart, b.mlpart, b.nsplit,
                            batch, L, d, c.heads, r_max, m_max, m->d_err, st)) {

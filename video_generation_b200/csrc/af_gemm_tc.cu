@@ -34,10 +34,10 @@ constexpr int BM = 128, BK = 64;
 template <int EPI> struct EpiShape {
   static constexpr int WARPS = (EPI == EPI_RESID || EPI == EPI_INPROJ) ? 8 : 16;
   static constexpr int THREADS = (4 + WARPS) * 32;
-  // residual add and GELU leave through TMA: each warp stages 32 rows x 16
-  // columns (two slots, alternating) in the output tensor map's swizzle and
-  // issues a bulk reduce-add (h += tile) or a bulk store (u = tile)
-  static constexpr bool TMA_OUT = EPI == EPI_RESID || EPI == EPI_GELU;
+  // residual add, GELU and QKV leave through TMA: each warp stages 32 rows x
+  // 16 columns (two slots, alternating) in the output tensor map's swizzle and
+  // issues a bulk reduce-add (h += tile) or a bulk store (u, q, K / V cache)
+  static constexpr bool TMA_OUT = EPI == EPI_RESID || EPI == EPI_GELU || EPI == EPI_QKV;
   static constexpr uint32_t SLOT = EPI == EPI_RESID ? 32 * 16 * 4 : 32 * 16 * 2;
 };
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -248,7 +248,8 @@ __device__ __forceinline__ void st_bf16x4(bf16* dst, float a, float b, float c, 
 template <int BN, int EPI, int CG>
 __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-              const __grid_constant__ CUtensorMap tmC, int N, int K, EpiArgs e, int* err) {
+              const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
+              const __grid_constant__ CUtensorMap tmC3, int N, int K, EpiArgs e, int* err) {
   using Cfg = TcCfg<BN, CG, EPI>;
   constexpr int S = Cfg::STAGES;
   constexpr int TM = BM * CG;               // accumulator rows per tile (both CTAs)
@@ -289,6 +290,10 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
     if (EpiShape<EPI>::TMA_OUT) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmC)) : "memory");
+    if (EPI == EPI_QKV) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmC2)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmC3)) : "memory");
+    }
   }
   if (warp == 1) {
     if (CG == 2) {
@@ -412,11 +417,15 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
       // GELU) and is written, in the output tensor map's swizzle, to one of the
       // warp's two staging slots; lane 0 then sends the 32 x 16 tile with a TMA
       // bulk reduce-add into h (each element gets exactly one add, so the result
-      // is deterministic) or a bulk store into u.  Rows past the last real row
-      // land in workspace rows no kernel reads; rows past the buffer are clipped.
+      // is deterministic) or a bulk store into u or q.  Rows past the last real
+      // row land in workspace rows no kernel reads; rows past the buffer are
+      // clipped.  K and V rows go to the cache at (sample, position): a warp's
+      // 32 rows are one TMA store when they lie in one sample, else each thread
+      // stores its row (a few slices per call straddle two samples).
       constexpr uint32_t SLOT = EpiShape<EPI>::SLOT;
       constexpr int NCH = HALF / 16;
       uint8_t* stg0 = reinterpret_cast<uint8_t*>(sEpi) + ew * 2 * SLOT;
+      const int R = e.ctl->R, p0 = e.ctl->p0;
       int cc = 0;                                       // chunks sent by this warp
       int i = 0;
       for (int t = unit; t < ntiles; t += nunits, ++i) {
@@ -426,6 +435,17 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
         const int row0 = mb * TM + (int)rank * BM + q * 32;
         const int n0 = nb * BN + hf * HALF;
         const uint32_t taddr = tmem + (uint32_t)(acc * BN + hf * HALF) + ((uint32_t)(q * 32) << 16);
+        // QKV: the tile lies in one of q, K, V (BN divides d); where its rows go
+        int which = 0, ycache = 0;
+        bool tma_ok = true;                             // warp-uniform
+        if (EPI == EPI_QKV) {
+          which = (nb * BN) / e.d;
+          if (which > 0) {
+            const int s0 = row0 / R;
+            tma_ok = row0 + 31 < M && (row0 + 31) / R == s0;
+            ycache = s0 * e.Lc + p0 + (row0 - s0 * R);
+          }
+        }
         // the wait's outcome is made warp-uniform before the .aligned TMEM loads
         if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * acc, use & 1u, abort_flag))) break;
         tc_fence_after();
@@ -463,25 +483,42 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
               const float4 bb = b4[jj];
-              const float2 g0 = gelu2_as7126(fadd2(make_float2(v[4 * jj], v[4 * jj + 1]), make_float2(bb.x, bb.y)));
-              const float2 g1 = gelu2_as7126(fadd2(make_float2(v[4 * jj + 2], v[4 * jj + 3]), make_float2(bb.z, bb.w)));
+              float2 g0 = fadd2(make_float2(v[4 * jj], v[4 * jj + 1]), make_float2(bb.x, bb.y));
+              float2 g1 = fadd2(make_float2(v[4 * jj + 2], v[4 * jj + 3]), make_float2(bb.z, bb.w));
+              if (EPI == EPI_GELU) {
+                g0 = gelu2_as7126(g0);
+                g1 = gelu2_as7126(g1);
+              }
               __nv_bfloat162 lo = __floats2bfloat162_rn(g0.x, g0.y), hi = __floats2bfloat162_rn(g1.x, g1.y);
               pk[2 * jj] = *reinterpret_cast<uint32_t*>(&lo);
               pk[2 * jj + 1] = *reinterpret_cast<uint32_t*>(&hi);
             }
-            uint8_t* rp = slot + lane * 32;
-            const int sw = (lane >> 2) & 1;
-            *reinterpret_cast<uint4*>(rp + (sw << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            *reinterpret_cast<uint4*>(rp + ((1 ^ sw) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            if (tma_ok) {
+              uint8_t* rp = slot + lane * 32;
+              const int sw = (lane >> 2) & 1;
+              *reinterpret_cast<uint4*>(rp + (sw << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              *reinterpret_cast<uint4*>(rp + ((1 ^ sw) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            } else if (row0 + lane < M) {
+              // a K / V slice straddling two samples: this thread's row, direct
+              const int r = row0 + lane, sm = r / R;
+              bf16* cache = reinterpret_cast<bf16*>(which == 1 ? e.kc : e.vc);
+              uint4* dst = reinterpret_cast<uint4*>(cache + ((size_t)sm * e.Lc + p0 + (r - sm * R)) * e.d +
+                                                    (col - which * e.d));
+              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
           }
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          __syncwarp();
-          if (lane == 0) {
-            if (EPI == EPI_RESID) tma_reduce_add_2d(&tmC, smem_u32(slot), col, row0);
-            else tma_store_2d(&tmC, smem_u32(slot), col, row0);
-            bulk_commit();
+          if (tma_ok) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
+              if (EPI == EPI_RESID) tma_reduce_add_2d(&tmC, smem_u32(slot), col, row0);
+              else if (EPI == EPI_GELU || which == 0) tma_store_2d(&tmC, smem_u32(slot), col - which * e.d, row0);
+              else tma_store_2d(which == 1 ? &tmC2 : &tmC3, smem_u32(slot), col - which * e.d, ycache);
+              bulk_commit();
+            }
+            ++cc;
           }
-          ++cc;
         }
       }
       if (lane == 0) bulk_wait_all();                   // the bulk writes are complete before the CTA exits
@@ -687,8 +724,8 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
 }
 
 template <int BN, int EPI, int CG>
-void launch_bn_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmC, int N, int K, int m_max,
-                   const EpiArgs& e,
+void launch_bn_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmC, const CUtensorMap& tmC2,
+                   const CUtensorMap& tmC3, int N, int K, int m_max, const EpiArgs& e,
                    int* err, int num_sms, cudaStream_t st) {
   using Cfg = TcCfg<BN, CG, EPI>;
   static int max_units = 0;
@@ -714,7 +751,7 @@ void launch_bn_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtenso
   const int tiles = ((m_max + BM * CG - 1) / (BM * CG)) * (N / BN);
   const int units = tiles < max_units ? tiles : max_units;
   if (CG == 1) {
-    launch_k(k_gemm_tc<BN, EPI, 1>, dim3(units), dim3(Cfg::THREADS), Cfg::SMEM, st, tmA, tmB, tmC, N, K, e, err);
+    launch_k(k_gemm_tc<BN, EPI, 1>, dim3(units), dim3(Cfg::THREADS), Cfg::SMEM, st, tmA, tmB, tmC, tmC2, tmC3, N, K, e, err);
   } else {
     cudaLaunchConfig_t c = {};
     c.gridDim = dim3(2 * units);
@@ -728,19 +765,20 @@ void launch_bn_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtenso
     a[1].val.programmaticStreamSerializationAllowed = g_pdl;
     c.attrs = a;
     c.numAttrs = 2;
-    cudaLaunchKernelEx(&c, k_gemm_tc<BN, EPI, CG>, tmA, tmB, tmC, N, K, e, err);
+    cudaLaunchKernelEx(&c, k_gemm_tc<BN, EPI, CG>, tmA, tmB, tmC, tmC2, tmC3, N, K, e, err);
   }
 }
 
 template <int BN, int CG>
-void launch_bn(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmC, int N, int K, int m_max,
+void launch_bn(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmC, const CUtensorMap& tmC2,
+               const CUtensorMap& tmC3, int N, int K, int m_max,
                const EpiArgs& e, int* err, int num_sms, cudaStream_t st) {
   switch (epi) {
-    case EPI_INPROJ: launch_bn_epi<BN, EPI_INPROJ, CG>(tmA, tmB, tmC, N, K, m_max, e, err, num_sms, st); break;
-    case EPI_QKV: launch_bn_epi<BN, EPI_QKV, CG>(tmA, tmB, tmC, N, K, m_max, e, err, num_sms, st); break;
-    case EPI_RESID: launch_bn_epi<BN, EPI_RESID, CG>(tmA, tmB, tmC, N, K, m_max, e, err, num_sms, st); break;
-    case EPI_GELU: launch_bn_epi<BN, EPI_GELU, CG>(tmA, tmB, tmC, N, K, m_max, e, err, num_sms, st); break;
-    default: launch_bn_epi<BN, EPI_HEAD, CG>(tmA, tmB, tmC, N, K, m_max, e, err, num_sms, st); break;
+    case EPI_INPROJ: launch_bn_epi<BN, EPI_INPROJ, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st); break;
+    case EPI_QKV: launch_bn_epi<BN, EPI_QKV, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st); break;
+    case EPI_RESID: launch_bn_epi<BN, EPI_RESID, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st); break;
+    case EPI_GELU: launch_bn_epi<BN, EPI_GELU, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st); break;
+    default: launch_bn_epi<BN, EPI_HEAD, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st); break;
   }
 }
 
@@ -785,40 +823,47 @@ bool make_tmap_out(CUtensorMap* map, const void* base, bool f32, int rows, int c
 }
 
 // Tile shape: SM-pair MMAs (256-row tiles) when there are at least 256 rows,
-// and the width (<= max_bn, dividing N, and `unit` when non-zero) with the fewest waves of
-// work, ceil(tiles / units) * BN; ties go to the wider tile.  Returns
-// BN * 10 + CG.
+// and the width (<= max_bn, dividing N, and `unit` when non-zero) with the
+// least work per unit, ceil(tiles / units) * BN, weighted by the shared-memory
+// traffic a narrower tile spends per flop (operand bytes per MMA flop grow as
+// 1/BN + 1/256: x1.15 at 192, x1.3 at 128, a measured trade-off against wave
+// quantisation); ties go to the wider tile.  Returns BN * 10 + CG.
 int gemm_tc_pick(int N, int m_max, int num_sms, int unit, int max_bn) {
   const int cands[3] = {256, 192, 128};
+  const int weight[3] = {100, 115, 130};
   const int cg = m_max >= 256 ? 2 : 1;
   const int units = num_sms / cg;
   int best = 0;
   long long best_cost = 0;
-  for (int bn : cands) {
+  for (int i = 0; i < 3; ++i) {
+    const int bn = cands[i];
     if (N % bn || (unit && unit % bn) || bn > max_bn) continue;
     const long long tiles = (long long)((m_max + BM * cg - 1) / (BM * cg)) * (N / bn);
-    const long long cost = ((tiles + units - 1) / units) * bn;
+    const long long cost = ((tiles + units - 1) / units) * bn * weight[i];
     if (!best || cost < best_cost) { best = bn; best_cost = cost; }
   }
   return best ? best * 10 + cg : 0;
 }
 
-void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap* tmC, int pick, int N,
-                    int K, int m_max,
+void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap* tmC,
+                    const CUtensorMap* tmC2, const CUtensorMap* tmC3, int pick, int N, int K, int m_max,
                     const EpiArgs& e, int* err, int num_sms, cudaStream_t st) {
   const int bn = pick / 10, cg = pick % 10;
-  const CUtensorMap& tmC_ = tmC ? *tmC : tmA;                // only the TMA epilogues read it
+  // only the TMA epilogues read them
+  const CUtensorMap& tmC_ = tmC ? *tmC : tmA;
+  const CUtensorMap& tmC2_ = tmC2 ? *tmC2 : tmA;
+  const CUtensorMap& tmC3_ = tmC3 ? *tmC3 : tmA;
   if (cg == 2) {
     switch (bn) {
-      case 256: launch_bn<256, 2>(epi, tmA, tmB, tmC_, N, K, m_max, e, err, num_sms, st); break;
-      case 192: launch_bn<192, 2>(epi, tmA, tmB, tmC_, N, K, m_max, e, err, num_sms, st); break;
-      default: launch_bn<128, 2>(epi, tmA, tmB, tmC_, N, K, m_max, e, err, num_sms, st); break;
+      case 256: launch_bn<256, 2>(epi, tmA, tmB, tmC_, tmC2_, tmC3_, N, K, m_max, e, err, num_sms, st); break;
+      case 192: launch_bn<192, 2>(epi, tmA, tmB, tmC_, tmC2_, tmC3_, N, K, m_max, e, err, num_sms, st); break;
+      default: launch_bn<128, 2>(epi, tmA, tmB, tmC_, tmC2_, tmC3_, N, K, m_max, e, err, num_sms, st); break;
     }
   } else {
     switch (bn) {
-      case 256: launch_bn<256, 1>(epi, tmA, tmB, tmC_, N, K, m_max, e, err, num_sms, st); break;
-      case 192: launch_bn<192, 1>(epi, tmA, tmB, tmC_, N, K, m_max, e, err, num_sms, st); break;
-      default: launch_bn<128, 1>(epi, tmA, tmB, tmC_, N, K, m_max, e, err, num_sms, st); break;
+      case 256: launch_bn<256, 1>(epi, tmA, tmB, tmC_, tmC2_, tmC3_, N, K, m_max, e, err, num_sms, st); break;
+      case 192: launch_bn<192, 1>(epi, tmA, tmB, tmC_, tmC2_, tmC3_, N, K, m_max, e, err, num_sms, st); break;
+      default: launch_bn<128, 1>(epi, tmA, tmB, tmC_, tmC2_, tmC3_, N, K, m_max, e, err, num_sms, st); break;
     }
   }
 }

@@ -66,10 +66,12 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int rows, int cols, int 
 bool make_tmap_out(CUtensorMap* map, const void* base, bool f32, int rows, int cols);
 // C[M, N] = A[M, K] W[N, K]^T with epilogue `epi`, K % 64 == 0.  `pick` =
 // BN * 10 + CG from gemm_tc_pick (N % BN == 0); tmA boxes are 128 rows, tmB
-// boxes BN / CG rows; tmC (make_tmap_out) is the output of EPI_RESID (h) and
-// EPI_GELU (u), unused (may be null) otherwise.
-void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap* tmC, int pick,
-                    int N, int K, int m_max, const EpiArgs& e, int* err, int num_sms, cudaStream_t st);
+// boxes BN / CG rows; tmC (make_tmap_out) is the output of EPI_RESID (h),
+// EPI_GELU (u) and EPI_QKV (q), tmC2 / tmC3 the K / V cache of EPI_QKV
+// ([batch * Lc, d]); unused ones may be null.
+void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap* tmC,
+                    const CUtensorMap* tmC2, const CUtensorMap* tmC3, int pick, int N, int K, int m_max,
+                    const EpiArgs& e, int* err, int num_sms, cudaStream_t st);
 int gemm_tc_pick(int N, int m_max, int num_sms, int unit, int max_bn);
 
 // Causal attention over the KV cache on tcgen05 (af_attn_tc.cu).  nsplit key
