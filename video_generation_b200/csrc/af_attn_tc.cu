@@ -54,11 +54,14 @@ template <int HD> struct AttnCfg {
   static constexpr uint32_t KV_BYTES = KCH * KVBOX;       // one K or one V tile
   // Per group: QB Q buffers (the next item's Q prefetched when two fit), a K
   // ring (a K tile is read only by its S = Q K^T), a V ring (held until P V)
-  // and two P tiles.
+  // and PB P tiles.
+  // hd 128 keeps one P tile, so that its V ring (the cache of a long video
+  // is read from HBM) can hold two tiles.
   static constexpr int QB = HD == 64 ? 2 : 1;
-  static constexpr int SK = 2, SV = HD == 64 ? 4 : 1;
+  static constexpr int PB = HD == 64 ? 2 : 1;
+  static constexpr int SK = 2, SV = HD == 64 ? 4 : 2;
   static constexpr uint32_t P_BYTES = QBOX;               // 128 rows x 64 keys
-  static constexpr uint32_t GROUP_BYTES = QB * Q_BYTES + (SK + SV) * KV_BYTES + 2 * P_BYTES;
+  static constexpr uint32_t GROUP_BYTES = QB * Q_BYTES + (SK + SV) * KV_BYTES + PB * P_BYTES;
   // barriers per group: QF[QB] QE[QB] KF[SK] KE[SK] VF[SV] VE[SV] SF SR PF[2] OD[2] OR DRAIN
   static constexpr int GBARS = 2 * QB + 2 * SK + 2 * SV + 8;
   static constexpr size_t SMEM = 1024 + 2 * (size_t)GROUP_BYTES + 2 * GBARS * 8;
@@ -168,6 +171,17 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// TMA bulk store of a staged tile (one thread), tracked as a bulk async-group.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(c0), "r"(c1)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 struct AttnArgs {
   const Ctl* ctl;
   bf16* o;           // [Mmax, d] output (nsplit == 1)
@@ -179,9 +193,10 @@ struct AttnArgs {
 template <int HD>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-              const __grid_constant__ CUtensorMap tmV, AttnArgs g, int* err) {
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, AttnArgs g,
+              int* err) {
   using Cfg = AttnCfg<HD>;
-  constexpr int BKV = Cfg::BKV, QB = Cfg::QB, SK = Cfg::SK, SV = Cfg::SV;
+  constexpr int BKV = Cfg::BKV, QB = Cfg::QB, PB = Cfg::PB, SK = Cfg::SK, SV = Cfg::SV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   __shared__ uint32_t s_tmem;
@@ -193,7 +208,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int grp = warp < 4 ? (warp >> 1) : ((warp - 4) >> 2);
   pdl_trigger();
 
-  // this group's shared memory: [Q buffers][K ring][V ring][2 P tiles]
+  // this group's shared memory: [Q buffers][K ring][V ring][P tiles]
   uint8_t* gs = smem + grp * Cfg::GROUP_BYTES;
   uint8_t* sQ = gs;
   uint8_t* sK = sQ + QB * Cfg::Q_BYTES;
@@ -318,10 +333,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int p_vst = 0, p_vph = 0, p_j = 0, p_iw = 0;
       bool ok = true;
       auto issue_pv = [&]() -> bool {
-        const int u = t - 1, pb = u & 1;
+        const int u = t - 1, pb = u % PB;
         // an item's first P*V overwrites O: the group has read the previous item's O
         if (p_j == 0 && p_iw >= 1 && !wait_fast(OR, (uint32_t)((p_iw - 1) & 1), abort_flag)) return false;
-        if (!wait_fast(PF + 8 * pb, (uint32_t)((u >> 1) & 1), abort_flag)) return false;
+        if (!wait_fast(PF + 8 * pb, (uint32_t)((u / PB) & 1), abort_flag)) return false;
         if (!wait_fast(VF + 8 * p_vst, (uint32_t)p_vph, abort_flag)) return false;
         tc_fence_after();
         const uint64_t a0 = dp + (uint64_t)(pb * (Cfg::P_BYTES >> 4));
@@ -365,9 +380,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (++vst == SV) { vst = 0; vph ^= 1u; }
           ++t;
         }
+        // the item's last P*V at once: the group's epilogue waits for it
+        if (ok && pend && !issue_pv()) ok = false;
+        pend = false;
         ++iw;
       }
-      if (ok && pend && !issue_pv()) ok = false;
       umma_commit(DRAIN);
       const uint64_t tw0 = globaltimer_ns();
       while (!mbar_try(DRAIN, 0)) {
@@ -386,6 +403,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint8_t* prow0 = sP + (q * 32 + lane) * 128;             // P row = TMEM lane
     const int sw = lane & 7;                                  // 128-byte swizzle of this row
     int tw = 0;                                               // tiles this group has consumed
+    int stg_buf = -1;                                         // P tile holding this warp's output staging
     bool alive = true;
     for (int k = w; alive; k += 2) {
       const int it = global_item(k);
@@ -450,12 +468,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             m_use = m_new;
           }
         }
-        // P tile tw % 2 is free once the group's P*V of tile tw - 2 has completed
-        const int pb = tw & 1;
-        if (tw >= 2 &&
-            !__all_sync(0xffffffffu, mbar_wait(OD + 8 * pb, (uint32_t)(((tw >> 1) - 1) & 1), abort_flag)))
+        // P tile tw % PB is free once the group's P*V of tile tw - PB has completed
+        const int pb = tw % PB;
+        if (tw >= PB &&
+            !__all_sync(0xffffffffu, mbar_wait(OD + 8 * pb, (uint32_t)(((tw / PB) - 1) & 1), abort_flag)))
           break;
         uint8_t* prow = prow0 + pb * Cfg::P_BYTES;
+        if (pb == stg_buf) {
+          // the output staging of the previous item must have been read by its TMA stores
+          if (lane == 0) bulk_wait_read0();
+          __syncwarp();
+          stg_buf = -1;
+        }
         if (wvalid) {
           // P = 2^(s * scale - m) in bf16, masked keys exactly 0
           const float2 nmb = splat((m_use == -INFINITY) ? 0.f : -m_use);
@@ -489,7 +513,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           // the max grew: rescale O, which must hold tiles 0..j-1, before this
           // tile's P*V is issued
           const int tl = tw - 1;
-          if (!__all_sync(0xffffffffu, mbar_wait(OD + 8 * (tl & 1), (uint32_t)((tl >> 1) & 1), abort_flag)))
+          if (!__all_sync(0xffffffffu, mbar_wait(OD + 8 * (tl % PB), (uint32_t)((tl / PB) & 1), abort_flag)))
             break;
           tc_fence_after();
 #pragma unroll
@@ -519,11 +543,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const size_t mrow = (size_t)xe.s * R + rloc;
       const int tl = tw - 1;
       const bool ok = __all_sync(
-          0xffffffffu, (j == x.nt) && mbar_wait(OD + 8 * (tl & 1), (uint32_t)((tl >> 1) & 1), abort_flag));
+          0xffffffffu, (j == x.nt) && mbar_wait(OD + 8 * (tl % PB), (uint32_t)((tl / PB) & 1), abort_flag));
       tc_fence_after();
       const float lt = l2.x + l2.y;
       const bool valid = ok && rloc >= 0 && rloc < R;
       const float inv = 1.f / lt;
+      // hd 64, one split: a warp whose 32 rows all lie in the sample stages them
+      // (bf16, 32-byte swizzle, 16 columns per 1 KB) in its quarter of a free P
+      // tile and writes them with TMA bulk stores; other rows are stored directly
+      const int q0 = x.q_begin + quarter * 32;
+      const bool tma_out = HD == 64 && g.nsplit == 1 && ok && q0 >= 0 && q0 + 31 < R;   // warp-uniform
+      const int sb = (tw + 1) % PB;                          // the P tile written last by the next item
+      uint8_t* stg = sP + sb * Cfg::P_BYTES + q * 4096;
+      if (tma_out && stg_buf >= 0) {
+        // at most one staging in flight: the previous item's stores have read theirs
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
+        stg_buf = -1;
+      }
       // 32 columns at a time; O is released after the last TMEM read
 #pragma unroll
       for (int h0 = 0; h0 < HD; h0 += 32) {
@@ -536,6 +573,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (h0 + 32 == HD) {
           tc_fence_before();
           mbar_arrive(OR);                           // O may be overwritten by the group's next item
+        }
+        if (tma_out) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 16) {
+            uint8_t* rp = stg + ((h0 + c) >> 4) * 1024 + lane * 32;
+            const int swz = (lane >> 2) & 1;
+            *reinterpret_cast<uint4*>(rp + (swz << 4)) =
+                make_uint4(pack_bf16(o[c] * inv, o[c + 1] * inv), pack_bf16(o[c + 2] * inv, o[c + 3] * inv),
+                           pack_bf16(o[c + 4] * inv, o[c + 5] * inv), pack_bf16(o[c + 6] * inv, o[c + 7] * inv));
+            *reinterpret_cast<uint4*>(rp + ((1 ^ swz) << 4)) =
+                make_uint4(pack_bf16(o[c + 8] * inv, o[c + 9] * inv), pack_bf16(o[c + 10] * inv, o[c + 11] * inv),
+                           pack_bf16(o[c + 12] * inv, o[c + 13] * inv), pack_bf16(o[c + 14] * inv, o[c + 15] * inv));
+          }
+          continue;
         }
         if (!valid) continue;
         if (g.nsplit == 1) {
@@ -551,6 +602,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int c = 0; c < 32; c += 4) dst[c >> 2] = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
         }
       }
+      if (tma_out) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+#pragma unroll
+          for (int ch = 0; ch < HD / 16; ++ch)
+            tma_store_2d(&tmO, smem_u32(stg + ch * 1024), xe.hh * HD + ch * 16, xe.s * R + q0);
+          bulk_commit();
+        }
+        stg_buf = sb;
+      }
       if (valid && g.nsplit > 1) {
         float* ml = g.mlpart + (((size_t)xe.split * g.m_max + mrow) * g.heads + xe.hh) * 2;
         ml[0] = m_use;
@@ -558,6 +620,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       alive = ok;
     }
+    if (lane == 0) bulk_wait_all();                           // the output stores are complete before exit
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -599,7 +663,8 @@ __global__ void __launch_bounds__(256) k_attn_combine(AttnArgs g) {
 }
 
 template <int HD>
-bool launch_hd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& g, int batch,
+bool launch_hd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+               const AttnArgs& g, int batch,
                int r_max, int* err, cudaStream_t st) {
   using Cfg = AttnCfg<HD>;
   static bool attr = false;
@@ -615,7 +680,7 @@ bool launch_hd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
   }
   const long long items = (long long)((r_max + BQ - 1) / BQ) * g.heads * batch * g.nsplit;
   const int grid = (int)(items < sms ? items : sms);
-  launch_k(k_attn_tc<HD>, dim3(grid), dim3(kAttnThreads), Cfg::SMEM, st, tq, tk, tv, g, err);
+  launch_k(k_attn_tc<HD>, dim3(grid), dim3(kAttnThreads), Cfg::SMEM, st, tq, tk, tv, to, g, err);
   if (g.nsplit > 1) {
     const long long warps = (long long)g.m_max * g.heads;
     launch_k(k_attn_combine<HD>, dim3((unsigned)((warps * 32 + 255) / 256)), dim3(256), 0, st, g);
@@ -641,9 +706,9 @@ bool launch_attn_tc2(const Ctl* ctl, const bf16* q, const bf16* kc, const bf16* 
                      cudaStream_t st) {
   const int hd = d / heads;
   const int bkv = hd == 64 ? AttnCfg<64>::BKV : AttnCfg<128>::BKV;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!make_tmap_bf16(&tq, q, m_max, d, 32) || !make_tmap_bf16(&tk, kc, batch * Lc, d, bkv) ||
-      !make_tmap_bf16(&tv, vc, batch * Lc, d, bkv))
+      !make_tmap_bf16(&tv, vc, batch * Lc, d, bkv) || !make_tmap_out(&to, o, false, m_max, d))
     return false;
   AttnArgs g;
   g.ctl = ctl;
@@ -658,8 +723,8 @@ bool launch_attn_tc2(const Ctl* ctl, const bf16* q, const bf16* kc, const bf16* 
   g.tiles_per_split = (key_tiles + nsplit - 1) / nsplit;
   g.m_max = m_max;
   g.batch = batch;
-  return hd == 64 ? launch_hd<64>(tq, tk, tv, g, batch, r_max, err, st)
-                  : launch_hd<128>(tq, tk, tv, g, batch, r_max, err, st);
+  return hd == 64 ? launch_hd<64>(tq, tk, tv, to, g, batch, r_max, err, st)
+                  : launch_hd<128>(tq, tk, tv, to, g, batch, r_max, err, st);
 }
 
 }  // namespace af
