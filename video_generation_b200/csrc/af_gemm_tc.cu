@@ -28,11 +28,11 @@ namespace af {
 namespace {
 
 constexpr int BM = 128, BK = 64;
-// Epilogue warps: 16 (4 per TMEM lane quarter) for the store-only epilogues,
-// 8 for those that also read a row of the residual stream or the positions
-// (more registers per thread).  Block = producer, MMA, 2 spare, epilogue.
+// Epilogue warps: 16 (4 per TMEM lane quarter), 8 for the position-add
+// epilogue, which also reads two rows of positions (more registers per
+// thread).  Block = producer, MMA, 2 spare, epilogue.
 template <int EPI> struct EpiShape {
-  static constexpr int WARPS = (EPI == EPI_RESID || EPI == EPI_INPROJ) ? 8 : 16;
+  static constexpr int WARPS = EPI == EPI_INPROJ ? 8 : 16;
   static constexpr int THREADS = (4 + WARPS) * 32;
   // residual add, GELU and QKV leave through TMA: each warp stages 32 rows x
   // 16 columns (two slots, alternating) in the output tensor map's swizzle and
@@ -446,6 +446,11 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
             ycache = s0 * e.Lc + p0 + (row0 - s0 * R);
           }
         }
+        // the bias of the first chunk is loaded before waiting for the accumulator,
+        // each later chunk's while the previous one is processed
+        float4 bnext[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) bnext[jj] = reinterpret_cast<const float4*>(e.bias + n0)[jj];
         // the wait's outcome is made warp-uniform before the .aligned TMEM loads
         if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * acc, use & 1u, abort_flag))) break;
         tc_fence_after();
@@ -453,6 +458,13 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
         tmem_ld16(taddr, vb[0]);
 #pragma unroll
         for (int k = 0; k < NCH; ++k) {
+          float4 b4[4];
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) b4[jj] = bnext[jj];
+          if (k + 1 < NCH) {
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) bnext[jj] = reinterpret_cast<const float4*>(e.bias + n0 + (k + 1) * 16)[jj];
+          }
           tmem_wait_ld();
           if (k + 1 < NCH) {
             tmem_ld16(taddr + (k + 1) * 16, vb[(k + 1) & 1]);
@@ -464,7 +476,6 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
           }
           const float* v = vb[k & 1];
           const int col = n0 + k * 16;
-          const float4* b4 = reinterpret_cast<const float4*>(e.bias + col);
           uint8_t* slot = stg0 + (cc & 1) * SLOT;
           if (lane == 0) bulk_wait_read1();             // the slot's previous tile has been read
           __syncwarp();
