@@ -7,18 +7,24 @@
 // block's causal Transformer: input projection, QKV, attention output
 // projection, the two MLP matrices and the (mu, log-sigma) head.
 //
-// Design (one persistent CTA per SM, 384 or 640 threads):
-//   warp 0      TMA producer: 128x64 A tile + BNx64 W tile per stage,
+// Design (persistent CTAs, one per SM, 384 or 640 threads):
+//   warp 0      TMA producer: 128x64 A tile + (BN/CG)x64 W tile per stage,
 //               128-byte swizzle, mbarrier transaction counts.
 //   warp 1      owns 512 TMEM columns; one thread issues tcgen05.mma
-//               (M=128, N=BN, K=16) into one of two accumulators and commits
-//               to the stage's "empty" barrier and the accumulator's "full".
+//               (M=128*CG, N=BN, K=16) into one of two accumulators and
+//               commits to the stage's "empty" barrier and the accumulator's
+//               "full".  CG = 2 pairs two SMs of a 2-CTA cluster on one
+//               256-row tile (cta_group::2): each CTA loads its own 128 rows
+//               of A and half of W, the leader issues the MMAs and its commits
+//               reach both CTAs.  No TMA load uses cluster multicast.
 //   warps 4..   epilogue, two or four warps per TMEM lane quarter (each takes
-//               a column group of the tile): tcgen05.ld 32 lanes x 16 columns,
-//               transpose through shared memory, apply the fused epilogue
-//               with row-coalesced stores, release the accumulator.
+//               a column group of the tile), tcgen05.ld 32 lanes x 16 columns
+//               at a time.  Residual add, GELU and QKV stage the result in
+//               the output tensor map's swizzle and leave by TMA (bulk
+//               reduce-add into h, bulk stores of u, q and the K / V cache);
+//               the position add transposes through shared memory for
+//               row-coalesced stores; the head works thread = row.
 // With two accumulators the epilogue of tile i overlaps the MMAs of tile i+1.
-// No cluster, no multicast: each CTA loads its own tiles.
 // Every wait is bounded (2 s); on expiry the CTA raises its abort flag, drains
 // its in-flight copies and MMAs, frees TMEM and reports ERR_GEMM_WAIT.
 #include <cudaTypedefs.h>
@@ -237,13 +243,6 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-__device__ __forceinline__ void st_bf16x4(bf16* dst, float a, float b, float c, float d) {
-  __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
-  uint2 u;
-  u.x = *reinterpret_cast<uint32_t*>(&lo);
-  u.y = *reinterpret_cast<uint32_t*>(&hi);
-  *reinterpret_cast<uint2*>(dst) = u;
-}
 
 template <int BN, int EPI, int CG>
 __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
@@ -402,13 +401,9 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
       }
     }
   } else if (warp >= 4) {
-      // ---------------------------------------------------------------- epilogue
+    // ---------------------------------------------------------------- epilogue
     // Warp 4+ew owns TMEM lane quarter q = ew % 4 (rows 32q..32q+31 of the
-    // tile) and column quarter ew / 4.  A 16-column chunk is read from TMEM
-    // (thread = row), transposed through a swizzled 32x16 staging tile, and
-    // applied with lane l on row 8*it + l/4, columns 4*(l%4)..+3: each store
-    // covers eight 64-byte row segments.  Row -> (sample, position) and the
-    // destination row pointers are computed once per tile.
+    // tile) and column group ew / 4, read 16 columns at a time.
     const int ew = warp - 4;
     const int q = ew & 3, hf = ew >> 2;                 // lane quarter, column group
     constexpr int HALF = BN / (Cfg::EPI_WARPS / 4);     // columns per warp
@@ -535,6 +530,13 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
       if (lane == 0) bulk_wait_all();                   // the bulk writes are complete before the CTA exits
       __syncwarp();
     } else {
+      // Position add (input projection) and the affine head.  For the position
+      // add a 16-column chunk read from TMEM (thread = row) is transposed
+      // through a swizzled 32 x 16 staging tile, so that lane l stores row
+      // 8 it + l / 4, columns 4 (l % 4) .. + 3: each store covers eight 64-byte
+      // row segments.  The head keeps thread = row.  Row -> (sample, position)
+      // and the row pointers are computed once per tile.
+      static_assert(EPI == EPI_INPROJ || EPI == EPI_HEAD, "epilogue without a TMA path");
       float* stg = sEpi + ew * 32 * 16;
       const int rl = lane >> 2, cq = lane & 3;
       const int sw_w = (lane >> 1) & 3;            // swizzle of the row this lane writes
@@ -549,31 +551,19 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
         const int row0 = mb * TM + (int)rank * BM + q * 32;
         const int n0 = nb * BN + hf * HALF;
         const uint32_t taddr = tmem + (uint32_t)(acc * BN + hf * HALF) + ((uint32_t)(q * 32) << 16);
-        // per-tile row info for the 4 rows this lane stores
-        char* rowp[4];
+        // position add: the 4 rows this lane stores and their position rows
+        float* rowp[4];
         const float* pos_s[4];
         const float* pos_t[4];
-        int colbase = 0;
-  #pragma unroll
-        for (int it = 0; it < 4; ++it) {
-          const int r = row0 + it * 8 + rl;
-          if (EPI == EPI_RESID) rowp[it] = reinterpret_cast<char*>(e.h + (size_t)r * e.d);
-          if (EPI == EPI_GELU) rowp[it] = reinterpret_cast<char*>(reinterpret_cast<bf16*>(e.out) + (size_t)r * e.ldo);
-          if (EPI == EPI_INPROJ || EPI == EPI_QKV) {
+        if (EPI == EPI_INPROJ) {
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            const int r = row0 + it * 8 + rl;
             const int sm = r / R;
             const int p = p0 + (r - sm * R);
-            if (EPI == EPI_INPROJ) {
-              rowp[it] = reinterpret_cast<char*>(e.h + (size_t)r * e.d);
-              pos_s[it] = e.pos_space + (size_t)(p % e.frame_len) * e.d;
-              pos_t[it] = e.pos_time + (size_t)(p / e.frame_len) * e.d;
-            } else {
-              const int which = (nb * BN) / e.d;            // the whole tile is q, k or v
-              if (which == 0) rowp[it] = reinterpret_cast<char*>(reinterpret_cast<bf16*>(e.out) + (size_t)r * e.d);
-              else
-                rowp[it] = reinterpret_cast<char*>(reinterpret_cast<bf16*>(which == 1 ? e.kc : e.vc) +
-                                                   ((size_t)sm * e.Lc + p) * e.d);
-              colbase = which * e.d;
-            }
+            rowp[it] = e.h + (size_t)r * e.d;
+            pos_s[it] = e.pos_space + (size_t)(p % e.frame_len) * e.d;
+            pos_t[it] = e.pos_time + (size_t)(p / e.frame_len) * e.d;
           }
         }
         // head: one row per thread, hoisted (sample, position, token) and row pointers
@@ -593,12 +583,12 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
           head_act = head_out && (e.head_mode == 0 || e.active[sm]);
         }
         // Loads that do not depend on the accumulator are issued before waiting
-        // for it (bias, and the first chunk's residual / position rows), and
-        // every chunk's TMEM load and global loads are in flight while the
-        // previous chunk is transposed and stored.
+        // for it (bias, and the first chunk's position / x rows), and every
+        // chunk's TMEM load and global loads are in flight while the previous
+        // chunk is processed.
         constexpr int NCH = HALF / 16;
         float4 bias4[NCH];
-  #pragma unroll
+#pragma unroll
         for (int k = 0; k < NCH; ++k) bias4[k] = *reinterpret_cast<const float4*>(e.bias + n0 + k * 16 + cq * 4);
         float4 pre[2][4], pre2[2][4];
         auto load_rows = [&](int k, float4* dst, float4* dst2) {
@@ -615,30 +605,27 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
             return;
           }
           const int col = n0 + k * 16 + cq * 4;
-  #pragma unroll
+#pragma unroll
           for (int it = 0; it < 4; ++it) {
             if (row0 + it * 8 + rl < M) {
-              if (EPI == EPI_RESID) dst[it] = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(rowp[it]) + col);
-              if (EPI == EPI_INPROJ) {
-                dst[it] = *reinterpret_cast<const float4*>(pos_s[it] + col);
-                dst2[it] = *reinterpret_cast<const float4*>(pos_t[it] + col);
-              }
+              dst[it] = *reinterpret_cast<const float4*>(pos_s[it] + col);
+              dst2[it] = *reinterpret_cast<const float4*>(pos_t[it] + col);
             }
           }
         };
-        if (EPI == EPI_RESID || EPI == EPI_INPROJ || EPI == EPI_HEAD) load_rows(0, pre[0], pre2[0]);
+        load_rows(0, pre[0], pre2[0]);
         // the wait's outcome is made warp-uniform before the .aligned TMEM loads
         if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * acc, use & 1u, abort_flag))) break;
         tc_fence_after();
         float vb[2][16];
         tmem_ld16(taddr, vb[0]);
-  #pragma unroll
+#pragma unroll
         for (int k = 0; k < NCH; ++k) {
           const int c = k * 16;
           tmem_wait_ld();
           if (k + 1 < NCH) {
             tmem_ld16(taddr + c + 16, vb[(k + 1) & 1]);
-            if (EPI == EPI_RESID || EPI == EPI_INPROJ || EPI == EPI_HEAD) load_rows(k + 1, pre[(k + 1) & 1], pre2[(k + 1) & 1]);
+            load_rows(k + 1, pre[(k + 1) & 1], pre2[(k + 1) & 1]);
           }
           const float* v = vb[k & 1];
           if (EPI == EPI_HEAD) {
@@ -650,7 +637,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
             const float* xi = reinterpret_cast<const float*>(pre[k & 1]);
             float r8[8];
             float a0 = 0.f, a1 = 0.f;
-  #pragma unroll
+#pragma unroll
             for (int jj = 0; jj < 8; ++jj) {
               const float mu = v[2 * jj] + e.bias[col0 + 2 * jj];
               const float sl = v[2 * jj + 1] + e.bias[col0 + 2 * jj + 1];
@@ -671,50 +658,23 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
             continue;
           }
           float4* srow = reinterpret_cast<float4*>(stg + lane * 16);
-  #pragma unroll
+#pragma unroll
           for (int j = 0; j < 4; ++j) srow[j ^ sw_w] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
           __syncwarp();
           float4 a[4];
-  #pragma unroll
+#pragma unroll
           for (int it = 0; it < 4; ++it) a[it] = reinterpret_cast<const float4*>(stg + (it * 8 + rl) * 16)[cq ^ sw_r];
           __syncwarp();
           const int col = n0 + c + cq * 4;
           const float4 bb = bias4[k];
-          if (EPI == EPI_RESID) {
-  #pragma unroll
-            for (int it = 0; it < 4; ++it) {
-              if (row0 + it * 8 + rl < M) {
-                float4 hv = pre[k & 1][it];
-                hv.x += a[it].x + bb.x; hv.y += a[it].y + bb.y;
-                hv.z += a[it].z + bb.z; hv.w += a[it].w + bb.w;
-                *reinterpret_cast<float4*>(reinterpret_cast<float*>(rowp[it]) + col) = hv;
-              }
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            if (row0 + it * 8 + rl < M) {
+              const float4 ps = pre[k & 1][it], pt = pre2[k & 1][it];
+              *reinterpret_cast<float4*>(rowp[it] + col) =
+                  make_float4(a[it].x + bb.x + ps.x + pt.x, a[it].y + bb.y + ps.y + pt.y,
+                              a[it].z + bb.z + ps.z + pt.z, a[it].w + bb.w + ps.w + pt.w);
             }
-          } else if (EPI == EPI_INPROJ) {
-  #pragma unroll
-            for (int it = 0; it < 4; ++it) {
-              if (row0 + it * 8 + rl < M) {
-                const float4 ps = pre[k & 1][it], pt = pre2[k & 1][it];
-                *reinterpret_cast<float4*>(reinterpret_cast<float*>(rowp[it]) + col) =
-                    make_float4(a[it].x + bb.x + ps.x + pt.x, a[it].y + bb.y + ps.y + pt.y,
-                                a[it].z + bb.z + ps.z + pt.z, a[it].w + bb.w + ps.w + pt.w);
-              }
-            }
-          } else if (EPI == EPI_GELU) {
-  #pragma unroll
-            for (int it = 0; it < 4; ++it) {
-              if (row0 + it * 8 + rl < M) {
-                const float2 g0 = gelu2_as7126(fadd2(make_float2(a[it].x, a[it].y), make_float2(bb.x, bb.y)));
-                const float2 g1 = gelu2_as7126(fadd2(make_float2(a[it].z, a[it].w), make_float2(bb.z, bb.w)));
-                st_bf16x4(reinterpret_cast<bf16*>(rowp[it]) + col, g0.x, g0.y, g1.x, g1.y);
-              }
-            }
-          } else if (EPI == EPI_QKV) {
-  #pragma unroll
-            for (int it = 0; it < 4; ++it)
-              if (row0 + it * 8 + rl < M)
-                st_bf16x4(reinterpret_cast<bf16*>(rowp[it]) + (col - colbase), a[it].x + bb.x, a[it].y + bb.y,
-                          a[it].z + bb.z, a[it].w + bb.w);
           }
         }
         tc_fence_before();
