@@ -1,0 +1,28 @@
+"""The reference arm of bench.py: the CPU float64 oracle timed on the host cores
+(one frame of the 21-frame f_S stack per step), printed as one JSON line with
+the keys and meanings the throughput line uses.  Runs without a GPU."""
+import json
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_reference_arm_prints_one_contract_line():
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1", "--warmup", "3",
+           "--ref-frames", "1"]
+    out = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["metric"] == "jacobi_inverse_latent_tokens_per_s" and line["unit"] == "tokens/s"
+    assert line["higher_is_better"] is True and line["value"] > 0
+    assert line["n_gpus"] == 1 and line["steps"] == 1 and line["warmup"] == 3
+    assert line["dtype"] == "f64" and line["data"] == "synthetic"
+    assert line["config"]["workload"] == "fs_stack_T3_4L_d768_21frames_bf16"
+    # the oracle runs on the host: no transfers, and the baseline is the line itself
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1 and cb["sample"]
