@@ -60,7 +60,9 @@ typedef enum { AF_L2R = 0, AF_R2L = 1 } af_dir;
 typedef enum { AF_FP32 = 0, AF_BF16 = 1 } af_dtype;
 
 /* Shape of one AF block.  max_len = frame_len * max_frames bounds L.
- * AF_BF16 requires C % 64 == 0, d % 64 == 0 and d / heads in {64, 128};
+ * Every config needs positive sizes, d % heads == 0, C % 8 == 0, d % 4 == 0.
+ * AF_BF16 also requires C % 64 == 0, d % 128 == 0, (mlp_ratio * d) % 128 == 0
+ * and d / heads in {64, 128} (the tensor-core tile shapes);
  * AF_FP32 requires d / heads in {16, 32, 64, 128}. */
 typedef struct {
   int C, d, heads, layers, mlp_ratio;
