@@ -279,6 +279,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // ------------------------------------------------------------------ TMA producer of the group
       int iw = 0, kst = 0, vst = 0;
       uint32_t kph = 0, vph = 0;
+      long long nq = 0, nk = 0, nv = 0;                       // loads issued per ring
       bool ok = true;
       for (int k = grp; ok; k += 2) {
         const int it = global_item(k);
@@ -298,6 +299,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int qq = 0; qq < 4; ++qq)
             tma_load_2d(smem_u32(sQ + qb * Cfg::Q_BYTES + kc * Cfg::QBOX + (grp ? 3 - qq : qq) * 4096), &tmQ,
                         QF + 8 * qb, x.hh * HD + kc * 64, x.s * R + x.q_begin + 32 * qq);
+        ++nq;
         for (int j = 0; j < x.nt; ++j) {
           const int krow = x.s * g.Lc + (x.t0 + j) * BKV;
           if (!mbar_wait(KE + 8 * kst, kph ^ 1u, abort_flag)) { ok = false; break; }
@@ -306,6 +308,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int kc = 0; kc < Cfg::KCH; ++kc)
             tma_load_2d(smem_u32(sK + kst * Cfg::KV_BYTES + kc * Cfg::KVBOX), &tmK, KF + 8 * kst, x.hh * HD + kc * 64,
                         krow);
+          ++nk;
           if (++kst == SK) { kst = 0; kph ^= 1u; }
           if (!mbar_wait(VE + 8 * vst, vph ^ 1u, abort_flag)) { ok = false; break; }
           mbar_expect_tx(VF + 8 * vst, Cfg::KV_BYTES);
@@ -313,9 +316,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int kc = 0; kc < Cfg::KCH; ++kc)
             tma_load_2d(smem_u32(sV + vst * Cfg::KV_BYTES + kc * Cfg::KVBOX), &tmV, VF + 8 * vst, x.hh * HD + kc * 64,
                         krow);
+          ++nv;
           if (++vst == SV) { vst = 0; vph ^= 1u; }
         }
         ++iw;
+      }
+      if (*abort_flag) {
+        // After an abort nothing consumes the loads still in flight: the latest
+        // load of every stage of each ring lands before the CTA frees its
+        // shared memory (one 2 s limit for the whole drain).
+        const uint64_t t0 = globaltimer_ns();
+        auto drain_ring = [&](uint32_t full0, int stages, long long issued) {
+          const long long n = issued < stages ? issued : stages;
+          for (long long jj = 1; jj <= n; ++jj) {
+            const long long idx = issued - jj;
+            const uint32_t bar = full0 + 8u * (uint32_t)(idx % stages);
+            const uint32_t ph = (uint32_t)((idx / stages) & 1);
+            while (!mbar_try(bar, ph)) {
+              if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+            }
+          }
+        };
+        drain_ring(QF, QB, nq);
+        drain_ring(KF, SK, nk);
+        drain_ring(VF, SV, nv);
       }
     }
   } else if (warp < 4) {
