@@ -204,6 +204,30 @@ def af_forward(blk: Block, x: np.ndarray, direction: int):
     return np.stack([o[0] for o in out]), np.array([o[1] for o in out])
 
 
+def af_forward_chunked_one(blk: Block, x: np.ndarray, direction: int, B: int, keep_from: int = 0):
+    """The forward pass of one sample computed B positions at a time through the
+    KV cache ([N] key design 3: finished blocks feed a KV cache), so that no
+    score matrix is larger than B x L -- the same z as ``af_forward_one`` (it
+    is the same causal computation), usable at lengths where an L x L score
+    matrix does not fit in memory.  Returns (z rows of working-order positions
+    >= keep_from, in working order, and the logdet of the whole sequence)."""
+    xw = _f(_work(x, direction))
+    L = xw.shape[0]
+    cache = None
+    zs, logdet = [], 0.0
+    for P in range(0, L, B):
+        Q = min(P + B, L)
+        mu, s, kv = transformer_rows(blk, masked_inputs(xw, P, Q), P, cache)
+        if Q > keep_from:
+            lo = max(P, keep_from) - P
+            zs.append(((xw[P:Q] - mu) * np.exp(-s))[lo:])
+        logdet -= s.sum()
+        cache = kv if cache is None else [(np.concatenate([cache[l][0], kv[l][0]]),
+                                           np.concatenate([cache[l][1], kv[l][1]]))
+                                          for l in range(blk.layers)]
+    return np.concatenate(zs), float(logdet)
+
+
 # ----------------------------------------------------------------------------
 # sequential inverse (textbook autoregressive inverse, token by token)
 
@@ -242,31 +266,43 @@ def converged(num, den, tau):
 
 
 def af_inverse_jacobi_one(blk: Block, z: np.ndarray, direction: int, B: int, tau: float,
-                          max_iter: int, warm_start: bool, x0=None, trace=None):
+                          max_iter: int, warm_start: bool, x0=None, trace=None,
+                          x_known=None, n_known: int = 0):
     """One sample.  Returns (x, iters [L/B], converged [L/B]).
 
     ``x0`` optionally overrides the first block's starting guess (used by the
     any-start prefix-exactness pin); ``trace`` collects every iterate of every
     block when given a list.
+
+    ``x_known`` [L, C] (original token order) with ``n_known`` > 0: the first
+    ``n_known`` blocks are observed, not sampled -- their x is taken as given
+    and only their K/V enter the cache ([N] "A complete example": I2V / V2V
+    encode the observed frames with the flow's forward pass into the KV cache,
+    then the following frames are generated autoregressively).  Those blocks
+    report 0 iterations and count as converged.
     """
     zw = _f(_work(z, direction))
     L, C = zw.shape
     assert L % B == 0
     nb = L // B
     xw = np.zeros_like(zw)
+    xk_w = _f(_work(x_known, direction)) if n_known else None
     cache = None
     iters = np.zeros(nb, np.int64)
     conv = np.zeros(nb, bool)
     for b in range(nb):
         P = b * B
         zb = zw[P:P + B]
-        if b == 0 and x0 is not None:
+        if b < n_known:                                   # observed block: x given
+            xk = xk_w[P:P + B].copy()
+            conv[b] = True
+        elif b == 0 and x0 is not None:
             xk = _f(_work(x0, direction))[P:P + B].copy()
         elif warm_start and b > 0:
             xk = xw[P - B:P].copy()                       # warm start from block b-1
         else:
             xk = zb.copy()                                # R5
-        for k in range(max_iter):
+        for k in range(0 if b < n_known else max_iter):
             xw[P:P + B] = xk
             mu, s, _ = transformer_rows(blk, masked_inputs(xw, P, P + B), P, cache)
             x_new = mu + np.exp(s) * zb
@@ -290,9 +326,14 @@ def af_inverse_jacobi_one(blk: Block, z: np.ndarray, direction: int, B: int, tau
 
 
 def af_inverse_jacobi(blk: Block, z: np.ndarray, direction: int, B: int, tau: float,
-                      max_iter: int, warm_start: bool):
-    """z [batch, L, C] -> x [batch, L, C], iters [batch, L/B], converged [batch, L/B]."""
-    out = [af_inverse_jacobi_one(blk, zb, direction, B, tau, max_iter, warm_start) for zb in z]
+                      max_iter: int, warm_start: bool, x_known=None, n_known: int = 0):
+    """z [batch, L, C] -> x [batch, L, C], iters [batch, L/B], converged [batch, L/B].
+
+    ``x_known`` [batch, L, C] with ``n_known`` observed leading blocks: see
+    ``af_inverse_jacobi_one``."""
+    out = [af_inverse_jacobi_one(blk, zb, direction, B, tau, max_iter, warm_start,
+                                 x_known=None if x_known is None else x_known[i], n_known=n_known)
+           for i, zb in enumerate(z)]
     return (np.stack([o[0] for o in out]), np.stack([o[1] for o in out]),
             np.stack([o[2] for o in out]))
 

@@ -78,6 +78,17 @@ def _residual_old_den(x_new, x_old):
     return float(((x_new - x_old) ** 2).sum()), float((x_old ** 2).sum())
 
 
+def _positions_no_time(blk, p):
+    return np.asarray(blk.pos_space, np.float64)[p % blk.frame_len]
+
+
+def _positions_time_by_length(blk, p):
+    # temporal row from the position divided by the sequence's whole length
+    n = blk.frame_len * blk.max_frames
+    return (np.asarray(blk.pos_space, np.float64)[p % blk.frame_len]
+            + np.asarray(blk.pos_time, np.float64)[p // n])
+
+
 MUTATIONS = {
     "gelu_tanh_approx": ("gelu", _gelu_tanh),
     "attention_scale": ("causal_attention", _attn_bad_scale),
@@ -85,6 +96,8 @@ MUTATIONS = {
     "logdet_sign": ("af_forward_one", _fwd_bad_sign),
     "mask_not_self_exclusive": ("masked_inputs", _masked_no_shift),
     "residual_denominator_old_iterate": ("jacobi_residual", _residual_old_den),
+    "positions_without_time_rows": ("positions", _positions_no_time),
+    "positions_time_index_by_length": ("positions", _positions_time_by_length),
 }
 
 
@@ -97,6 +110,7 @@ def _any_pin_fails():
     err, sign, upper, diag = P.pin_logdet_bruteforce(O.L2R)
     checks.append(err > 1e-7 or upper > 1e-9 or diag > 1e-7)
     checks.append(P.pin_roundtrip_seq(O.R2L) > 1e-12)
+    checks.append(P.pin_positions_hand_written() != 0.0)
     try:
         test_jacobi_iteration_count_closed_form(True)
         checks.append(False)

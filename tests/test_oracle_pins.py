@@ -271,3 +271,89 @@ def test_residual_edge_cases():
     assert not O.converged(1.0, 0.0, 1e-3)
     assert not O.converged(1e-3, 1.0, 1e-3)          # strict <
     assert O.converged(0.99e-3, 1.0, 1e-3)
+
+
+# ---------------------------------------------------------------------------- positions, chunked forward, known prefix
+
+POS_SHAPE = syn.ModelShape(C=4, d=4, heads=1, layers=1, mlp_ratio=1, frame_len=2, max_frames=3, dtype="fp32")
+
+
+def pin_positions_hand_written():
+    """pos[p] for 3 frames of 2 tokens, written out by hand (R10: the spatial
+    row is p mod frame_len, the temporal row p div frame_len).
+
+    P_space rows are 1 and 2 in column 0; P_time rows are 10, 20, 30 in column
+    1 and 100, 200, 300 in column 2; column 3 stays 0.  Returns the max abs
+    error over positions 0..5."""
+    w = syn.make_weights(POS_SHAPE, zero=("w", "pos", "head", "bias", "shift", "headbias"))
+    w[2] = np.array([[1, 0, 0, 0], [2, 0, 0, 0]], np.float32)                            # P_space
+    w[3] = np.array([[0, 10, 100, 0], [0, 20, 200, 0], [0, 30, 300, 0]], np.float32)    # P_time
+    blk = O.Block(POS_SHAPE, w)
+    expect = np.array([[1, 10, 100, 0],      # p = 0: frame 0, token 0
+                       [2, 10, 100, 0],      # p = 1: frame 0, token 1
+                       [1, 20, 200, 0],      # p = 2: frame 1, token 0
+                       [2, 20, 200, 0],      # p = 3: frame 1, token 1
+                       [1, 30, 300, 0],      # p = 4: frame 2, token 0
+                       [2, 30, 300, 0]],     # p = 5: frame 2, token 1
+                      np.float64)
+    return float(np.abs(O.positions(blk, np.arange(6)) - expect).max())
+
+
+def test_positions_match_hand_written_table():
+    assert pin_positions_hand_written() == 0.0
+
+
+def test_positions_reach_the_transformer_per_frame():
+    """Two tokens with the same input but in different frames get different
+    (mu, s) exactly when their temporal rows differ (and equal ones when only
+    the frame's content, not its position, is shared)."""
+    shape = syn.ModelShape(C=4, d=16, heads=2, layers=1, mlp_ratio=2, frame_len=2, max_frames=3, dtype="fp32")
+    w = syn.make_weights(shape, perturb=True, head_std=0.3)
+    blk = O.Block(shape, w)
+    x_in = np.ones((6, 4))
+    mu, s, _ = O.transformer_rows(blk, x_in, 0)
+    w2 = [a.copy() for a in w]
+    w2[3][:] = w2[3][0]                       # all temporal rows equal
+    mu2, _, _ = O.transformer_rows(O.Block(shape, w2), x_in, 0)
+    w3 = [a.copy() for a in w]
+    w3[3][1:] += np.linspace(-1.0, 1.0, shape.d, dtype=np.float32)   # frames 1 and 2 only (not a
+    #                                           constant shift, which LayerNorm would remove)
+    mu3, _, _ = O.transformer_rows(O.Block(shape, w3), x_in, 0)
+    np.testing.assert_array_equal(mu3[:2], mu[:2])     # frame 0 untouched (causal, row 0 of P_time)
+    assert np.abs(mu3[2:] - mu[2:]).max() > 1e-3
+    assert np.abs(mu2 - mu).max() > 1e-3
+
+
+def test_chunked_forward_equals_plain_forward():
+    blk = tiny_block()
+    x = np.random.default_rng(13).standard_normal((2, 22, TINY.C))
+    for direction in (O.L2R, O.R2L):
+        z, ld = O.af_forward(blk, x, direction)
+        for B in (5, 8, 22):
+            for i in range(2):
+                zc, ldc = O.af_forward_chunked_one(blk, x[i], direction, B)
+                zc = zc[::-1] if direction == O.R2L else zc
+                assert rel(zc, z[i]) < 1e-12 and abs(ldc - ld[i]) < 1e-12 * max(1.0, abs(ld[i]))
+                tail, _ = O.af_forward_chunked_one(blk, x[i], direction, B, keep_from=13)
+                zw = z[i][::-1] if direction == O.R2L else z[i]
+                assert rel(tail, zw[13:]) < 1e-12
+
+
+def test_known_prefix_continues_the_same_inverse():
+    """Observed leading blocks (x given) followed by Jacobi blocks: with the
+    oracle's own first blocks as the observation the result is bitwise the
+    full Jacobi run; with tau = 0 and B sweeps it reaches the exact inverse of
+    the forward pass whatever prefix is observed."""
+    blk = tiny_block(head_std=0.2)
+    rng = np.random.default_rng(14)
+    z = rng.standard_normal((2, 24, TINY.C))
+    for warm in (False, True):
+        x_full, it_full, _ = O.af_inverse_jacobi(blk, z, O.R2L, 8, 1e-6, 8, warm)
+        x_tf, it_tf, conv_tf = O.af_inverse_jacobi(blk, z, O.R2L, 8, 1e-6, 8, warm, x_known=x_full, n_known=2)
+        np.testing.assert_array_equal(x_tf, x_full)
+        assert (it_tf[:, :2] == 0).all() and conv_tf[:, :2].all()
+        np.testing.assert_array_equal(it_tf[:, 2:], it_full[:, 2:])
+    x_true = rng.standard_normal((2, 24, TINY.C))
+    zt, _ = O.af_forward(blk, x_true, O.L2R)
+    x_tf, _, _ = O.af_inverse_jacobi(blk, zt, O.L2R, 8, 0.0, 8, True, x_known=x_true, n_known=1)
+    assert rel(x_tf, x_true) < 1e-12
