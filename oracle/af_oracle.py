@@ -48,6 +48,11 @@ section:
        before the block and restores it after.
     R12 bf16 models: the weights are rounded to bf16 (round to nearest even)
        once; the oracle then computes in float64 with those values.
+    R13 warm start per token: position p of a new block starts from the
+       converged x at p - k*frame_len, the same spatial position in the most
+       recent finished frame (smallest k >= 1 reaching before the block), or
+       from z where no frame before it has finished.  With one-frame blocks
+       this is the previous block's converged x at the same offsets.
 """
 from __future__ import annotations
 
@@ -189,12 +194,16 @@ def _work(a, direction):            # R11
 # ----------------------------------------------------------------------------
 # forward: z and logdet ([N] key design 1, affine AF equation; loss section)
 
-def af_forward_one(blk: Block, x: np.ndarray, direction: int):
+def af_forward_one(blk: Block, x: np.ndarray, direction: int, with_abs: bool = False):
+    """z and logdet of one sample; with ``with_abs`` also sum |s| (the scale
+    against which tests judge a logdet that is a sum of many cancelling s)."""
     xw = _f(_work(x, direction))
     L = xw.shape[0]
     mu, s, _ = transformer_rows(blk, masked_inputs(xw, 0, L), 0)
     zw = (xw - mu) * np.exp(-s)               # sigma = exp(s)   (R2)
     logdet = -s.sum()                         # log|det dz/dx| = -sum log sigma (R3)
+    if with_abs:
+        return _work(zw, direction).copy(), float(logdet), float(np.abs(s).sum())
     return _work(zw, direction).copy(), float(logdet)
 
 
@@ -210,11 +219,12 @@ def af_forward_chunked_one(blk: Block, x: np.ndarray, direction: int, B: int, ke
     score matrix is larger than B x L -- the same z as ``af_forward_one`` (it
     is the same causal computation), usable at lengths where an L x L score
     matrix does not fit in memory.  Returns (z rows of working-order positions
-    >= keep_from, in working order, and the logdet of the whole sequence)."""
+    >= keep_from, in working order; the logdet of the whole sequence; and its
+    sum of |s|)."""
     xw = _f(_work(x, direction))
     L = xw.shape[0]
     cache = None
-    zs, logdet = [], 0.0
+    zs, logdet, sabs = [], 0.0, 0.0
     for P in range(0, L, B):
         Q = min(P + B, L)
         mu, s, kv = transformer_rows(blk, masked_inputs(xw, P, Q), P, cache)
@@ -222,10 +232,11 @@ def af_forward_chunked_one(blk: Block, x: np.ndarray, direction: int, B: int, ke
             lo = max(P, keep_from) - P
             zs.append(((xw[P:Q] - mu) * np.exp(-s))[lo:])
         logdet -= s.sum()
+        sabs += np.abs(s).sum()
         cache = kv if cache is None else [(np.concatenate([cache[l][0], kv[l][0]]),
                                            np.concatenate([cache[l][1], kv[l][1]]))
                                           for l in range(blk.layers)]
-    return np.concatenate(zs), float(logdet)
+    return np.concatenate(zs), float(logdet), float(sabs)
 
 
 # ----------------------------------------------------------------------------
@@ -265,11 +276,44 @@ def converged(num, den, tau):
     return num / den < tau
 
 
-def af_inverse_jacobi_one(blk: Block, z: np.ndarray, direction: int, B: int, tau: float,
+def block_starts(L: int, B) -> List[int]:
+    """Start positions of the blocks of a sequence of L tokens, and L last.
+
+    ``B`` is one block size (every block B tokens; L % B == 0), or a list of
+    block sizes in sequence order summing to L ([N] "Key findings": the block
+    size can change along the video, e.g. 64 for the first frame and 512
+    later)."""
+    sizes = [B] * (L // B) if isinstance(B, (int, np.integer)) else [int(b) for b in B]
+    if isinstance(B, (int, np.integer)):
+        assert L % B == 0
+    assert sum(sizes) == L and all(b > 0 for b in sizes)
+    return [0] + list(np.cumsum(sizes))
+
+
+def warm_start_guess(xw: np.ndarray, zw: np.ndarray, P: int, Q: int, frame_len: int) -> np.ndarray:
+    """x^(0) of the block of positions P..Q-1 under the video-aware warm start.
+
+    [N] key design 3: a new frame starts from the previous frame's converged
+    state.  Per token (R13): the token at position p starts from the
+    converged x of the same spatial position in the most recent finished
+    frame, p - k*frame_len with the smallest k >= 1 that lands before the
+    block (p - k*frame_len < P); a token with no such finished position (the
+    first frame) starts from z (R5).  With blocks of exactly one frame this is
+    "block b starts from block b-1's x"."""
+    out = np.empty((Q - P, zw.shape[1]))
+    for p in range(P, Q):
+        k = (p - P) // frame_len + 1
+        src = p - k * frame_len
+        out[p - P] = xw[src] if src >= 0 else zw[p]
+    return out
+
+
+def af_inverse_jacobi_one(blk: Block, z: np.ndarray, direction: int, B, tau: float,
                           max_iter: int, warm_start: bool, x0=None, trace=None,
                           x_known=None, n_known: int = 0):
-    """One sample.  Returns (x, iters [L/B], converged [L/B]).
+    """One sample.  Returns (x, iters [n_blocks], converged [n_blocks]).
 
+    ``B`` is the block size, or the list of block sizes (see ``block_starts``).
     ``x0`` optionally overrides the first block's starting guess (used by the
     any-start prefix-exactness pin); ``trace`` collects every iterate of every
     block when given a list.
@@ -283,28 +327,28 @@ def af_inverse_jacobi_one(blk: Block, z: np.ndarray, direction: int, B: int, tau
     """
     zw = _f(_work(z, direction))
     L, C = zw.shape
-    assert L % B == 0
-    nb = L // B
+    starts = block_starts(L, B)
+    nb = len(starts) - 1
     xw = np.zeros_like(zw)
     xk_w = _f(_work(x_known, direction)) if n_known else None
     cache = None
     iters = np.zeros(nb, np.int64)
     conv = np.zeros(nb, bool)
     for b in range(nb):
-        P = b * B
-        zb = zw[P:P + B]
+        P, Q = starts[b], starts[b + 1]
+        zb = zw[P:Q]
         if b < n_known:                                   # observed block: x given
-            xk = xk_w[P:P + B].copy()
+            xk = xk_w[P:Q].copy()
             conv[b] = True
         elif b == 0 and x0 is not None:
-            xk = _f(_work(x0, direction))[P:P + B].copy()
-        elif warm_start and b > 0:
-            xk = xw[P - B:P].copy()                       # warm start from block b-1
+            xk = _f(_work(x0, direction))[P:Q].copy()
+        elif warm_start:
+            xk = warm_start_guess(xw, zw, P, Q, blk.frame_len)   # previous frame's state (R13)
         else:
             xk = zb.copy()                                # R5
         for k in range(0 if b < n_known else max_iter):
-            xw[P:P + B] = xk
-            mu, s, _ = transformer_rows(blk, masked_inputs(xw, P, P + B), P, cache)
+            xw[P:Q] = xk
+            mu, s, _ = transformer_rows(blk, masked_inputs(xw, P, Q), P, cache)
             x_new = mu + np.exp(s) * zb
             num, den = jacobi_residual(x_new, xk)
             xk = x_new
@@ -314,9 +358,9 @@ def af_inverse_jacobi_one(blk: Block, z: np.ndarray, direction: int, B: int, tau
             if converged(num, den, tau):
                 conv[b] = True
                 break
-        xw[P:P + B] = xk                                  # R6
+        xw[P:Q] = xk                                      # R6
         if b + 1 < nb:                                    # commit K/V of the final x (R7)
-            _, _, kv = transformer_rows(blk, masked_inputs(xw, P, P + B), P, cache)
+            _, _, kv = transformer_rows(blk, masked_inputs(xw, P, Q), P, cache)
             if cache is None:
                 cache = [(k_, v_) for (k_, v_) in kv]
             else:
@@ -325,12 +369,12 @@ def af_inverse_jacobi_one(blk: Block, z: np.ndarray, direction: int, B: int, tau
     return _work(xw, direction).copy(), iters, conv
 
 
-def af_inverse_jacobi(blk: Block, z: np.ndarray, direction: int, B: int, tau: float,
+def af_inverse_jacobi(blk: Block, z: np.ndarray, direction: int, B, tau: float,
                       max_iter: int, warm_start: bool, x_known=None, n_known: int = 0):
-    """z [batch, L, C] -> x [batch, L, C], iters [batch, L/B], converged [batch, L/B].
+    """z [batch, L, C] -> x [batch, L, C], iters [batch, n_blocks], converged [batch, n_blocks].
 
-    ``x_known`` [batch, L, C] with ``n_known`` observed leading blocks: see
-    ``af_inverse_jacobi_one``."""
+    ``B``: one block size or the list of block sizes.  ``x_known`` [batch, L,
+    C] with ``n_known`` observed leading blocks: see ``af_inverse_jacobi_one``."""
     out = [af_inverse_jacobi_one(blk, zb, direction, B, tau, max_iter, warm_start,
                                  x_known=None if x_known is None else x_known[i], n_known=n_known)
            for i, zb in enumerate(z)]

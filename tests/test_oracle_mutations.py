@@ -1,11 +1,13 @@
 """Plant plausible mistakes in the CPU oracle and check that a pin catches each.
 
-Also pins the Jacobi stopping rule and iteration count with a closed form: for
-a head-only model (every weight 0 except b_head) mu and s are constants, so
-x^(1) = mu + exp(s) z exactly and x^(2) = x^(1); the residual of the first
-update, ||x^(1) - x^(0)||^2 / ||x^(1)||^2, is then known in closed form and
-decides whether a block stops after 1 or 2 updates ("STARFlow-V ... paper
-notes", key design 3: the scale-normalised residual and tau).
+Also pins the Jacobi stopping rule, the warm start and the iteration count
+with a closed form: for a head-only model (every weight 0 except b_head) mu
+and s are constants, so x^(1) = mu + exp(s) z exactly and x^(2) = x^(1); the
+residual of the first update, ||x^(1) - x^(0)||^2 / ||x^(1)||^2, is then known
+in closed form from x^(0) -- z, or with warm start the previous frame's
+converged tokens -- and decides whether a block stops after 1 or 2 updates
+("STARFlow-V ... paper notes", key design 3: the scale-normalised residual and
+tau; a new frame starts from the previous frame's converged state).
 """
 import math
 
@@ -30,9 +32,12 @@ def test_jacobi_iteration_count_closed_form(warm):
     B, nb = 4, 3
     z = np.random.default_rng(12).standard_normal((1, B * nb, C))
     x_exact = mu + sg * z[0]
+    F = P.TINY.frame_len                 # 8: two blocks of 4 per frame
     r1 = []
     for b in range(nb):
-        x0 = x_exact[(b - 1) * B:b * B] if (warm and b > 0) else z[0, b * B:(b + 1) * B]
+        # warm start: each token starts from the same spatial token of the previous
+        # frame once that frame is finished (block 2 from block 0), else from z
+        x0 = np.array([x_exact[p - F] if (warm and p - F >= 0) else z[0, p] for p in range(b * B, (b + 1) * B)])
         x1 = x_exact[b * B:(b + 1) * B]
         r1.append(((x1 - x0) ** 2).sum() / (x1 ** 2).sum())
     r1 = np.array(r1)
@@ -78,6 +83,12 @@ def _residual_old_den(x_new, x_old):
     return float(((x_new - x_old) ** 2).sum()), float((x_old ** 2).sum())
 
 
+def _warm_from_previous_block(xw, zw, P, Q, frame_len):
+    # the previous block's converged x at the same offsets, whatever the frame
+    B = Q - P
+    return np.array([xw[p - B] if p - B >= 0 else zw[p] for p in range(P, Q)])
+
+
 def _positions_no_time(blk, p):
     return np.asarray(blk.pos_space, np.float64)[p % blk.frame_len]
 
@@ -97,6 +108,7 @@ MUTATIONS = {
     "mask_not_self_exclusive": ("masked_inputs", _masked_no_shift),
     "residual_denominator_old_iterate": ("jacobi_residual", _residual_old_den),
     "positions_without_time_rows": ("positions", _positions_no_time),
+    "warm_start_from_previous_block": ("warm_start_guess", _warm_from_previous_block),
     "positions_time_index_by_length": ("positions", _positions_time_by_length),
 }
 
@@ -111,6 +123,7 @@ def _any_pin_fails():
     checks.append(err > 1e-7 or upper > 1e-9 or diag > 1e-7)
     checks.append(P.pin_roundtrip_seq(O.R2L) > 1e-12)
     checks.append(P.pin_positions_hand_written() != 0.0)
+    checks.append(P.pin_warm_start_guess() != 0.0)
     try:
         test_jacobi_iteration_count_closed_form(True)
         checks.append(False)

@@ -331,10 +331,10 @@ def test_chunked_forward_equals_plain_forward():
         z, ld = O.af_forward(blk, x, direction)
         for B in (5, 8, 22):
             for i in range(2):
-                zc, ldc = O.af_forward_chunked_one(blk, x[i], direction, B)
+                zc, ldc, _ = O.af_forward_chunked_one(blk, x[i], direction, B)
                 zc = zc[::-1] if direction == O.R2L else zc
                 assert rel(zc, z[i]) < 1e-12 and abs(ldc - ld[i]) < 1e-12 * max(1.0, abs(ld[i]))
-                tail, _ = O.af_forward_chunked_one(blk, x[i], direction, B, keep_from=13)
+                tail, _, _ = O.af_forward_chunked_one(blk, x[i], direction, B, keep_from=13)
                 zw = z[i][::-1] if direction == O.R2L else z[i]
                 assert rel(tail, zw[13:]) < 1e-12
 
@@ -357,3 +357,51 @@ def test_known_prefix_continues_the_same_inverse():
     zt, _ = O.af_forward(blk, x_true, O.L2R)
     x_tf, _, _ = O.af_inverse_jacobi(blk, zt, O.L2R, 8, 0.0, 8, True, x_known=x_true, n_known=1)
     assert rel(x_tf, x_true) < 1e-12
+
+
+# ---------------------------------------------------------------------------- block-size schedules
+
+def test_schedule_of_equal_blocks_is_the_uniform_call():
+    blk = tiny_block(head_std=0.2)
+    z = np.random.default_rng(15).standard_normal((2, 24, TINY.C))
+    for warm in (False, True):
+        a = O.af_inverse_jacobi(blk, z, O.L2R, 8, 1e-6, 8, warm)
+        b = O.af_inverse_jacobi(blk, z, O.L2R, [8, 8, 8], 1e-6, 8, warm)
+        for u, v in zip(a, b):
+            np.testing.assert_array_equal(u, v)
+
+
+@pytest.mark.parametrize("sizes", [[3, 5, 8, 8], [1, 2, 21], [10, 14], [24]])
+def test_any_schedule_with_enough_sweeps_is_the_sequential_inverse(sizes):
+    """The triangular guarantee per block: B_b sweeps make block b exact from
+    any start, so a schedule of any sizes (tau = 0, max_iter = largest block)
+    reproduces the token-by-token inverse, warm started or not."""
+    blk = tiny_block(head_std=0.3)
+    z = np.random.default_rng(16).standard_normal((2, 24, TINY.C))
+    xs = O.af_inverse_seq(blk, z, O.R2L)
+    for warm in (False, True):
+        xj, it, conv = O.af_inverse_jacobi(blk, z, O.R2L, sizes, 0.0, max(sizes), warm)
+        assert rel(xj, xs) < 1e-12
+        assert it.shape == (2, len(sizes)) and (it == max(sizes)).all()
+
+
+def pin_warm_start_guess():
+    """Blocks larger than a frame: tokens of the block's second frame start
+    from the last finished frame (two frames back), tokens of the first
+    frame with no finished frame start from z.  Returns the max abs error
+    against the hand-derived sources."""
+    zw = np.arange(40, dtype=np.float64).reshape(20, 2)            # 20 tokens, frames of 4
+    xw = -np.arange(40, dtype=np.float64).reshape(20, 2)
+    err = 0.0
+    g = O.warm_start_guess(xw, zw, 8, 18, 4)                       # block of positions 8..17
+    src = [4, 5, 6, 7, 4, 5, 6, 7, 4, 5]                           # p - k*4 < 8, smallest k
+    err = max(err, np.abs(g - xw[src]).max())
+    g0 = O.warm_start_guess(xw, zw, 0, 6, 4)                       # first block: nothing finished
+    err = max(err, np.abs(g0 - zw[0:6]).max())
+    g1 = O.warm_start_guess(xw, zw, 2, 9, 4)                       # positions 2..8
+    err = max(err, np.abs(g1 - np.concatenate([zw[2:4], xw[0:2], zw[6:8], xw[0:1]])).max())
+    return float(err)
+
+
+def test_warm_start_reaches_back_whole_frames():
+    assert pin_warm_start_guess() == 0.0
