@@ -1,26 +1,35 @@
 """Throughput of the STARFlow-V affine-autoregressive-flow hot path on B200.
 
-Workload (default): the shallow f_S stack -- T = 3 AF blocks of alternating
-direction (L->R, R->L, L->R), 4 layers each, d = 768, 12 heads, MLP 4x, bf16
-tensor cores -- applied per frame to 21 latent frames x 390 tokens x 192
-channels (a 5 s, 480p, 16 fps clip after a 16x/4x 48-channel VAE and 2x2
-patches).  One step = flow_stack_forward(x) -> (z, logdet) followed by the
-block-Jacobi flow_stack_inverse(z') of a fresh z' ~ N(0, 1) (B = 390, tau =
-1e-3, max_iter = 390), both over the 8190 tokens.
+Workload (default, config 3): the shallow f_S stack -- T = 3 AF blocks of
+alternating direction (L->R, R->L, L->R), 4 layers each, d = 768, 12 heads,
+MLP 4x, bf16 tensor cores -- applied per frame to latent frames of 390 tokens
+x 192 channels (480p, 16 fps, 16x/4x 48-channel VAE, 2x2 patches); 21 frames
+(a 5 s clip) per GPU.  One step = flow_stack_forward(x) -> (z, logdet) then
+the block-Jacobi flow_stack_inverse(z') of a fresh z' ~ N(0, 1) (B = 390, tau
+= 1e-3, max_iter = 390) over the frames.
 
-Reported: value = Jacobi-inverse latent tokens/s (whole job, all ranks),
-fwd_tokens_per_s, and the tensor-core roofline of the inverse graph from the
-algorithmic flops of the updates actually run.  `--impl reference` times the
+Several GPUs (`--gpus N`, one process per GPU; without torchrun the script
+relaunches itself under torch.distributed.run): the job is a clip of N x 21
+frames; rank r takes a contiguous range of frames (video_generation_b200.shard),
+runs the stack on them and the clip is assembled by one NCCL all-gather of z,
+logdet and x per step, inside the timed region.  Per-GPU work is fixed (weak
+scaling); time is the max over ranks.  The deep-flow configs (4, 5: one video
+is sequential across blocks) run one video per rank with no exchange.
+
+Reported: value = Jacobi-inverse latent tokens/s of the whole job;
+fwd_tokens_per_s; the tensor-core roofline of the inverse graph from the
+algorithmic flops of the updates actually run; e2e through pinned host
+buffers (upload of the next step's z and download of the previous step's x
+overlap the current step on a copy stream); with one GPU also configs 2, 4
+and 5 (`extra`) and the CPU oracle baselines.  `--impl reference` times the
 CPU float64 oracle on a bounded sample of the same workload instead.
-
-Multi-GPU (torchrun): each rank inverts its own clip (independent frames, no
-collective on the data path): weak scaling, max-over-ranks time.
 """
 from __future__ import annotations
 
 import argparse
 import json
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -33,9 +42,10 @@ sys.path.insert(0, ROOT)
 
 import synthetic as syn  # noqa: E402
 from video_generation_b200 import flops as FL  # noqa: E402
-from video_generation_b200 import replicas  # noqa: E402
+from video_generation_b200 import shard  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SMS = 148
 
 
 def load_peaks():
@@ -98,11 +108,20 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def count_launches(w, iters_np):
+# ----------------------------------------------------------------------------- bookkeeping
+
+def attention_may_split(w) -> bool:
+    """Whether libaf's attention launches its split-merge kernel for this workload
+    (some pass has too few query tiles to fill the GPU and keys beyond 512)."""
+    return w.shape.dtype == "bf16" and w.shape.heads * w.batch < 2 * SMS and w.L > 512
+
+
+def count_launches(w, iters_np, batch):
     """Kernels of libaf launched by one step (forward stack + inverse stack)."""
-    per_pass = 4 + 7 * w.shape.layers
+    comb = w.shape.layers if attention_may_split(w) else 0
+    per_pass = 4 + 7 * w.shape.layers + comb
     fwd = w.T * (1 + per_pass + 1)
-    inv = 0
+    inv = 1                                    # block table
     nb = w.L // w.B
     for t in range(w.T):
         inv += 1                               # call init
@@ -112,31 +131,54 @@ def count_launches(w, iters_np):
     return fwd + inv
 
 
-def run_oracle_sample(w, frames: int):
-    """The CPU oracle on `frames` frames of the workload: forward stack and Jacobi inverse.
+def frame_sharded(w) -> bool:
+    """Workloads whose sequences are single frames (the shallow stack): frames shard across ranks."""
+    return w.L == w.shape.frame_len
 
-    Frames are batch entries for the per-frame shallow stack, and the first
-    `frames` blocks of the sequence (a causal prefix) for the deep flow.
-    Returns (tokens, fwd seconds, inverse seconds, threads used)."""
-    from oracle import af_oracle as O
-    blocks = [O.Block(w.shape, syn.make_weights(w.shape, block=t)) for t in range(w.T)]
-    if w.L > w.B:
-        x = syn.workload_latents(w, "x")[:1, :frames * w.B]
-        z = syn.workload_latents(w, "z")[:1, :frames * w.B]
-    else:
-        x = syn.workload_latents(w, "x")[:frames]
-        z = syn.workload_latents(w, "z")[:frames]
-    t0 = time.perf_counter()
-    O.stack_forward(blocks, w.dirs, x)
-    t1 = time.perf_counter()
-    O.stack_inverse(blocks, w.dirs, z, w.B, w.tau, w.max_iter, bool(w.warm_start))
-    t2 = time.perf_counter()
+
+# ----------------------------------------------------------------------------- CPU oracle legs
+
+def oracle_threads():
     try:
         from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:
-        threads = os.cpu_count()
-    return x.shape[0] * x.shape[1], t1 - t0, t2 - t1, threads
+        return os.cpu_count()
+
+
+def run_oracle_sample(w, frames: int, single_thread: bool = False):
+    """The CPU oracle on `frames` frames of the workload: forward stack and Jacobi inverse.
+
+    Frames are batch entries for per-frame workloads, and the first `frames`
+    blocks of the sequence (a causal prefix) for the deep flow.
+    Returns (tokens, fwd seconds, inverse seconds, threads used, inverse flops)."""
+    from oracle import af_oracle as O
+    blocks = [O.Block(w.shape, syn.make_weights(w.shape, block=t)) for t in range(w.T)]
+    if frame_sharded(w):
+        x = syn.clip_frames(w, "x", 0, frames)
+        z = syn.clip_frames(w, "z", 0, frames)
+    else:
+        x = syn.workload_latents(w, "x")[:1, :frames * w.B]
+        z = syn.workload_latents(w, "z")[:1, :frames * w.B]
+
+    def go():
+        t0 = time.perf_counter()
+        O.stack_forward(blocks, w.dirs, x)
+        t1 = time.perf_counter()
+        _, it = O.stack_inverse(blocks, w.dirs, z, w.B, w.tau, w.max_iter, bool(w.warm_start))
+        t2 = time.perf_counter()
+        return t1 - t0, t2 - t1, it
+
+    if single_thread:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            tf, ti, it = go()
+        threads = 1
+    else:
+        tf, ti, it = go()
+        threads = oracle_threads()
+    inv_flops = FL.jacobi_flops(w.shape, it, x.shape[1], w.B)
+    return x.shape[0] * x.shape[1], tf, ti, threads, inv_flops
 
 
 def reference_arm(args, w, rank, world):
@@ -145,8 +187,9 @@ def reference_arm(args, w, rank, world):
         return
     frames = args.ref_frames
     vals = []
+    threads = 1
     for i in range(args.warmup + args.steps):
-        tok, tf, ti, threads = run_oracle_sample(w, frames)
+        tok, tf, ti, threads, _ = run_oracle_sample(w, frames)
         if i >= args.warmup:
             vals.append((tok, tf, ti))
     tok = sum(v[0] for v in vals)
@@ -166,60 +209,68 @@ def reference_arm(args, w, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
-    ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", type=int, default=3, help="workload id (3 = f_S stack, the default)")
-    ap.add_argument("--ref-frames", type=int, default=2, help="frames per oracle step (reference arm)")
-    ap.add_argument("--cpu-frames", type=int, default=2, help="frames in the cpu_baseline sample")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    args = ap.parse_args()
-    if args.warmup < 3:
-        args.warmup = 3
+def cpu_baselines(w, args, gpu_inv_flops_per_step, gpu_tokens_per_step):
+    """The oracle on bounded samples: all-core and single-thread rates; for the
+    deep flow also the time of the full inverse, extrapolated (labelled as
+    such) from the oracle's measured flop rate on the first frame."""
+    tok, tf, ti, threads, inv_fl = run_oracle_sample(w, args.cpu_frames)
+    out = {"value": tok / ti, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+           "sample": f"{args.cpu_frames} frame(s) of the workload, full T={w.T} stack Jacobi inverse "
+                     f"(forward: {tok / tf:.1f} tokens/s)"}
+    tok1, tf1, ti1, _, _ = run_oracle_sample(w, 1, single_thread=True)
+    out["single_thread_value"] = tok1 / ti1
+    out["single_thread_sample"] = "1 frame, one BLAS thread"
+    if not frame_sharded(w):
+        rate = inv_fl / ti                                  # oracle flop/s on the causal prefix
+        t_full = gpu_inv_flops_per_step / rate
+        out["extrapolated_full_inverse_s"] = t_full
+        out["extrapolated_tokens_per_s"] = gpu_tokens_per_step / t_full
+        out["extrapolation"] = ("full-sequence inverse time = its algorithmic flops (from the GPU run's "
+                                "iteration counts) / the oracle's measured flop rate on the first frame")
+    return out
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    w = syn.WORKLOADS[args.config]
 
-    if args.impl == "reference":
-        reference_arm(args, w, rank, world)
-        return
+# ----------------------------------------------------------------------------- one workload on the GPU
 
+def measure(w, args, rank, world, dist, dev, with_e2e=True):
+    """Times `args.steps` steps (forward + inverse) of workload w on this rank,
+    max over ranks.  Returns a dict of results."""
     import torch
-    import torch.distributed as dist
     from video_generation_b200 import flow
 
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-
     models = [flow.AFModel(w.shape, syn.make_weights(w.shape, block=t)) for t in range(w.T)]
-    # each rank inverts its own clip: distinct seeds per rank
-    x_np = syn.make_latents(w.batch, w.L, w.shape.C, replicas.rank_seed(syn.DATA_SEED + w.cid, rank))
-    z_np = syn.make_latents(w.batch, w.L, w.shape.C, replicas.rank_seed(syn.DATA_SEED + w.cid + 100, rank))
+    sharded = frame_sharded(w) and world > 1
+    if frame_sharded(w):
+        n_frames = w.batch * world                      # weak scaling: w.batch frames per GPU
+        lo, hi = shard.frame_ranges(n_frames, world)[rank]
+        x_np = syn.clip_frames(w, "x", lo, hi)
+        z_np = syn.clip_frames(w, "z", lo, hi)
+    else:                                               # one video per rank
+        n_frames = world
+        x_np = syn.make_latents(1, w.L, w.shape.C, syn.DATA_SEED + w.cid + 1000 * rank)
+        z_np = syn.make_latents(1, w.L, w.shape.C, syn.DATA_SEED + w.cid + 100 + 1000 * rank)
+    batch = x_np.shape[0]
     x = torch.from_numpy(x_np).to(dev)
     z_in = torch.from_numpy(z_np).to(dev)
-    ws_f = models[0].workspace(w.batch, w.L, w.L, device=dev)
-    ws_i = models[0].workspace(w.batch, w.L, w.B, device=dev)
+    ws_f = models[0].workspace(batch, w.L, w.L, device=dev)
+    ws_i = models[0].workspace(batch, w.L, w.B, device=dev)
     zf = torch.empty_like(x)
-    ld = torch.empty(w.batch, dtype=torch.float32, device=dev)
+    ld = torch.empty(batch, dtype=torch.float32, device=dev)
     xi = torch.empty_like(x)
-    iters = torch.zeros((w.T, w.batch, w.L // w.B), dtype=torch.int32, device=dev)
+    iters = torch.zeros((w.T, batch, w.L // w.B), dtype=torch.int32, device=dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)   # > 126 MB L2
     st = torch.cuda.current_stream()
 
     def fwd():
         flow.flow_stack_forward(models, w.dirs, x, ws=ws_f, z=zf, logdet=ld)
+        if sharded:
+            shard.gather_frames(zf, n_frames, dist)
+            shard.gather_frames(ld, n_frames, dist)
 
-    def inv():
-        flow.flow_stack_inverse(models, w.dirs, z_in, w.B, w.tau, w.max_iter, w.warm_start, ws=ws_i, x=xi,
+    def inv(zsrc=z_in, xdst=xi):
+        flow.flow_stack_inverse(models, w.dirs, zsrc, w.B, w.tau, w.max_iter, w.warm_start, ws=ws_i, x=xdst,
                                 iters=iters)
+        return shard.gather_frames(xdst, n_frames, dist) if sharded else xdst
 
     for _ in range(args.warmup):
         fwd()
@@ -234,7 +285,7 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev.index) as clk:
         for i in range(args.steps):
             flush.zero_()                         # L2 flushed between timed steps
             ev[i][0].record(st)
@@ -248,47 +299,145 @@ def main():
         dist.barrier()
     t_fwd = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
     t_inv = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
-    t = replicas.max_over_ranks(torch.tensor([t_fwd, t_inv], dtype=torch.float64, device=dev), dist)
+    t = shard.max_over_ranks(torch.tensor([t_fwd, t_inv], dtype=torch.float64, device=dev), dist)
     t_fwd, t_inv = float(t[0]), float(t[1])
+    it_np = [a.cpu().numpy() for a in iters_all]
+    r = {"t_fwd": t_fwd, "t_inv": t_inv, "it_np": it_np, "batch": batch, "clk": clk.summary(),
+         "tokens_per_step_rank": batch * w.L,
+         "inv_flops_rank": sum(FL.jacobi_flops(w.shape, a, w.L, w.B) for a in it_np),
+         "fwd_flops_rank": args.steps * FL.forward_flops(w.shape, batch, w.L, w.T),
+         "launches": sum(count_launches(w, a, batch) for a in it_np) // args.steps}
 
-    # algorithmic work from the iterations actually run
-    it_np = [i.cpu().numpy() for i in iters_all]
-    inv_flops = sum(FL.jacobi_flops(w.shape, a, w.L, w.B) for a in it_np)
-    fwd_flops = args.steps * FL.forward_flops(w.shape, w.batch, w.L, w.T)
-    tok = w.batch * w.L * args.steps * world
-    peaks, peak_kind = load_peaks()
-    inv_tf = inv_flops / t_inv / 1e12
-    fwd_tf = fwd_flops / t_fwd / 1e12
-    launches = sum(count_launches(w, a) for a in it_np)
+    if with_e2e:
+        # end to end through the public API with host buffers: every step uploads
+        # its z from pinned memory and downloads its x; the copies of step i+1
+        # (upload) and i-1 (download) overlap step i on a copy stream, the buffers
+        # double-buffered
+        cp = torch.cuda.Stream(device=dev)
+        z_host = torch.from_numpy(z_np).pin_memory()
+        n_out = batch * world if sharded else batch
+        x_host = torch.empty((n_out, w.L, w.shape.C), dtype=torch.float32).pin_memory()
+        z_dev = [torch.empty_like(z_in) for _ in range(2)]
+        x_dev = [torch.empty_like(z_in) for _ in range(2)]
+        up = [torch.cuda.Event() for _ in range(2)]
+        done = [torch.cuda.Event() for _ in range(2)]
+        down = [torch.cuda.Event() for _ in range(2)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0.record(st)
+        cp.wait_stream(st)
+        for i in range(args.steps):
+            j = i % 2
+            with torch.cuda.stream(cp):
+                if i >= 2:
+                    cp.wait_event(done[j])               # z_dev[j] read by step i-2's inverse
+                z_dev[j].copy_(z_host, non_blocking=True)
+                up[j].record(cp)
+            st.wait_event(up[j])
+            if i >= 2:
+                st.wait_event(down[j])                   # x_dev[j] downloaded by step i-2
+            out = inv(z_dev[j], x_dev[j])
+            done[j].record(st)
+            with torch.cuda.stream(cp):
+                cp.wait_event(done[j])
+                x_host.copy_(out, non_blocking=True)
+                down[j].record(cp)
+        st.wait_stream(cp)
+        t1.record(st)
+        torch.cuda.synchronize()
+        te = shard.max_over_ranks(torch.tensor([t0.elapsed_time(t1) / 1e3], dtype=torch.float64, device=dev), dist)
+        r["t_e2e"] = float(te[0])
+        r["h2d"] = z_host.numel() * 4
+        r["d2h"] = x_host.numel() * 4
+    for m in models:
+        m.close()
+    return r
 
-    # end to end through the public API with host buffers: pinned z -> device,
-    # inverse, x -> pinned host, every step inside the timed region
-    z_host = torch.from_numpy(z_np).pin_memory()
-    x_host = torch.empty_like(z_host).pin_memory()
-    z_dev = torch.empty_like(z_in)
-    e2e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+
+def extra_line(w, args, dev, peaks):
+    """One more workload on this GPU (single process), as a dict for the `extra` key."""
+    r = measure(w, args, 0, 1, None, dev, with_e2e=False)
+    tok = r["tokens_per_step_rank"] * args.steps
+    inv_tf = r["inv_flops_rank"] / r["t_inv"] / 1e12
+    out = {"workload": w.name, "steps": args.steps, "warmup": args.warmup,
+           "inverse_tokens_per_s": tok / r["t_inv"], "fwd_tokens_per_s": tok / r["t_fwd"],
+           "inverse_tflops": inv_tf, "fwd_tflops": r["fwd_flops_rank"] / r["t_fwd"] / 1e12,
+           "inverse_frac_of_bf16_peak": inv_tf / peaks["bf16_tflops"],
+           "mean_iters_per_block": float(np.mean([a.mean() for a in r["it_np"]])),
+           "clocks": r["clk"]}
+    return out, r
+
+
+# ----------------------------------------------------------------------------- main
+
+def relaunch_under_torchrun(args):
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    os.execv(sys.executable, cmd)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", type=int, default=3, help="workload id (3 = f_S stack, the default)")
+    ap.add_argument("--ref-frames", type=int, default=2, help="frames per oracle step (reference arm)")
+    ap.add_argument("--cpu-frames", type=int, default=2, help="frames in the cpu_baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip configs 2, 4, 5 in a one-GPU run")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        relaunch_under_torchrun(args)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        sys.stderr.write(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}\n")
+        sys.exit(2)
+    w = syn.WORKLOADS[args.config]
+
+    if args.impl == "reference":
+        reference_arm(args, w, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
     if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e2e_ev[0].record(st)
-    for _ in range(args.steps):
-        z_dev.copy_(z_host, non_blocking=True)
-        flow.flow_stack_inverse(models, w.dirs, z_dev, w.B, w.tau, w.max_iter, w.warm_start, ws=ws_i, x=xi,
-                                iters=iters)
-        x_host.copy_(xi, non_blocking=True)
-    e2e_ev[1].record(st)
-    torch.cuda.synchronize()
-    t_e2e = replicas.max_over_ranks(
-        torch.tensor([e2e_ev[0].elapsed_time(e2e_ev[1]) / 1e3], dtype=torch.float64, device=dev), dist)
-    e2e_val = tok / float(t_e2e[0])
-    bytes_step = w.batch * w.L * w.shape.C * 4
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        ctok, ctf, cti, threads = run_oracle_sample(w, args.cpu_frames)
-        cpu = {"value": ctok / cti, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-               "sample": f"{args.cpu_frames} of {w.batch} frames, full T={w.T} stack Jacobi inverse "
-                         f"(forward: {ctok / ctf:.1f} tokens/s)"}
+    r = measure(w, args, rank, world, dist if world > 1 else None, dev)
+    peaks, peak_kind = load_peaks()
+    tok = r["tokens_per_step_rank"] * args.steps * world
+    inv_tf_rank = r["inv_flops_rank"] / r["t_inv"] / 1e12
+    fwd_tf_rank = r["fwd_flops_rank"] / r["t_fwd"] / 1e12
+
+    extras, cpu = {}, None
+    if world == 1 and rank == 0:
+        if not args.no_extras and args.config == 3:
+            ex_args = argparse.Namespace(**vars(args))
+            for cid, steps in ((2, max(3, min(args.steps, 20))), (4, 2), (5, 1)):
+                ex_args.steps = steps
+                try:
+                    extras[syn.WORKLOADS[cid].name], _ = extra_line(syn.WORKLOADS[cid], ex_args, dev, peaks)
+                except Exception as e:          # an extra must not lose the headline line
+                    extras[syn.WORKLOADS[cid].name] = {"error": repr(e)[:200]}
+        if not args.no_cpu_baseline:
+            cpu = cpu_baselines(w, args, r["inv_flops_rank"] / args.steps, r["tokens_per_step_rank"])
 
     if world > 1:
         dist.barrier()
@@ -297,28 +446,32 @@ def main():
         return
     peak = peaks["bf16_tflops"]
     line = {
-        "metric": "jacobi_inverse_latent_tokens_per_s", "value": tok / t_inv, "unit": "tokens/s",
+        "metric": "jacobi_inverse_latent_tokens_per_s", "value": tok / r["t_inv"], "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * (t_fwd + t_inv) / args.steps, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": 1e3 * (r["t_fwd"] + r["t_inv"]) / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "frames": w.batch, "tokens_per_frame": w.L, "T": w.T,
-                   "layers": w.shape.layers, "d_model": w.shape.d, "B": w.B, "tau": w.tau,
-                   "max_iter": w.max_iter, "l2": "flushed between steps", "parallelism": f"replicas{world}"},
-        "fwd_tokens_per_s": tok / t_fwd,
-        "fwd_tflops": fwd_tf,
-        "inverse_tflops": inv_tf,
-        "mean_iters_per_block": float(np.mean([a.mean() for a in it_np])),
-        "max_iters_per_block": int(max(a.max() for a in it_np)),
-        "roofline": {"bound": "tensor", "achieved": inv_tf, "peak": peak, "unit": "TFLOP/s",
-                     "frac": inv_tf / peak, "traffic": None,
-                     "kernel": "flow_stack_inverse graph (tcgen05 GEMMs dominate)",
+        "config": {"workload": w.name, "frames_per_gpu": r["batch"] if frame_sharded(w) else None,
+                   "tokens_per_frame": w.shape.frame_len, "L": w.L, "T": w.T, "layers": w.shape.layers,
+                   "d_model": w.shape.d, "B": w.B, "tau": w.tau, "max_iter": w.max_iter,
+                   "l2": "flushed between steps",
+                   "parallelism": (f"frames{world}" if frame_sharded(w) else f"replicas{world}")},
+        "fwd_tokens_per_s": tok / r["t_fwd"],
+        "fwd_tflops": fwd_tf_rank * world,
+        "inverse_tflops": inv_tf_rank * world,
+        "mean_iters_per_block": float(np.mean([a.mean() for a in r["it_np"]])),
+        "max_iters_per_block": int(max(a.max() for a in r["it_np"])),
+        "roofline": {"bound": "tensor", "achieved": inv_tf_rank, "peak": peak, "unit": "TFLOP/s",
+                     "frac": inv_tf_rank / peak, "traffic": None,
+                     "kernel": "flow_stack_inverse graph, per GPU (tcgen05 GEMMs dominate)",
                      "peak_kind": f"bf16 dense burst, {peak_kind}",
-                     "frac_of_sustained": inv_tf / peaks.get("bf16_tflops_sustained", peak)},
-        "clocks": clk.summary(),
-        "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": bytes_step,
-                "d2h_bytes_per_step": bytes_step},
-        "gpu_launches": launches,
+                     "frac_of_sustained": inv_tf_rank / peaks.get("bf16_tflops_sustained", peak)},
+        "clocks": r["clk"],
+        "e2e": {"value": tok / r["t_e2e"], "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": r["launches"] * args.steps,
     }
+    if extras:
+        line["extra"] = extras
     if cpu is not None:
         line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)

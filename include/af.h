@@ -11,7 +11,7 @@
  *   - its inverse by video-aware block-wise Jacobi iteration
  *     x^(k+1) = mu(x^(k)*m) + sigma(x^(k)*m) * z, blocks of B tokens in
  *     sequence, parallel inside a block, finished blocks kept in a KV cache,
- *     warm start from the previous block's converged x, stop when
+ *     warm start from the previous frame's converged x, stop when
  *     ||x^(k+1)-x^(k)||^2 / ||x^(k+1)||^2 < tau (section "Key design 3:
  *     video-aware block-wise Jacobi iteration");
  *   - stacks of T blocks of alternating direction, inverted last to first
@@ -90,10 +90,11 @@ af_status af_model_create(const af_config* cfg, const float* const* tensors, int
                           af_model** out);
 af_status af_model_destroy(af_model* m);
 
-/* Workspace bytes for a call on `batch` sequences of L tokens with Jacobi
- * block size B (pass B = L for af_forward).  Includes the KV cache of all
- * layers over L positions.  The same workspace serves every block of a
- * stack made of models with the same config.  0 on bad arguments. */
+/* Workspace bytes for a call on `batch` sequences of L tokens whose Jacobi
+ * blocks hold at most B tokens (pass B = L for af_forward; B need not divide
+ * L).  Includes the KV cache of all layers over L positions.  The same
+ * workspace serves every block of a stack made of models with the same
+ * config.  0 on bad arguments. */
 size_t af_workspace_bytes(const af_model* m, int batch, int L, int B);
 
 /* Forward pass of one AF block: z and logdet (= -sum_{i,c} s_{i,c} per
@@ -103,11 +104,18 @@ af_status af_forward(const af_model* m, const float* x, int batch, int L, af_dir
 
 /* Block-wise Jacobi inverse of one AF block.  Requires L % B == 0,
  * max_iter >= 1, tau >= 0 and finite.  Block b starts from z_b, or, when
- * warm_start != 0 and b > 0, from block b-1's final x.  A sample leaves the
- * iteration of a block at the first update whose residual is < tau (0/0
- * counts as converged); iters[s * (L/B) + b] counts the updates computed.
- * All iterations, tests and block changes run on the device: one graph
- * launch per call, no host round trip per iteration. */
+ * warm_start != 0, from the previous frame's converged state ("Key design
+ * 3": a new frame is warm-started from the previous frame's converged x):
+ * the token at working-order position p starts from the converged x at
+ * p - k*frame_len, the same spatial position in the most recent finished
+ * frame (smallest k >= 1 landing before the block), and from z where no
+ * frame before it has finished.  With B = frame_len this is "block b starts
+ * from block b-1's final x".  A sample leaves the iteration of a block at
+ * the first update whose residual is < tau (0/0 counts as converged);
+ * iters[s * (L/B) + b] counts the updates computed.  All iterations, tests
+ * and block changes run on the device: one graph launch per call (after one
+ * small kernel that writes the block table into ws), no host round trip per
+ * iteration. */
 af_status af_inverse_jacobi(const af_model* m, const float* z, int batch, int L, af_dir dir,
                             int B, float tau, int max_iter, int warm_start, float* x,
                             int32_t* iters, void* ws, size_t ws_bytes, void* stream);
@@ -125,6 +133,68 @@ af_status flow_stack_inverse(const af_model* const* blocks, const af_dir* dirs, 
                              int warm_start, float* x, int32_t* iters, void* ws,
                              size_t ws_bytes, void* stream);
 
+/* Block-wise Jacobi inverse with a schedule of block sizes, over a range of
+ * blocks (section "Key findings": runtime is U-shaped in the block size, and
+ * the method uses a smaller block for the first frame and larger ones after;
+ * "A complete example": I2V / V2V generation continues a sequence whose
+ * first frames are observed).  block_sizes[0 .. n_blocks-1] (HOST array,
+ * each >= 1, summing to L) cut the sequence into consecutive blocks; the
+ * call inverts blocks b_begin .. b_end-1 (0 <= b_begin < b_end <= n_blocks)
+ * with the rules of af_inverse_jacobi (warm start per frame as described
+ * there), writing x and iters[s * n_blocks + b] of those blocks only.
+ * ws needs af_workspace_bytes(m, batch, L, largest block).  When
+ * b_begin > 0, x must already hold the final values of the blocks before
+ * b_begin, and ws the K/V of the positions before block b_begin - 1 -- as
+ * left by an earlier call on the same ws that ended at b_begin, or by
+ * af_prefix_encode of those positions (the first update of block b_begin
+ * recomputes block b_begin - 1's K/V from x).  af_last_convergence counts
+ * accumulate over calls and restart with a call whose b_begin is 0. */
+af_status af_inverse_jacobi_schedule(const af_model* m, const float* z, int batch, int L, af_dir dir,
+                                     const int* block_sizes, int n_blocks, int b_begin, int b_end, float tau,
+                                     int max_iter, int warm_start, float* x, int32_t* iters, void* ws,
+                                     size_t ws_bytes, void* stream);
+
+/* Flow-encode of observed tokens ("A complete example": I2V / V2V -- the
+ * flow's forward pass writes the observed frames into the KV cache, no
+ * separate encoder): writes the K/V of working-order positions
+ * 0 .. n_tokens-1, computed from x, into the cache of a workspace laid out
+ * for (batch, L, B) (size af_workspace_bytes(m, batch, L, B)), ready for
+ * af_inverse_jacobi_schedule to continue at the block starting at n_tokens
+ * (x must then hold the observed tokens too).  Runs passes of at most 2B
+ * positions each; writes nothing but the cache and workspace scratch.
+ * Requires 1 <= n_tokens <= L. */
+af_status af_prefix_encode(const af_model* m, const float* x, int batch, int L, af_dir dir, int B, int n_tokens,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* Bytes of the shallow-side workspace of flow_pipeline_inverse for T shallow
+ * blocks (config of `shallow`), `batch` videos, frames of frame_len tokens. */
+size_t flow_pipeline_workspace_bytes(const af_model* shallow, int T, int batch, int frame_len);
+
+/* Pipelined deep -> shallow decoding ("Key design 3": the deep flow
+ * f_D runs without pause while the shallow blocks f_S consume its output
+ * frame by frame; end-to-end latency is set by the deep block):
+ * x = f_S^{-1}(f_D^{-1}(z)) with f_S applied to each frame on its own.
+ * f_D^{-1} (`deep`, direction L->R, blocks of B tokens, tau, max_iter_deep,
+ * warm_start) runs on stream_deep, one frame's blocks per graph launch;
+ * after each frame an event lets stream_shallow run the T-block stack
+ * inverse of that frame (blocks shallow[0..T-1], directions shallow_dirs,
+ * one Jacobi block per frame, no warm start, tau, max_iter_shallow) while
+ * the deep flow moves on.  z, x: [batch, L, C]; frame_len = the deep model's
+ * frame_len (the shallow models must accept frames of that length and C);
+ * L % frame_len == 0 and frame_len % B == 0.  iters_deep [batch, L/B],
+ * iters_shallow [T, batch, L/frame_len].  ws_deep: af_workspace_bytes(deep,
+ * batch, L, B); ws_shallow: flow_pipeline_workspace_bytes(shallow[0], T,
+ * batch, frame_len).  The two streams may be the same stream (no overlap).
+ * On return all work is enqueued; stream_deep waits for the last frame's
+ * shallow work, so synchronising stream_deep covers the whole call.  The
+ * result is bit-identical to af_inverse_jacobi followed by
+ * flow_stack_inverse of each frame. */
+af_status flow_pipeline_inverse(const af_model* deep, const af_model* const* shallow, const af_dir* shallow_dirs, int T,
+                                const float* z, int batch, int L, int B, float tau, int max_iter_deep,
+                                int max_iter_shallow, int warm_start, float* x, int32_t* iters_deep,
+                                int32_t* iters_shallow, void* ws_deep, size_t ws_deep_bytes, void* ws_shallow,
+                                size_t ws_shallow_bytes, void* stream_deep, void* stream_shallow);
+
 /* af_forward for callers that cannot allocate device memory -- a host that
  * owns the whole GPU memory through its own allocator, or a plugin that is
  * handed only its input and output buffers, and so cannot provide a
@@ -141,8 +211,10 @@ af_status af_forward_noalloc(const af_model* m, const float* x, int batch, int L
                              float* z, float* logdet, void* stream);
 
 /* Synchronises `stream` and reports how many (sample, block) pairs of the
- * last inverse call on this workspace stopped at max_iter without passing
- * the test: AF_OK if none, AF_NOT_CONVERGED otherwise (*n_unconverged set). */
+ * last inverse call on this workspace (of the calls since the last one that
+ * started at block 0, for af_inverse_jacobi_schedule) stopped at max_iter
+ * without passing the test: AF_OK if none, AF_NOT_CONVERGED otherwise
+ * (*n_unconverged set). */
 af_status af_last_convergence(void* ws, int* n_unconverged, void* stream);
 
 /* Synchronises the device and returns AF_ERR_DEVICE (and clears the flag)

@@ -163,3 +163,16 @@ def make_latents(batch: int, L: int, C: int, seed: int, scale: float = 1.0) -> n
 def workload_latents(w: Workload, which: str = "x") -> np.ndarray:
     off = {"x": 0, "z": 100}[which]
     return make_latents(w.batch, w.L, w.shape.C, DATA_SEED + w.cid + off)
+
+
+def clip_frames(w: Workload, which: str, lo: int, hi: int) -> np.ndarray:
+    """Frames lo..hi-1 of a clip of per-frame sequences (the shallow stack's
+    workload: frames are its batch), [hi - lo, L, C].  Frame f is drawn from
+    its own seed, so a process can draw any range of a clip of any length
+    without drawing the rest."""
+    off = {"x": 0, "z": 100}[which]
+    out = np.empty((hi - lo, w.L, w.shape.C), np.float32)
+    for i, f in enumerate(range(lo, hi)):
+        rng = np.random.default_rng([DATA_SEED + w.cid + off, f])
+        out[i] = rng.standard_normal((w.L, w.shape.C), dtype=np.float32)
+    return out

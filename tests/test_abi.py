@@ -12,7 +12,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def _declared():
     src = open(os.path.join(ROOT, "include", "af.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(af_\w+|flow_stack_\w+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(af_\w+|flow_\w+)\s*\(", src)))
 
 
 @pytest.fixture(scope="module")

@@ -23,7 +23,7 @@
 using namespace af;
 
 namespace af {
-int g_pdl = 1;
+thread_local int g_pdl = 1;
 }
 
 namespace {
@@ -74,11 +74,14 @@ struct af_model {
   float* b_head;      // interleaved the same way
   int* d_err;
   int num_sms;
+  int device;         // the CUDA device holding the weights
+  int pdl;            // launch with programmatic dependent launch (see af_kernels.h)
   std::vector<void*> allocs;
   // graph cache (keyed by every pointer and scalar baked into the graph)
   std::map<std::string, cudaGraphExec_t> graphs;
   std::vector<std::string> graph_order;
   cudaStream_t cap, cap2;   // private streams used for capture only
+  cudaEvent_t ev_frame = nullptr, ev_done = nullptr;   // pipelined decoding (created on first use)
 };
 
 namespace {
@@ -97,13 +100,16 @@ struct Bufs {
   void* kv;
   size_t kv_bytes;
   float* tmp;
+  int* btab;      // Jacobi block table (af_common.cuh)
   float* opart;   // split-attention partials (bf16 path)
   float* mlpart;
   int nsplit;
   size_t total;
 };
 
-int rows_per_sample(int L, int B) { return B >= L ? L : 2 * B; }
+// Rows per sample a pass may carry: a Jacobi update of a block of at most B
+// tokens, plus the previous block's tokens on the update that commits them.
+int rows_per_sample(int L, int B) { return B >= L ? L : (2 * B < L ? 2 * B : L); }
 
 Bufs carve(const af_model* m, void* ws, int batch, int L, int B) {
   const af_config& c = m->cfg;
@@ -129,6 +135,7 @@ Bufs carve(const af_model* m, void* ws, int batch, int L, int B) {
   b.kv_bytes = es * (size_t)c.layers * 2 * batch * L * c.d;
   b.kv = take(b.kv_bytes);
   b.tmp = (float*)take(sizeof(float) * (size_t)batch * L * c.C);
+  b.btab = (int*)take(sizeof(int) * btab_ints(L));
   b.nsplit = m->bf ? attn_tc_splits(batch, c.heads, rows_per_sample(L, B), L, m->num_sms) : 1;
   if (b.nsplit > 1) {
     b.opart = (float*)take(sizeof(float) * (size_t)b.nsplit * mmax * c.d);
@@ -249,7 +256,7 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
       }
       if (!gemm(EPI_QKV, tA_a, w.w_qkv, 3 * d, d, eq)) { set_err("GEMM plan failed (qkv)"); return AF_ERR_CUDA; }
       if (!launch_attn_tc2(b.ctl, q, (const bf16*)kvl, (const bf16*)(kvl + kv_layer), a, b.opart, b.mlpart, b.nsplit,
-                           batch, L, d, c.heads, r_max, m_max, m->d_err, st)) {
+                           batch, L, d, c.heads, r_max, m_max, m->num_sms, m->d_err, st)) {
         set_err("attention plan failed");
         return AF_ERR_CUDA;
       }
@@ -307,17 +314,38 @@ struct JacobiJob {
   bool reset_nonconv;
 };
 
+// Block schedule of a Jacobi call, as held on the host before it is written
+// to the workspace's block table.
+struct Schedule {
+  std::vector<int> starts;   // nb + 1 start positions, the last = L
+  int b_begin, b_end;
+  int B_max;                 // the largest block
+  bool uniform;              // every block the same size
+};
+
+Schedule uniform_schedule(int L, int B) {
+  Schedule sc;
+  for (int p = 0; p <= L; p += B) sc.starts.push_back(p);
+  sc.b_begin = 0;
+  sc.b_end = L / B;
+  sc.B_max = B;
+  sc.uniform = true;
+  return sc;
+}
+
 // Capture the block-Jacobi inverse of one AF block into the stream `cs`,
 // which is capturing: [call init] WHILE(blocks) { [block init]
 // WHILE(updates) { pass; [jacobi step] } [block advance] }.
-af_status capture_jacobi(const JacobiJob& jb, const Bufs& b, int batch, int L, int B, float tau, int max_iter,
+// The block sizes, the number of blocks and the range of blocks come from the
+// workspace's block table at run time; B_max (the largest block) sizes the
+// passes, so one graph serves every schedule and range with that bound.
+af_status capture_jacobi(const JacobiJob& jb, const Bufs& b, int batch, int L, int B_max, float tau, int max_iter,
                          int warm, cudaStream_t cs) {
   const af_model* m = jb.m;
-  const int nb = L / B;
   const int G = (2 * m->cfg.C) / 16;
-  const int r_max = rows_per_sample(L, B);
+  const int r_max = rows_per_sample(L, B_max);
   const int m_max = batch * r_max;
-  launch_call_init(b.ctl, jb.reset_nonconv ? 1 : 0, cs);
+  launch_call_init(b.ctl, b.btab, jb.reset_nonconv ? 1 : 0, cs);
   cudaGraphConditionalHandle h_outer, h_inner;
   cudaGraph_t body_outer, body_inner;
   af_status s = add_while(cs, &h_outer, 1, cudaGraphCondAssignDefault, &body_outer);
@@ -337,7 +365,11 @@ af_status capture_jacobi(const JacobiJob& jb, const Bufs& b, int batch, int L, i
       set_err("conditional handle creation failed"); rc = AF_ERR_CUDA;
     }
     if (!rc) {
-      launch_block_init(b.ctl, b.active, jb.z, jb.x, batch, L, m->cfg.C, B, jb.dir, warm, h_inner, cs2);
+      // bf16: V rows of layer l at kv + (2l + 1) * (batch * L * d) elements
+      const size_t kv_layer = (size_t)batch * L * m->cfg.d * 2;
+      bf16* vtail = m->bf ? (bf16*)((char*)b.kv + kv_layer) : nullptr;
+      launch_block_init(b.ctl, b.btab, b.active, jb.z, jb.x, batch, L, m->cfg.C, B_max, m->cfg.frame_len, jb.dir, warm,
+                        vtail, 2 * kv_layer, m->cfg.layers, m->cfg.d, h_inner, cs2);
       cudaStreamCaptureStatus st2;
       cudaGraph_t g2;
       const cudaGraphNode_t* deps = nullptr;
@@ -358,7 +390,7 @@ af_status capture_jacobi(const JacobiJob& jb, const Bufs& b, int batch, int L, i
           body_inner = p.conditional.phGraph_out[0];
         }
       }
-      if (!rc) launch_block_advance(b.ctl, nb, h_outer, cs2);
+      if (!rc) launch_block_advance(b.ctl, b.btab, h_outer, cs2);
     }
     cudaGraph_t dummy;
     if (cudaStreamEndCapture(cs2, &dummy) != cudaSuccess && !rc) { set_err("end of block-loop capture failed"); rc = AF_ERR_CUDA; }
@@ -369,7 +401,7 @@ af_status capture_jacobi(const JacobiJob& jb, const Bufs& b, int batch, int L, i
     }
     HeadIO hio{1, jb.z, jb.x};
     rc = enqueue_pass(m, b, batch, L, jb.dir, m_max, r_max, jb.x, hio, cs2);
-    if (!rc) launch_jacobi_step(b.ctl, b.active, b.part, batch, B, G, tau, max_iter, jb.iters, nb, h_inner, cs2);
+    if (!rc) launch_jacobi_step(b.ctl, b.btab, b.active, b.part, batch, G, tau, max_iter, jb.iters, h_inner, cs2);
     if (cudaStreamEndCapture(cs2, &dummy) != cudaSuccess && !rc) { set_err("end of update capture failed"); rc = AF_ERR_CUDA; }
   } while (0);
   return rc;
@@ -381,6 +413,7 @@ af_status graph_run(const af_model* mc, const std::string& key, cudaStream_t st,
   auto it = m->graphs.find(key);
   if (it == m->graphs.end()) {
     cudaGraphExec_t ex;
+    g_pdl = m->pdl;
     for (int attempt = 0;; ++attempt) {
       cudaGraph_t g;
       CK(cudaGraphCreate(&g, 0));
@@ -395,6 +428,7 @@ af_status graph_run(const af_model* mc, const std::string& key, cudaStream_t st,
       cudaGetLastError();
       if (attempt == 0 && g_pdl) {   // programmatic edges refused here: plain edges instead
         g_pdl = 0;
+        m->pdl = 0;
         continue;
       }
       if (s) return s;
@@ -458,8 +492,10 @@ af_status build_forward(void* vctx, cudaStream_t cs) {
   FwdCtx* c = static_cast<FwdCtx*>(vctx);
   const int G = (2 * c->blocks[0]->cfg.C) / 16;
   const int m_max = c->batch * c->L;
-  // keys past a tile's last needed position are masked, but must be finite
-  if (c->blocks[0]->bf) CK(cudaMemsetAsync(c->b.kv, 0, c->b.kv_bytes, cs));
+  // No cache clearing: a forward pass writes K / V of every position before
+  // its attention reads them; the key tile past a sample's last position
+  // holds the next sample's rows (written by the same pass) or lies past the
+  // cache, where the TMA load fills zeros.
   for (int t = 0; t < c->T; ++t) {
     // block t writes z when T-1-t is even, else tmp; block t reads what t-1 wrote
     const float* in = t == 0 ? c->x : (((c->T - t) % 2 == 0) ? c->z : c->b.tmp);
@@ -477,7 +513,7 @@ af_status build_forward(void* vctx, cudaStream_t cs) {
 struct InvCtx {
   const af_model* const* blocks;
   const af_dir* dirs;
-  int T, batch, L, B, max_iter, warm;
+  int T, batch, L, B_max, nb, max_iter, warm;
   float tau;
   const float* z;
   float* x;
@@ -487,27 +523,96 @@ struct InvCtx {
 
 af_status build_inverse(void* vctx, cudaStream_t cs) {
   InvCtx* c = static_cast<InvCtx*>(vctx);
-  const int nb = c->L / c->B;
-  if (c->blocks[0]->bf) CK(cudaMemsetAsync(c->b.kv, 0, c->b.kv_bytes, cs));
+  // the masked V rows each block's attention reads are zeroed by its block init
   for (int t = c->T - 1; t >= 0; --t) {
     float* out = (t % 2 == 0) ? c->x : c->b.tmp;
     const float* in = (t == c->T - 1) ? c->z : ((((t + 1) % 2) == 0) ? c->x : c->b.tmp);
-    JacobiJob jb{c->blocks[t], in, out, c->dirs[t], c->iters + (size_t)t * c->batch * nb, t == c->T - 1};
-    af_status s = capture_jacobi(jb, c->b, c->batch, c->L, c->B, c->tau, c->max_iter, c->warm, cs);
+    JacobiJob jb{c->blocks[t], in, out, c->dirs[t], c->iters + (size_t)t * c->batch * c->nb, t == c->T - 1};
+    af_status s = capture_jacobi(jb, c->b, c->batch, c->L, c->B_max, c->tau, c->max_iter, c->warm, cs);
     if (s) return s;
   }
   CK(cudaGetLastError());
   return AF_OK;
 }
 
-af_status stack_checks(const af_model* const* blocks, const af_dir* dirs, int T) {
+// Writes the schedule into the workspace's block table on `st`, then runs
+// (capturing on first use) the Jacobi graph of the stack.  The graph depends
+// on B_max, not on the schedule or range, which are data.
+af_status run_inverse(const af_model* const* blocks, const af_dir* dirs, int T, const float* z, int batch, int L,
+                      const Schedule& sc, float tau, int max_iter, int warm, float* x, int32_t* iters, void* ws,
+                      cudaStream_t st, bool write_table = true) {
+  const int nb = (int)sc.starts.size() - 1;
+  InvCtx c{blocks, dirs, T, batch, L, sc.B_max, nb, max_iter, warm ? 1 : 0, tau, z, x, iters,
+           carve(blocks[0], ws, batch, L, sc.B_max)};
+  g_pdl = blocks[0]->pdl;
+  if (write_table) launch_table_write(c.b.btab, sc.starts.data(), nb, sc.b_begin, sc.b_end, st);
+  CK(cudaGetLastError());
+  uint32_t taubits;
+  memcpy(&taubits, &tau, 4);
+  std::string key = keyf("inv", {(long long)z, (long long)x, (long long)iters, (long long)ws, batch, L, sc.B_max, nb,
+                                 (long long)taubits, max_iter, c.warm, T});
+  for (int t = 0; t < T; ++t) key += keyf("", {(long long)blocks[t], dirs[t]});
+  return graph_run(blocks[0], key, st, build_inverse, &c);
+}
+
+// The work of a call runs on the current device; every model's weights must
+// live there, and so must the stream (when it is not the default stream).
+af_status device_checks(const af_model* m, cudaStream_t st) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); set_err("no current CUDA device"); return AF_ERR_CUDA; }
+  if (dev != m->device) {
+    set_err("the model's weights are on device %d but device %d is current", m->device, dev);
+    return AF_ERR_ARG;
+  }
+  if (st) {
+    int sdev = -1;
+    if (cudaStreamGetDevice(st, &sdev) != cudaSuccess) {
+      cudaGetLastError();
+      set_err("the stream is not a valid CUDA stream");
+      return AF_ERR_ARG;
+    }
+    if (sdev != dev) { set_err("the stream belongs to device %d, the model to device %d", sdev, dev); return AF_ERR_ARG; }
+  }
+  return AF_OK;
+}
+
+struct EncCtx {
+  const af_model* m;
+  const float* x;
+  int batch, L, B, n_tokens, dir;
+  Bufs b;
+};
+
+// Flow-encode of observed tokens 0 .. n_tokens-1 into the KV cache: passes of
+// at most rows_per_sample(L, B) positions, in order, each attending the cache
+// of the passes before it; no head output.
+af_status build_encode(void* vctx, cudaStream_t cs) {
+  EncCtx* c = static_cast<EncCtx*>(vctx);
+  const af_model* m = c->m;
+  const int r_max = rows_per_sample(c->L, c->B);
+  const int m_max = c->batch * r_max;
+  const size_t kv_layer = (size_t)c->batch * c->L * m->cfg.d * 2;
+  bf16* vtail = m->bf ? (bf16*)((char*)c->b.kv + kv_layer) : nullptr;
+  for (int p0 = 0; p0 < c->n_tokens; p0 += r_max) {
+    const int R = (c->n_tokens - p0) < r_max ? (c->n_tokens - p0) : r_max;
+    launch_set_pass(c->b.ctl, p0, R, c->batch, vtail, 2 * kv_layer, m->cfg.layers, c->L, m->cfg.d, cs);
+    HeadIO hio{1, c->x, c->b.tmp};                 // no row reaches the head's output
+    af_status s = enqueue_pass(m, c->b, c->batch, c->L, c->dir, m_max, r_max, c->x, hio, cs);
+    if (s) return s;
+  }
+  CK(cudaGetLastError());
+  return AF_OK;
+}
+
+af_status stack_checks(const af_model* const* blocks, const af_dir* dirs, int T, cudaStream_t st) {
   if (!blocks || !dirs || T < 1) { set_err("blocks/dirs/T"); return AF_ERR_ARG; }
   for (int t = 0; t < T; ++t) {
     if (!blocks[t]) { set_err("null block %d", t); return AF_ERR_ARG; }
     if (!same_cfg(blocks[t]->cfg, blocks[0]->cfg)) { set_err("blocks must share one config"); return AF_ERR_ARG; }
     if (dirs[t] != AF_L2R && dirs[t] != AF_R2L) { set_err("bad direction"); return AF_ERR_ARG; }
+    if (blocks[t]->device != blocks[0]->device) { set_err("blocks must live on one device"); return AF_ERR_ARG; }
   }
-  return AF_OK;
+  return device_checks(blocks[0], st);
 }
 
 }  // namespace
@@ -518,15 +623,23 @@ namespace af {
 
 void set_error_text(const char* msg) { set_err("%s", msg); }
 
+// AF_OK when `m` lives on the current device and `st` (if not the default
+// stream) belongs to it; used by entry points outside this file.
+af_status check_call_device(const af_model* m, cudaStream_t st) {
+  if (!m) { set_err("null model"); return AF_ERR_ARG; }
+  return device_checks(m, st);
+}
+
 // The forward pass of one block launched kernel by kernel on `st`, with the
 // workspace at `ws`; used by af_forward_noalloc.
 af_status forward_direct(const af_model* m, const float* x, int batch, int L, af_dir dir, float* z, float* logdet,
                          void* ws, size_t ws_bytes, cudaStream_t st) {
   const af_model* blocks[1] = {m};
   af_dir dirs[1] = {dir};
-  if (af_status s = stack_checks(blocks, dirs, 1)) return s;
+  if (af_status s = stack_checks(blocks, dirs, 1, st)) return s;
   if (af_status s = check_ws(m, ws, ws_bytes, batch, L, L)) return s;
   FwdCtx c{blocks, dirs, 1, batch, L, x, z, logdet, carve(m, ws, batch, L, L)};
+  g_pdl = m->pdl;
   return build_forward(&c, st);
 }
 
@@ -562,14 +675,16 @@ af_status af_model_create(const af_config* cfg, const float* const* tensors, int
   for (int i = 0; i < n_tensors; ++i)
     if (!tensors[i]) { set_err("null tensor %d", i); return AF_ERR_ARG; }
 
-  if (const char* v = getenv("AF_PDL")) g_pdl = atoi(v) != 0;
   af_model* m = new af_model();
+  m->pdl = 1;
+  if (const char* v = getenv("AF_PDL")) m->pdl = atoi(v) != 0;
   m->cfg = c;
   m->fd = c.mlp_ratio * c.d;
   m->hd = hd;
   m->bf = c.dtype == AF_BF16;
   int dev = 0;
   cudaGetDevice(&dev);
+  m->device = dev;
   if (cudaDeviceGetAttribute(&m->num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
     set_err("no CUDA device");
     delete m;
@@ -668,13 +783,15 @@ af_status af_model_destroy(af_model* m) {
   for (void* p : m->allocs) cudaFree(p);
   cudaStreamDestroy(m->cap);
   cudaStreamDestroy(m->cap2);
+  if (m->ev_frame) cudaEventDestroy(m->ev_frame);
+  if (m->ev_done) cudaEventDestroy(m->ev_done);
   delete m;
   return AF_OK;
 }
 
 size_t af_workspace_bytes(const af_model* m, int batch, int L, int B) {
-  if (!m || batch < 1 || L < 1 || B < 1 || L > m->cfg.frame_len * m->cfg.max_frames || L % B) return 0;
-  return carve(m, nullptr, batch, L, B).total;
+  if (!m || batch < 1 || L < 1 || B < 1 || L > m->cfg.frame_len * m->cfg.max_frames) return 0;
+  return carve(m, nullptr, batch, L, B < L ? B : L).total;
 }
 
 af_status af_forward(const af_model* m, const float* x, int batch, int L, af_dir dir, float* z, float* logdet,
@@ -687,7 +804,7 @@ af_status af_forward(const af_model* m, const float* x, int batch, int L, af_dir
 
 af_status flow_stack_forward(const af_model* const* blocks, const af_dir* dirs, int T, const float* x, int batch,
                              int L, float* z, float* logdet, void* ws, size_t ws_bytes, void* stream) {
-  if (af_status s = stack_checks(blocks, dirs, T)) return s;
+  if (af_status s = stack_checks(blocks, dirs, T, (cudaStream_t)stream)) return s;
   if (!x || !z || !logdet || x == z) { set_err("x/z/logdet (x and z must not alias)"); return AF_ERR_ARG; }
   if (af_status s = check_ws(blocks[0], ws, ws_bytes, batch, L, L)) return s;
   FwdCtx c{blocks, dirs, T, batch, L, x, z, logdet, carve(blocks[0], ws, batch, L, L)};
@@ -711,21 +828,139 @@ af_status af_inverse_jacobi(const af_model* m, const float* z, int batch, int L,
 af_status flow_stack_inverse(const af_model* const* blocks, const af_dir* dirs, int T, const float* z, int batch,
                              int L, int B, float tau, int max_iter, int warm_start, float* x, int32_t* iters,
                              void* ws, size_t ws_bytes, void* stream) {
-  if (af_status s = stack_checks(blocks, dirs, T)) return s;
+  if (af_status s = stack_checks(blocks, dirs, T, (cudaStream_t)stream)) return s;
   if (!z || !x || !iters || x == z) { set_err("z/x/iters (x and z must not alias)"); return AF_ERR_ARG; }
   if (B < 1 || L % B || max_iter < 1 || !(tau >= 0.f) || tau == INFINITY) {
     set_err("need L %% B == 0, max_iter >= 1, finite tau >= 0");
     return AF_ERR_ARG;
   }
   if (af_status s = check_ws(blocks[0], ws, ws_bytes, batch, L, B)) return s;
-  InvCtx c{blocks, dirs, T, batch, L, B, max_iter, warm_start ? 1 : 0, tau, z, x, iters,
-           carve(blocks[0], ws, batch, L, B)};
-  uint32_t taubits;
-  memcpy(&taubits, &tau, 4);
-  std::string key = keyf("inv", {(long long)z, (long long)x, (long long)iters, (long long)ws, batch, L, B,
-                                 (long long)taubits, max_iter, c.warm, T});
-  for (int t = 0; t < T; ++t) key += keyf("", {(long long)blocks[t], dirs[t]});
-  return graph_run(blocks[0], key, (cudaStream_t)stream, build_inverse, &c);
+  return run_inverse(blocks, dirs, T, z, batch, L, uniform_schedule(L, B), tau, max_iter, warm_start, x, iters, ws,
+                     (cudaStream_t)stream);
+}
+
+af_status af_inverse_jacobi_schedule(const af_model* m, const float* z, int batch, int L, af_dir dir,
+                                     const int* block_sizes, int n_blocks, int b_begin, int b_end, float tau,
+                                     int max_iter, int warm_start, float* x, int32_t* iters, void* ws,
+                                     size_t ws_bytes, void* stream) {
+  af_dir dirs[1] = {dir};
+  const af_model* blocks[1] = {m};
+  if (af_status s = stack_checks(blocks, dirs, 1, (cudaStream_t)stream)) return s;
+  if (!z || !x || !iters || x == z) { set_err("z/x/iters (x and z must not alias)"); return AF_ERR_ARG; }
+  if (!block_sizes || n_blocks < 1 || n_blocks > L || b_begin < 0 || b_end > n_blocks || b_begin >= b_end) {
+    set_err("need 1 <= n_blocks <= L and 0 <= b_begin < b_end <= n_blocks");
+    return AF_ERR_ARG;
+  }
+  if (max_iter < 1 || !(tau >= 0.f) || tau == INFINITY) { set_err("need max_iter >= 1, finite tau >= 0"); return AF_ERR_ARG; }
+  Schedule sc;
+  sc.starts.push_back(0);
+  sc.B_max = 0;
+  sc.uniform = true;
+  for (int i = 0; i < n_blocks; ++i) {
+    const int bs = block_sizes[i];
+    if (bs < 1 || sc.starts.back() > L - bs) { set_err("block %d: sizes must be >= 1 and sum to L", i); return AF_ERR_ARG; }
+    sc.starts.push_back(sc.starts.back() + bs);
+    if (bs > sc.B_max) sc.B_max = bs;
+    if (bs != block_sizes[0]) sc.uniform = false;
+  }
+  if (sc.starts.back() != L) { set_err("block sizes sum to %d, not L = %d", sc.starts.back(), L); return AF_ERR_ARG; }
+  sc.b_begin = b_begin;
+  sc.b_end = b_end;
+  if (af_status s = check_ws(m, ws, ws_bytes, batch, L, sc.B_max)) return s;
+  return run_inverse(blocks, dirs, 1, z, batch, L, sc, tau, max_iter, warm_start, x, iters, ws, (cudaStream_t)stream);
+}
+
+af_status af_prefix_encode(const af_model* m, const float* x, int batch, int L, af_dir dir, int B, int n_tokens,
+                           void* ws, size_t ws_bytes, void* stream) {
+  af_dir dirs[1] = {dir};
+  const af_model* blocks[1] = {m};
+  if (af_status s = stack_checks(blocks, dirs, 1, (cudaStream_t)stream)) return s;
+  if (!x || n_tokens < 1 || n_tokens > L || B < 1) { set_err("need x, 1 <= n_tokens <= L, B >= 1"); return AF_ERR_ARG; }
+  if (af_status s = check_ws(m, ws, ws_bytes, batch, L, B)) return s;
+  const int Bc = B < L ? B : L;
+  EncCtx c{m, x, batch, L, Bc, n_tokens, dir, carve(m, ws, batch, L, Bc)};
+  g_pdl = m->pdl;
+  std::string key = keyf("enc", {(long long)x, (long long)ws, batch, L, Bc, n_tokens, dir});
+  return graph_run(m, key, (cudaStream_t)stream, build_encode, &c);
+}
+
+size_t flow_pipeline_workspace_bytes(const af_model* shallow, int T, int batch, int frame_len) {
+  if (!shallow || T < 1) return 0;
+  const size_t stack = af_workspace_bytes(shallow, batch, frame_len, frame_len);
+  if (!stack) return 0;
+  const size_t frame = align256((size_t)batch * frame_len * shallow->cfg.C * sizeof(float));
+  return stack + 2 * frame + align256((size_t)T * batch * sizeof(int32_t));
+}
+
+af_status flow_pipeline_inverse(const af_model* deep, const af_model* const* shallow, const af_dir* shallow_dirs, int T,
+                                const float* z, int batch, int L, int B, float tau, int max_iter_deep,
+                                int max_iter_shallow, int warm_start, float* x, int32_t* iters_deep,
+                                int32_t* iters_shallow, void* ws_deep, size_t ws_deep_bytes, void* ws_shallow,
+                                size_t ws_shallow_bytes, void* stream_deep, void* stream_shallow) {
+  cudaStream_t sd = (cudaStream_t)stream_deep, ss = (cudaStream_t)stream_shallow;
+  af_dir ddir[1] = {AF_L2R};
+  const af_model* dblk[1] = {deep};
+  if (af_status s = stack_checks(dblk, ddir, 1, sd)) return s;
+  if (af_status s = stack_checks(shallow, shallow_dirs, T, ss)) return s;
+  if (shallow[0]->device != deep->device) { set_err("deep and shallow models on different devices"); return AF_ERR_ARG; }
+  const int F = deep->cfg.frame_len;
+  const int C = deep->cfg.C;
+  if (shallow[0]->cfg.C != C || shallow[0]->cfg.frame_len * shallow[0]->cfg.max_frames < F) {
+    set_err("the shallow blocks must take frames of %d tokens of %d channels", F, C);
+    return AF_ERR_ARG;
+  }
+  if (!z || !x || !iters_deep || !iters_shallow || x == z) { set_err("z/x/iters (x and z must not alias)"); return AF_ERR_ARG; }
+  if (B < 1 || L % F || F % B || max_iter_deep < 1 || max_iter_shallow < 1 || !(tau >= 0.f) || tau == INFINITY) {
+    set_err("need L %% frame_len == 0, frame_len %% B == 0, max_iter >= 1, finite tau >= 0");
+    return AF_ERR_ARG;
+  }
+  if (af_status s = check_ws(deep, ws_deep, ws_deep_bytes, batch, L, B)) return s;
+  const size_t need_s = flow_pipeline_workspace_bytes(shallow[0], T, batch, F);
+  if (!ws_shallow || (reinterpret_cast<uintptr_t>(ws_shallow) & 255u) || ws_shallow_bytes < need_s) {
+    set_err("shallow workspace: need %zu bytes, 256-aligned; got %zu", need_s, ws_shallow_bytes);
+    return AF_ERR_WORKSPACE;
+  }
+  af_model* dm = const_cast<af_model*>(deep);
+  if (!dm->ev_frame) {
+    CK(cudaEventCreateWithFlags(&dm->ev_frame, cudaEventDisableTiming));
+    CK(cudaEventCreateWithFlags(&dm->ev_done, cudaEventDisableTiming));
+  }
+  // the shallow side's workspace: the stack's own, then the staged frame in / out and counts
+  const size_t stack_bytes = af_workspace_bytes(shallow[0], batch, F, F);
+  const size_t frame = align256((size_t)batch * F * C * sizeof(float));
+  char* wsS = static_cast<char*>(ws_shallow);
+  float* stage_in = (float*)(wsS + stack_bytes);
+  float* stage_out = (float*)(wsS + stack_bytes + frame);
+  int32_t* stage_it = (int32_t*)(wsS + stack_bytes + 2 * frame);
+  // the deep flow's output u (the shallow stack's input) stays in its workspace
+  float* u = carve(deep, ws_deep, batch, L, B).tmp;
+  const int nf = L / F, bpf = F / B;
+  Schedule sc = uniform_schedule(L, B);
+  const size_t row = (size_t)F * C * sizeof(float);
+  for (int f = 0; f < nf; ++f) {
+    // f_D^{-1}: the blocks of frame f (the table once, then only the range)
+    sc.b_begin = f * bpf;
+    sc.b_end = (f + 1) * bpf;
+    if (f > 0) launch_set_range(carve(deep, ws_deep, batch, L, B).btab, sc.b_begin, sc.b_end, sd);
+    if (af_status s = run_inverse(dblk, ddir, 1, z, batch, L, sc, tau, max_iter_deep, warm_start, u, iters_deep,
+                                  ws_deep, sd, f == 0))
+      return s;
+    CK(cudaEventRecord(dm->ev_frame, sd));
+    // f_S^{-1} of frame f on the second stream, while f_D goes on with frame f + 1
+    CK(cudaStreamWaitEvent(ss, dm->ev_frame, 0));
+    CK(cudaMemcpy2DAsync(stage_in, row, u + (size_t)f * F * C, (size_t)L * C * sizeof(float), row, batch,
+                         cudaMemcpyDeviceToDevice, ss));
+    if (af_status s = flow_stack_inverse(shallow, shallow_dirs, T, stage_in, batch, F, F, tau, max_iter_shallow, 0,
+                                         stage_out, stage_it, ws_shallow, stack_bytes, ss))
+      return s;
+    CK(cudaMemcpy2DAsync(x + (size_t)f * F * C, (size_t)L * C * sizeof(float), stage_out, row, row, batch,
+                         cudaMemcpyDeviceToDevice, ss));
+    CK(cudaMemcpy2DAsync(iters_shallow + f, (size_t)nf * sizeof(int32_t), stage_it, sizeof(int32_t), sizeof(int32_t),
+                         (size_t)T * batch, cudaMemcpyDeviceToDevice, ss));
+  }
+  CK(cudaEventRecord(dm->ev_done, ss));
+  CK(cudaStreamWaitEvent(sd, dm->ev_done, 0));
+  return AF_OK;
 }
 
 af_status af_last_convergence(void* ws, int* n_unconverged, void* stream) {

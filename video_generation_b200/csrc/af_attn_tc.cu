@@ -184,11 +184,41 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 
 struct AttnArgs {
   const Ctl* ctl;
-  bf16* o;           // [Mmax, d] output (nsplit == 1)
-  float* opart;      // [nsplit, Mmax, d] unnormalised partial outputs (nsplit > 1)
-  float* mlpart;     // [nsplit, Mmax, heads, 2] running max (log2 units) and row sum
-  int Lc, d, heads, nsplit, tiles_per_split, m_max, batch;
+  bf16* o;           // [Mmax, d] output (one split)
+  float* opart;      // [nsplit_max, Mmax, d] unnormalised partial outputs (several splits)
+  float* mlpart;     // [nsplit_max, Mmax, heads, 2] running max (log2 units) and row sum
+  int Lc, d, heads, nsplit_max, m_max, batch, sms;
 };
+
+// Key splits of a pass, decided from the rows the pass really has (ctl->R
+// query rows per sample at positions p0 ..) rather than from the cache's
+// length: a pass whose (query tile, head, sample) items already fill the GPU
+// twice over runs unsplit; otherwise the live key range (keys 0 .. p0 + R - 1)
+// is cut into up to nsplit_max splits of at least kMinSplitTiles 64-key tiles,
+// aiming at about 4 items per SM.  The attention kernel and the combine kernel
+// evaluate this from the same control block, so they agree.
+constexpr int kMinSplitTiles = 8;
+constexpr int kMaxSplits = 32;
+constexpr int kMaxDevices = 64;
+struct SplitPlan { int q_tiles, nsplit, tps; };
+__host__ __device__ __forceinline__ SplitPlan split_plan(int R, int p0, int heads, int batch, int nsplit_max,
+                                                         int sms, int bkv) {
+  SplitPlan sp;
+  sp.q_tiles = (R + BQ - 1) / BQ;
+  const int live = (p0 + R + bkv - 1) / bkv;               // key tiles up to the last key any row needs
+  const int base = sp.q_tiles * heads * batch;
+  int n = 1;
+  if (nsplit_max > 1 && base < 2 * sms) {
+    const int want = (4 * sms + base - 1) / base;
+    const int by_len = (live + kMinSplitTiles - 1) / kMinSplitTiles;
+    n = want < by_len ? want : by_len;
+    if (n > nsplit_max) n = nsplit_max;
+    if (n < 1) n = 1;
+  }
+  sp.tps = (live + n - 1) / n;
+  sp.nsplit = (live + sp.tps - 1) / sp.tps;
+  return sp;
+}
 
 template <int HD>
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -244,8 +274,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   pdl_wait();                                                 // q, the cache and the row layout come from upstream
   const Ctl* ctl = g.ctl;
   const int R = ctl->R, p0 = ctl->p0;
-  const int q_tiles = (R + BQ - 1) / BQ;
-  const int n_items = q_tiles * g.heads * g.batch * g.nsplit;
+  const SplitPlan plan = split_plan(R, p0, g.heads, g.batch, g.nsplit_max, g.sms, BKV);
+  const int q_tiles = plan.q_tiles, nsplit = plan.nsplit, tps = plan.tps;
+  const int n_items = q_tiles * g.heads * g.batch * nsplit;
 
   // Work item -> (query tile, head, sample, key split) and its key-tile range.
   // Query tiles end at R, R - 128, ...: the ragged tile is the first one, whose
@@ -253,7 +284,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   // query tile varies slowest and the last (causally heaviest) tiles come
   // first, so CTAs taking items round-robin get a balanced mix of work.
   struct Item { int qt, hh, s, split, q_begin, t0, nt; };
-  const int per_qt = g.heads * g.batch * g.nsplit;
+  const int per_qt = g.heads * g.batch * nsplit;
   const int pad = q_tiles * BQ - R;
   auto item_of = [&](int it) {
     Item x;
@@ -261,13 +292,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     int r = it % per_qt;
     x.hh = r % g.heads;
     r /= g.heads;
-    x.split = r % g.nsplit;
-    x.s = r / g.nsplit;
+    x.split = r % nsplit;
+    x.s = r / nsplit;
     x.q_begin = x.qt * BQ - pad;
     const int q_end = x.q_begin + BQ;
     const int ntiles = (p0 + q_end - 1) / BKV + 1;          // key tiles up to the last needed key
-    x.t0 = x.split * g.tiles_per_split;
-    x.nt = min(ntiles, x.t0 + g.tiles_per_split) - x.t0;
+    x.t0 = x.split * tps;
+    x.nt = min(ntiles, x.t0 + tps) - x.t0;
     return x;
   };
   // The CTA's k-th item (k = 0, 1, ...) is global item blockIdx.x + k * gridDim.x
@@ -576,7 +607,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // (bf16, 32-byte swizzle, 16 columns per 1 KB) in its quarter of a free P
       // tile and writes them with TMA bulk stores; other rows are stored directly
       const int q0 = x.q_begin + quarter * 32;
-      const bool tma_out = HD == 64 && g.nsplit == 1 && ok && q0 >= 0 && q0 + 31 < R;   // warp-uniform
+      const bool tma_out = HD == 64 && nsplit == 1 && ok && q0 >= 0 && q0 + 31 < R;   // warp-uniform
       const int sb = (tw + 1) % PB;                          // the P tile written last by the next item
       uint8_t* stg = sP + sb * Cfg::P_BYTES + q * 4096;
       if (tma_out && stg_buf >= 0) {
@@ -613,7 +644,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           continue;
         }
         if (!valid) continue;
-        if (g.nsplit == 1) {
+        if (nsplit == 1) {
           uint4* dst = reinterpret_cast<uint4*>(g.o + mrow * g.d + xe.hh * HD + h0);
 #pragma unroll
           for (int c = 0; c < 32; c += 8)
@@ -637,7 +668,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         stg_buf = sb;
       }
-      if (valid && g.nsplit > 1) {
+      if (valid && nsplit > 1) {
         float* ml = g.mlpart + (((size_t)xe.split * g.m_max + mrow) * g.heads + xe.hh) * 2;
         ml[0] = m_use;
         ml[1] = lt;
@@ -663,16 +694,17 @@ __global__ void __launch_bounds__(256) k_attn_combine(AttnArgs g) {
   pdl_wait();
   const int wg = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int M = g.ctl->M;
-  if (wg >= M * g.heads) return;
+  const int nsplit = split_plan(g.ctl->R, g.ctl->p0, g.heads, g.batch, g.nsplit_max, g.sms, AttnCfg<HD>::BKV).nsplit;
+  if (nsplit == 1 || wg >= M * g.heads) return;      // one split: the attention kernel wrote o itself
   const int row = wg / g.heads, hh = wg - row * g.heads;
   float mx = -INFINITY;
-  for (int i = 0; i < g.nsplit; ++i) mx = fmaxf(mx, g.mlpart[(((size_t)i * g.m_max + row) * g.heads + hh) * 2]);
+  for (int i = 0; i < nsplit; ++i) mx = fmaxf(mx, g.mlpart[(((size_t)i * g.m_max + row) * g.heads + hh) * 2]);
   constexpr int PER = HD / 32;
   float acc[PER];
 #pragma unroll
   for (int k = 0; k < PER; ++k) acc[k] = 0.f;
   float lsum = 0.f;
-  for (int i = 0; i < g.nsplit; ++i) {
+  for (int i = 0; i < nsplit; ++i) {
     const float* ml = g.mlpart + (((size_t)i * g.m_max + row) * g.heads + hh) * 2;
     if (ml[0] == -INFINITY) continue;
     const float w = exp2f(ml[0] - mx);
@@ -688,24 +720,22 @@ __global__ void __launch_bounds__(256) k_attn_combine(AttnArgs g) {
 
 template <int HD>
 bool launch_hd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
-               const AttnArgs& g, int batch,
-               int r_max, int* err, cudaStream_t st) {
+               const AttnArgs& g, int batch, int r_max, int* err, cudaStream_t st) {
   using Cfg = AttnCfg<HD>;
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_attn_tc<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM);
-    attr = true;
+  // the shared-memory opt-in is a per-device setting of the function
+  static bool attr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  if (!attr[dev]) {
+    if (cudaFuncSetAttribute(k_attn_tc<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM) != cudaSuccess)
+      return false;
+    attr[dev] = true;
   }
-  static int sms = 0;
-  if (!sms) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  }
-  const long long items = (long long)((r_max + BQ - 1) / BQ) * g.heads * batch * g.nsplit;
-  const int grid = (int)(items < sms ? items : sms);
+  // an upper bound of the items of any pass with at most r_max rows per sample
+  const long long items = (long long)((r_max + BQ - 1) / BQ) * g.heads * batch * g.nsplit_max;
+  const int grid = (int)(items < g.sms ? items : g.sms);
   launch_k(k_attn_tc<HD>, dim3(grid), dim3(kAttnThreads), Cfg::SMEM, st, tq, tk, tv, to, g, err);
-  if (g.nsplit > 1) {
+  if (g.nsplit_max > 1) {
     const long long warps = (long long)g.m_max * g.heads;
     launch_k(k_attn_combine<HD>, dim3((unsigned)((warps * 32 + 255) / 256)), dim3(256), 0, st, g);
   }
@@ -715,19 +745,21 @@ bool launch_hd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
 }  // namespace
 
 int attn_tc_splits(int batch, int heads, int r_max, int Lc, int num_sms) {
-  const int q_tiles = (r_max + BQ - 1) / BQ;
-  const long long ctas = (long long)q_tiles * heads * batch;
-  if (ctas >= 2LL * num_sms) return 1;
-  const int key_tiles = (Lc + 127) / 128;                   // in 128-key units
-  int n = (key_tiles + 15) / 16;
-  if (n < 1) n = 1;
-  if (n > 64) n = 64;
-  return n;
+  (void)r_max;
+  const int bkv = 64;
+  const int base_min = heads * batch;                       // a pass with a single query tile
+  if (base_min >= 2 * num_sms) return 1;
+  const int want = (4 * num_sms + base_min - 1) / base_min;
+  const int key_tiles = (Lc + bkv - 1) / bkv;
+  const int by_len = (key_tiles + kMinSplitTiles - 1) / kMinSplitTiles;
+  int n = want < by_len ? want : by_len;
+  if (n > kMaxSplits) n = kMaxSplits;
+  return n < 1 ? 1 : n;
 }
 
 bool launch_attn_tc2(const Ctl* ctl, const bf16* q, const bf16* kc, const bf16* vc, bf16* o, float* opart,
-                     float* mlpart, int nsplit, int batch, int Lc, int d, int heads, int r_max, int m_max, int* err,
-                     cudaStream_t st) {
+                     float* mlpart, int nsplit_max, int batch, int Lc, int d, int heads, int r_max, int m_max,
+                     int num_sms, int* err, cudaStream_t st) {
   const int hd = d / heads;
   const int bkv = hd == 64 ? AttnCfg<64>::BKV : AttnCfg<128>::BKV;
   CUtensorMap tq, tk, tv, to;
@@ -742,11 +774,10 @@ bool launch_attn_tc2(const Ctl* ctl, const bf16* q, const bf16* kc, const bf16* 
   g.Lc = Lc;
   g.d = d;
   g.heads = heads;
-  g.nsplit = nsplit;
-  const int key_tiles = (Lc + bkv - 1) / bkv;
-  g.tiles_per_split = (key_tiles + nsplit - 1) / nsplit;
+  g.nsplit_max = nsplit_max;
   g.m_max = m_max;
   g.batch = batch;
+  g.sms = num_sms;
   return hd == 64 ? launch_hd<64>(tq, tk, tv, to, g, batch, r_max, err, st)
                   : launch_hd<128>(tq, tk, tv, to, g, batch, r_max, err, st);
 }

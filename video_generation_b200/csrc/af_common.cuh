@@ -3,12 +3,12 @@
 // Row convention.  One "pass" of an AF block runs its Transformer over a set
 // of rows.  Row r belongs to sample s = r / R and sits at sequence position
 // p = p0 + r % R of the working order (the order after the direction flip).
-// The forward pass uses p0 = 0, R = L.  A Jacobi iteration of block b uses
-// p0 = P = b*B, R = B, except its first iteration for b > 0, which also
-// carries block b-1 (p0 = P - B, R = 2B) so that block b-1's K/V are
-// recomputed from its final x and written to the cache in the same pass
-// (the KV-cache commit of "STARFlow-V ... paper notes", key design 3).
-// Rows at p < P produce no (mu, s) output.
+// The forward pass uses p0 = 0, R = L.  A Jacobi iteration of block b
+// (positions P .. P+B-1) uses p0 = P, R = B, except its first iteration for
+// b > 0, which also carries block b-1 (p0 = its first position, R = both
+// blocks' tokens) so that block b-1's K/V are recomputed from its final x and
+// written to the cache in the same pass (the KV-cache commit of "STARFlow-V
+// ... paper notes", key design 3).  Rows at p < P produce no (mu, s) output.
 #pragma once
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -29,7 +29,19 @@ struct Ctl {
   int n_active;   // samples still iterating in this block
   int nonconv;    // (sample, block) pairs that stopped at max_iter unconverged
   int done;       // CTAs of the current Jacobi step that finished their sample
+  int B;          // tokens of the current Jacobi block
 };
+
+// Block table of a Jacobi call (in the workspace, written before the call's
+// graph runs): the schedule of block sizes as start positions, and the range
+// of blocks the call inverts.  Blocks need not be equal ("STARFlow-V ...
+// paper notes", key findings: a smaller block for the first frame, larger
+// ones later).
+enum : int { BT_NB = 0, BT_BEGIN = 1, BT_END = 2, BT_STARTS = 4 };
+// btab[BT_NB] = number of blocks nb, btab[BT_BEGIN] / btab[BT_END] = the range
+// [begin, end) of blocks this call inverts, btab[BT_STARTS + i] = first
+// position of block i (i = 0 .. nb; the last entry is L).
+__host__ __device__ inline size_t btab_ints(int L) { return (size_t)BT_STARTS + (size_t)L + 1; }
 
 // Error codes written to the model's device error word.
 enum : int { ERR_NONE = 0, ERR_GEMM_WAIT = 1, ERR_GEMM_DRAIN = 2, ERR_ATTN_WAIT = 3 };

@@ -47,6 +47,7 @@ template <int EPI> struct EpiShape {
   static constexpr uint32_t SLOT = EPI == EPI_RESID ? 32 * 16 * 4 : 32 * 16 * 2;
 };
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr int kMaxDevices = 64;
 
 template <int BN, int CG, int EPI> struct TcCfg {
   // CG = CTAs per MMA: 1, or 2 for the SM-pair MMA (tile of 256 rows, each CTA
@@ -699,7 +700,11 @@ void launch_bn_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtenso
                    const CUtensorMap& tmC3, int N, int K, int m_max, const EpiArgs& e,
                    int* err, int num_sms, cudaStream_t st) {
   using Cfg = TcCfg<BN, CG, EPI>;
-  static int max_units = 0;
+  // the shared-memory opt-in and the co-resident cluster count are per device
+  static int units_of_dev[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return;
+  int& max_units = units_of_dev[dev];
   if (!max_units) {
     cudaFuncSetAttribute(k_gemm_tc<BN, EPI, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM);
     max_units = num_sms / CG;

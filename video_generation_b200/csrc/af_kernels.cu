@@ -55,27 +55,82 @@ int grid_for(long long work, int per_block) {
 __global__ void k_ctl_forward(Ctl* ctl, int batch, int L) {
   pdl_trigger();
   pdl_wait();
-  ctl->P = 0; ctl->p0 = 0; ctl->R = L; ctl->M = batch * L;
+  ctl->P = 0; ctl->p0 = 0; ctl->R = L; ctl->M = batch * L; ctl->B = L;
   ctl->block = 0; ctl->iter = 0; ctl->n_active = 0;
 }
 
-__global__ void k_call_init(Ctl* ctl, int reset_nonconv) {
+// Block table of a call (af_common.cuh): written in chunks of kTabChunk
+// entries from kernel arguments, so that writing it needs no host memory
+// copy and can be captured.
+struct TabChunk { int v[kTabChunk]; };
+__global__ void k_table_write(int* btab, int first, int n, TabChunk ch, int nb, int b_begin, int b_end) {
   pdl_trigger();
   pdl_wait();
-  ctl->block = 0;
-  if (reset_nonconv) ctl->nonconv = 0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) btab[BT_STARTS + first + i] = ch.v[i];
+  if (threadIdx.x == 0 && first == 0) {
+    btab[BT_NB] = nb;
+    btab[BT_BEGIN] = b_begin;
+    btab[BT_END] = b_end;
+  }
 }
 
-// Start of Jacobi block b = ctl->block: the row layout of the first update
-// (block b-1 rides along to commit its K/V), fresh per-sample flags, and the
-// starting guess x^(0) = z_b, or block b-1's final x when warm starting.
-__global__ void k_block_init(Ctl* ctl, int* active, const float* __restrict__ z, float* x, int batch,
-                             int L, int C, int B, int dir, int warm,
-                             cudaGraphConditionalHandle inner) {
+__global__ void k_set_range(int* btab, int b_begin, int b_end) {
+  pdl_trigger();
+  pdl_wait();
+  btab[BT_BEGIN] = b_begin;
+  btab[BT_END] = b_end;
+}
+
+// Start of a call's block loop.  The count of unconverged (sample, block)
+// pairs restarts with a call whose range starts at block 0 and accumulates
+// over calls that continue a sequence.
+__global__ void k_call_init(Ctl* ctl, const int* btab, int reset_nonconv) {
+  pdl_trigger();
+  pdl_wait();
+  ctl->block = btab[BT_BEGIN];
+  if (reset_nonconv && btab[BT_BEGIN] == 0) ctl->nonconv = 0;
+}
+
+// Zero the V rows r0 .. (end of the 64-key tile holding r0 - 1) of every layer
+// and sample (bf16 cache): the tensor-core attention reads whole key tiles,
+// and although the causal mask gives keys not yet written probability 0,
+// 0 * V must be finite.  `vtail` is layer 0's V cache, layer l's is kv_stride
+// bytes further; positions are per sample (Lc of them).
+__device__ void zero_vtail(bf16* vtail, size_t kv_stride, int layers, int batch, int Lc, int d, int r0) {
+  const int r1 = min(((r0 + 63) >> 6) << 6, Lc);
+  if (r1 <= r0) return;
+  const int dv = d >> 3;                                   // 16-byte units per row
+  const long long nz = (long long)layers * batch * (r1 - r0) * dv;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < nz;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int u = (int)(i % dv);
+    long long rest = i / dv;
+    const int r = r0 + (int)(rest % (r1 - r0));
+    rest /= (r1 - r0);
+    const int s = (int)(rest % batch);
+    const int l = (int)(rest / batch);
+    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<char*>(vtail) + (size_t)l * kv_stride +
+                                          (((size_t)s * Lc + r) * d) * sizeof(bf16)) + u;
+    *dst = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// Start of Jacobi block b = ctl->block (positions P .. Q-1 of the table):
+// the row layout of the first update (block b-1 rides along to commit its
+// K/V), fresh per-sample flags, and the starting guess: z, or with warm start
+// the previous frame's converged state ("STARFlow-V ... paper notes", key
+// design 3) -- position p takes the converged x of p - k*F, the same spatial
+// position in the most recent finished frame (smallest k >= 1 with
+// p - k*F < P), or z where no frame before it has finished.  With a bf16
+// cache (vtail != null) it also zeroes the masked V tail (zero_vtail) past Q.
+__global__ void k_block_init(Ctl* ctl, const int* btab, int* active, const float* __restrict__ z, float* x,
+                             int batch, int L, int C, int F, int dir, int warm, bf16* vtail, size_t kv_stride,
+                             int layers, int d, cudaGraphConditionalHandle inner) {
   pdl_trigger();
   pdl_wait();
   const int b = ctl->block;
-  const int P = b * B;
+  const int P = btab[BT_STARTS + b], Q = btab[BT_STARTS + b + 1];
+  const int B = Q - P;
   const int nvec = C >> 2;
   const long long n = (long long)batch * B * nvec;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
@@ -84,22 +139,26 @@ __global__ void k_block_init(Ctl* ctl, int* active, const float* __restrict__ z,
     const long long st = i / nvec;
     const int t = (int)(st % B);
     const int s = (int)(st / B);
-    const size_t dst = ((size_t)s * L + tok_of(P + t, L, dir)) * C + cv * 4;
+    const int p = P + t;
+    const size_t dst = ((size_t)s * L + tok_of(p, L, dir)) * C + cv * 4;
+    const int src = p - (t / F + 1) * F;
     float4 v;
-    if (warm && b > 0)
-      v = *reinterpret_cast<const float4*>(x + ((size_t)s * L + tok_of(P - B + t, L, dir)) * C + cv * 4);
+    if (warm && src >= 0)
+      v = *reinterpret_cast<const float4*>(x + ((size_t)s * L + tok_of(src, L, dir)) * C + cv * 4);
     else
       v = *reinterpret_cast<const float4*>(z + dst);
     *reinterpret_cast<float4*>(x + dst) = v;
   }
+  if (vtail) zero_vtail(vtail, kv_stride, layers, batch, L, d, Q);
   if (blockIdx.x == 0) {
     for (int s = threadIdx.x; s < batch; s += blockDim.x) active[s] = 1;
     if (threadIdx.x == 0) {
-      const int p0 = b > 0 ? P - B : P;
+      const int p0 = b > 0 ? btab[BT_STARTS + b - 1] : P;
       ctl->P = P;
+      ctl->B = B;
       ctl->p0 = p0;
-      ctl->R = P + B - p0;
-      ctl->M = batch * (P + B - p0);
+      ctl->R = Q - p0;
+      ctl->M = batch * (Q - p0);
       ctl->iter = 0;
       ctl->n_active = batch;
       ctl->done = 0;
@@ -111,15 +170,16 @@ __global__ void k_block_init(Ctl* ctl, int* active, const float* __restrict__ z,
 // End of one Jacobi update: per-sample residual from the head's partial sums
 // (one CTA per sample, fixed summation order), the stopping test, the
 // iteration counters; the last CTA to finish sets the inner loop condition.
-__global__ void __launch_bounds__(512) k_jacobi_step(Ctl* ctl, int* active, const float* __restrict__ part,
-                                                     int batch, int B, int G, float tau, int max_iter,
-                                                     int32_t* iters, int nblocks,
+__global__ void __launch_bounds__(512) k_jacobi_step(Ctl* ctl, const int* btab, int* active,
+                                                     const float* __restrict__ part, int batch, int G, float tau,
+                                                     int max_iter, int32_t* iters,
                                                      cudaGraphConditionalHandle inner) {
   pdl_trigger();
   pdl_wait();
   __shared__ int s_last;
   const int s = blockIdx.x;
-  const int R = ctl->R, p0 = ctl->p0, P = ctl->P, iter = ctl->iter, blk = ctl->block;
+  const int R = ctl->R, p0 = ctl->p0, P = ctl->P, B = ctl->B, iter = ctl->iter, blk = ctl->block;
+  const int nblocks = btab[BT_NB];
   if (active[s]) {                                     // uniform over the CTA
     const float2* p = reinterpret_cast<const float2*>(part + ((size_t)s * R + (P - p0)) * G * 2);
     const int n = B * G;
@@ -158,12 +218,29 @@ __global__ void __launch_bounds__(512) k_jacobi_step(Ctl* ctl, int* active, cons
   }
 }
 
-__global__ void k_block_advance(Ctl* ctl, int nblocks, cudaGraphConditionalHandle outer) {
+__global__ void k_block_advance(Ctl* ctl, const int* btab, cudaGraphConditionalHandle outer) {
   pdl_trigger();
   pdl_wait();
   const int b = ctl->block + 1;
   ctl->block = b;
-  cudaGraphSetConditional(outer, b < nblocks ? 1u : 0u);
+  cudaGraphSetConditional(outer, b < btab[BT_END] ? 1u : 0u);
+}
+
+// A pass over positions p0 .. p0+R-1 of every sample whose rows give no head
+// output (P = p0 + R): the flow-encode of observed tokens into the KV cache.
+// Zeroes the masked V tail past the pass, like a block init.
+__global__ void k_set_pass(Ctl* ctl, int p0, int R, int batch, bf16* vtail, size_t kv_stride, int layers, int Lc,
+                           int d) {
+  pdl_trigger();
+  pdl_wait();
+  if (vtail) zero_vtail(vtail, kv_stride, layers, batch, Lc, d, p0 + R);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    ctl->P = p0 + R;
+    ctl->p0 = p0;
+    ctl->R = R;
+    ctl->M = batch * R;
+    ctl->B = R;
+  }
 }
 
 // ------------------------------------------------------------------ row-wise
@@ -393,8 +470,28 @@ __global__ void __launch_bounds__(256) k_attn_simt(const Ctl* ctl, const float* 
 void launch_ctl_forward(Ctl* ctl, int batch, int L, cudaStream_t st) {
   launch_k(k_ctl_forward, dim3(1), dim3(1), 0, st, ctl, batch, L);
 }
-void launch_call_init(Ctl* ctl, int reset_nonconv, cudaStream_t st) {
-  launch_k(k_call_init, dim3(1), dim3(1), 0, st, ctl, reset_nonconv);
+void launch_call_init(Ctl* ctl, const int* btab, int reset_nonconv, cudaStream_t st) {
+  launch_k(k_call_init, dim3(1), dim3(1), 0, st, ctl, btab, reset_nonconv);
+}
+
+void launch_table_write(int* btab, const int* starts, int nb, int b_begin, int b_end, cudaStream_t st) {
+  for (int first = 0; first <= nb; first += kTabChunk) {
+    TabChunk ch;
+    const int n = (nb + 1 - first) < kTabChunk ? (nb + 1 - first) : kTabChunk;
+    for (int i = 0; i < n; ++i) ch.v[i] = starts[first + i];
+    launch_k(k_table_write, dim3(1), dim3(256), 0, st, btab, first, n, ch, nb, b_begin, b_end);
+  }
+}
+
+void launch_set_range(int* btab, int b_begin, int b_end, cudaStream_t st) {
+  launch_k(k_set_range, dim3(1), dim3(1), 0, st, btab, b_begin, b_end);
+}
+
+void launch_set_pass(Ctl* ctl, int p0, int R, int batch, bf16* vtail, size_t kv_stride, int layers, int Lc, int d,
+                     cudaStream_t st) {
+  const long long work = vtail ? (long long)layers * batch * 64 * (d / 8) : 1;
+  launch_k(k_set_pass, dim3(grid_for(work, kThreads)), dim3(kThreads), 0, st, ctl, p0, R, batch, vtail, kv_stride,
+           layers, Lc, d);
 }
 
 template <typename T>
@@ -426,20 +523,22 @@ void launch_logdet_finalize(const float* part, int batch, int L, int G, float* l
   launch_k(k_logdet_finalize, dim3(batch), dim3(512), 0, st, part, L, G, logdet, accumulate);
 }
 
-void launch_block_init(Ctl* ctl, int* active, const float* z, float* x, int batch, int L, int C, int B,
-                       int dir, int warm, cudaGraphConditionalHandle inner, cudaStream_t st) {
-  launch_k(k_block_init, dim3(grid_for((long long)batch * B * (C / 4), kThreads)), dim3(kThreads), 0, st, 
-      ctl, active, z, x, batch, L, C, B, dir, warm, inner);
+void launch_block_init(Ctl* ctl, const int* btab, int* active, const float* z, float* x, int batch, int L, int C,
+                       int B_max, int F, int dir, int warm, bf16* vtail, size_t kv_stride, int layers, int d,
+                       cudaGraphConditionalHandle inner, cudaStream_t st) {
+  const long long work = (long long)batch * B_max * (C / 4) + (vtail ? (long long)layers * batch * 64 * (d / 8) : 0);
+  launch_k(k_block_init, dim3(grid_for(work, kThreads)), dim3(kThreads), 0, st, ctl, btab, active, z, x, batch, L,
+           C, F, dir, warm, vtail, kv_stride, layers, d, inner);
 }
 
-void launch_jacobi_step(Ctl* ctl, int* active, const float* part, int batch, int B, int G, float tau,
-                        int max_iter, int32_t* iters, int nblocks, cudaGraphConditionalHandle inner,
-                        cudaStream_t st) {
-  launch_k(k_jacobi_step, dim3(batch), dim3(512), 0, st, ctl, active, part, batch, B, G, tau, max_iter, iters, nblocks, inner);
+void launch_jacobi_step(Ctl* ctl, const int* btab, int* active, const float* part, int batch, int G, float tau,
+                        int max_iter, int32_t* iters, cudaGraphConditionalHandle inner, cudaStream_t st) {
+  launch_k(k_jacobi_step, dim3(batch), dim3(512), 0, st, ctl, btab, active, part, batch, G, tau, max_iter, iters,
+           inner);
 }
 
-void launch_block_advance(Ctl* ctl, int nblocks, cudaGraphConditionalHandle outer, cudaStream_t st) {
-  launch_k(k_block_advance, dim3(1), dim3(1), 0, st, ctl, nblocks, outer);
+void launch_block_advance(Ctl* ctl, const int* btab, cudaGraphConditionalHandle outer, cudaStream_t st) {
+  launch_k(k_block_advance, dim3(1), dim3(1), 0, st, ctl, btab, outer);
 }
 
 void launch_gemm_simt(int epi, const float* A, const float* W, int N, int K, int m_max, const EpiArgs& e,

@@ -7,10 +7,13 @@
 
 namespace af {
 
-// Launches with programmatic stream serialization when g_pdl is set (the
-// default; AF_PDL=0 in the environment turns it off), so that a kernel's
-// launch and set-up overlap the tail of the kernel before it.
-extern int g_pdl;
+// Launches with programmatic stream serialization when g_pdl is set, so that
+// a kernel's launch and set-up overlap the tail of the kernel before it.  The
+// calling thread sets it from its model before enqueueing (each model keeps
+// its own setting: on by default, AF_PDL=0 in the environment turns it off,
+// and a model whose capture refused programmatic edges turns it off for
+// itself).
+extern thread_local int g_pdl;
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                             Args&&... args) {
@@ -39,15 +42,25 @@ void launch_layernorm(const Ctl* ctl, const float* h, const float* g, const floa
                       int d, int m_max, cudaStream_t st);
 void launch_logdet_finalize(const float* part, int batch, int L, int G, float* logdet,
                             int accumulate, cudaStream_t st);
-void launch_call_init(Ctl* ctl, int reset_nonconv, cudaStream_t st);
-void launch_block_init(Ctl* ctl, int* active, const float* z, float* x, int batch, int L, int C,
-                       int B, int dir, int warm, cudaGraphConditionalHandle inner,
-                       cudaStream_t st);
-void launch_jacobi_step(Ctl* ctl, int* active, const float* part, int batch, int B, int G,
-                        float tau, int max_iter, int32_t* iters, int nblocks,
-                        cudaGraphConditionalHandle inner, cudaStream_t st);
-void launch_block_advance(Ctl* ctl, int nblocks, cudaGraphConditionalHandle outer,
-                          cudaStream_t st);
+// Jacobi driver (af_kernels.cu).  The block table (af_common.cuh) is written
+// from kernel arguments in chunks of kTabChunk start positions.
+constexpr int kTabChunk = 1000;
+void launch_table_write(int* btab, const int* starts, int nb, int b_begin, int b_end, cudaStream_t st);
+void launch_set_range(int* btab, int b_begin, int b_end, cudaStream_t st);
+void launch_call_init(Ctl* ctl, const int* btab, int reset_nonconv, cudaStream_t st);
+// vtail: layer 0's V cache (bf16 path) whose masked tail rows the block's
+// attention reads, layer l's at kv_stride bytes further; null for fp32.
+// B_max: the largest block of the table (sizes the grid); F: frame length.
+void launch_block_init(Ctl* ctl, const int* btab, int* active, const float* z, float* x, int batch, int L, int C,
+                       int B_max, int F, int dir, int warm, bf16* vtail, size_t kv_stride, int layers, int d,
+                       cudaGraphConditionalHandle inner, cudaStream_t st);
+void launch_jacobi_step(Ctl* ctl, const int* btab, int* active, const float* part, int batch, int G, float tau,
+                        int max_iter, int32_t* iters, cudaGraphConditionalHandle inner, cudaStream_t st);
+void launch_block_advance(Ctl* ctl, const int* btab, cudaGraphConditionalHandle outer, cudaStream_t st);
+// Row layout of a pass over positions p0 .. p0+R-1 with no head output
+// (flow-encode into the cache), zeroing the masked V tail past it.
+void launch_set_pass(Ctl* ctl, int p0, int R, int batch, bf16* vtail, size_t kv_stride, int layers, int Lc, int d,
+                     cudaStream_t st);
 
 // ---- fp32 SIMT path (af_kernels.cu) -----------------------------------------
 void launch_gemm_simt(int epi, const float* A, const float* W, int N, int K, int m_max,
@@ -74,13 +87,14 @@ void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, con
                     const EpiArgs& e, int* err, int num_sms, cudaStream_t st);
 int gemm_tc_pick(int N, int m_max, int num_sms, int unit, int max_bn);
 
-// Causal attention over the KV cache on tcgen05 (af_attn_tc.cu).  nsplit key
-// splits (attn_tc_splits); with nsplit > 1, opart [nsplit, m_max, d] and
-// mlpart [nsplit, m_max, heads, 2] hold the partials.  False if a tensor map
-// cannot be encoded.
+// Causal attention over the KV cache on tcgen05 (af_attn_tc.cu).  Each pass
+// splits its live key range into at most nsplit_max splits (attn_tc_splits
+// gives the most a call on a cache of Lc positions can use); with
+// nsplit_max > 1, opart [nsplit_max, m_max, d] and mlpart [nsplit_max, m_max,
+// heads, 2] hold the partials.  False if a tensor map cannot be encoded.
 int attn_tc_splits(int batch, int heads, int r_max, int Lc, int num_sms);
 bool launch_attn_tc2(const Ctl* ctl, const bf16* q, const bf16* kc, const bf16* vc, bf16* o, float* opart,
-                     float* mlpart, int nsplit, int batch, int Lc, int d, int heads, int r_max, int m_max, int* err,
-                     cudaStream_t st);
+                     float* mlpart, int nsplit_max, int batch, int Lc, int d, int heads, int r_max, int m_max,
+                     int num_sms, int* err, cudaStream_t st);
 
 }  // namespace af

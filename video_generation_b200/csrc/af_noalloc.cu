@@ -28,6 +28,7 @@
 namespace af {
 af_status forward_direct(const af_model* m, const float* x, int batch, int L, af_dir dir, float* z,
                          float* logdet, void* ws, size_t ws_bytes, cudaStream_t st);
+af_status check_call_device(const af_model* m, cudaStream_t st);
 void set_error_text(const char* msg);
 }  // namespace af
 
@@ -62,6 +63,9 @@ extern "C" af_status af_forward_noalloc(const af_model* m, const float* x, int b
     af::set_error_text(msg);
     return AF_ERR_WORKSPACE;
   }
+  // the scratch used is the current device's: the model's weights and the
+  // stream must be on that device too
+  if (af_status s = af::check_call_device(m, (cudaStream_t)stream)) return s;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     af::set_error_text("af_forward_noalloc: no usable current CUDA device");

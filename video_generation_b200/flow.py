@@ -26,7 +26,9 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libaf.so")
 
 EXPORTS = ("af_num_tensors", "af_model_create", "af_model_destroy", "af_workspace_bytes", "af_forward",
            "af_inverse_jacobi", "flow_stack_forward", "flow_stack_inverse", "af_last_convergence",
-           "af_device_error", "af_status_string", "af_last_error_string", "af_forward_noalloc")
+           "af_device_error", "af_status_string", "af_last_error_string", "af_forward_noalloc",
+           "af_inverse_jacobi_schedule", "af_prefix_encode", "flow_pipeline_workspace_bytes",
+           "flow_pipeline_inverse")
 
 
 class AFConfigC(ctypes.Structure):
@@ -52,6 +54,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.flow_stack_forward.argtypes = [P(vp), P(i), i, vp, i, i, vp, vp, vp, sz, vp]
     lib.flow_stack_inverse.argtypes = [P(vp), P(i), i, vp, i, i, i, f, i, i, vp, vp, vp, sz, vp]
     lib.af_forward_noalloc.argtypes = [vp, vp, i, i, i, vp, vp, vp]
+    lib.af_inverse_jacobi_schedule.argtypes = [vp, vp, i, i, i, P(i), i, i, i, f, i, i, vp, vp, vp, sz, vp]
+    lib.af_prefix_encode.argtypes = [vp, vp, i, i, i, i, i, vp, sz, vp]
+    lib.flow_pipeline_workspace_bytes.argtypes = [vp, i, i, i]
+    lib.flow_pipeline_workspace_bytes.restype = sz
+    lib.flow_pipeline_inverse.argtypes = [vp, P(vp), P(i), i, vp, i, i, i, f, i, i, i, vp, vp, vp, vp, sz, vp, sz,
+                                          vp, vp]
     lib.af_last_convergence.argtypes = [vp, P(i), vp]
     lib.af_device_error.argtypes = [vp, P(i)]
     lib.af_status_string.argtypes = [i]
@@ -59,7 +67,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.af_last_error_string.argtypes = []
     lib.af_last_error_string.restype = ctypes.c_char_p
     for name in EXPORTS:
-        if name not in ("af_status_string", "af_last_error_string", "af_num_tensors", "af_workspace_bytes"):
+        if name not in ("af_status_string", "af_last_error_string", "af_num_tensors", "af_workspace_bytes",
+                        "flow_pipeline_workspace_bytes"):
             getattr(lib, name).restype = i
     return lib
 
@@ -190,3 +199,66 @@ def last_convergence(ws: torch.Tensor, stream=None) -> int:
     if s not in (AF_OK, AF_NOT_CONVERGED):
         _check(s, "af_last_convergence")
     return n.value
+
+
+def af_inverse_jacobi_schedule(model: AFModel, z: torch.Tensor, direction: int, block_sizes: Sequence[int],
+                               tau: float, max_iter: int, warm_start: bool, b_begin: int = 0, b_end: int | None = None,
+                               ws: torch.Tensor | None = None, x: torch.Tensor | None = None,
+                               iters: torch.Tensor | None = None, stream=None):
+    """Block-Jacobi inverse over a schedule of block sizes, blocks b_begin..b_end-1.
+
+    Returns (x, iters [batch, n_blocks]); only the range's entries are written."""
+    batch, L, _ = z.shape
+    n = len(block_sizes)
+    b_end = n if b_end is None else b_end
+    if ws is None:
+        ws = model.workspace(batch, L, max(block_sizes), device=z.device)
+    x = torch.empty_like(z) if x is None else x
+    iters = torch.zeros((batch, n), dtype=torch.int32, device=z.device) if iters is None else iters
+    sizes = (ctypes.c_int * n)(*[int(b) for b in block_sizes])
+    _check(lib().af_inverse_jacobi_schedule(model.handle, _ptr(z), batch, L, direction, sizes, n, b_begin, b_end,
+                                            float(tau), int(max_iter), int(bool(warm_start)), _ptr(x), _ptr(iters),
+                                            _ptr(ws), ws.numel(), _stream(stream)), "af_inverse_jacobi_schedule")
+    return x, iters
+
+
+def af_prefix_encode(model: AFModel, x: torch.Tensor, direction: int, B: int, n_tokens: int, ws: torch.Tensor,
+                     stream=None):
+    """Writes the K/V of positions 0..n_tokens-1 of x into ws (laid out for blocks of at most B)."""
+    batch, L, _ = x.shape
+    _check(lib().af_prefix_encode(model.handle, _ptr(x), batch, L, direction, B, n_tokens, _ptr(ws), ws.numel(),
+                                  _stream(stream)), "af_prefix_encode")
+
+
+def pipeline_workspace(shallow: List[AFModel], batch: int, frame_len: int, device=None) -> torch.Tensor:
+    n = int(lib().flow_pipeline_workspace_bytes(shallow[0].handle, len(shallow), batch, frame_len))
+    if n == 0:
+        raise AFError(AF_ERR_ARG, "flow_pipeline_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def flow_pipeline_inverse(deep: AFModel, shallow: List[AFModel], shallow_dirs: Sequence[int], z: torch.Tensor,
+                          B: int, tau: float, max_iter_deep: int, max_iter_shallow: int, warm_start: bool,
+                          ws_deep: torch.Tensor | None = None, ws_shallow: torch.Tensor | None = None,
+                          x: torch.Tensor | None = None, iters_deep: torch.Tensor | None = None,
+                          iters_shallow: torch.Tensor | None = None, stream=None, stream_shallow=None):
+    """x = f_S^{-1}(f_D^{-1}(z)), the shallow stack of each frame on a second stream as the deep flow
+    finishes it.  Returns (x, iters_deep [batch, L/B], iters_shallow [T, batch, L/frame_len])."""
+    batch, L, _ = z.shape
+    F = deep.shape.frame_len
+    T = len(shallow)
+    ws_deep = deep.workspace(batch, L, B, device=z.device) if ws_deep is None else ws_deep
+    ws_shallow = pipeline_workspace(shallow, batch, F, device=z.device) if ws_shallow is None else ws_shallow
+    x = torch.empty_like(z) if x is None else x
+    if iters_deep is None:
+        iters_deep = torch.zeros((batch, L // B), dtype=torch.int32, device=z.device)
+    if iters_shallow is None:
+        iters_shallow = torch.zeros((T, batch, L // F), dtype=torch.int32, device=z.device)
+    hs = (ctypes.c_void_p * T)(*[m.handle for m in shallow])
+    ds = (ctypes.c_int * T)(*shallow_dirs)
+    s2 = stream_shallow if stream_shallow is not None else (stream if stream is not None else torch.cuda.current_stream())
+    _check(lib().flow_pipeline_inverse(deep.handle, hs, ds, T, _ptr(z), batch, L, B, float(tau), int(max_iter_deep),
+                                       int(max_iter_shallow), int(bool(warm_start)), _ptr(x), _ptr(iters_deep),
+                                       _ptr(iters_shallow), _ptr(ws_deep), ws_deep.numel(), _ptr(ws_shallow),
+                                       ws_shallow.numel(), _stream(stream), _stream(s2)), "flow_pipeline_inverse")
+    return x, iters_deep, iters_shallow
