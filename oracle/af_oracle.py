@@ -406,6 +406,66 @@ def stack_inverse(blocks: List[Block], dirs: Sequence[int], z: np.ndarray, B: in
 
 
 # ----------------------------------------------------------------------------
+# flow-score-matching denoiser s_phi ([N] key design 2: a light causal
+# Transformer denoiser regressed on the model's score, with one frame of
+# look-ahead; x is refined as x_noisy + sigma * s_phi(x_noisy), the Tweedie
+# step x ~ x_noisy + sigma^2 grad log p with s_phi ~ sigma grad log p)
+# Readings (D1-D3; the pages give only "8-layer Transformer, width of the
+# shallow blocks", the look-ahead s_phi(x_{<=n+1}) ~ (sigma grad log p)_n and
+# the loss):
+#   D1 the denoiser reads x_noisy itself (no shift): h = x W_in^T + b_in + pos;
+#   D2 the same pre-LN layers as the AF block; attention is by frames
+#      (frame_len tokens a frame, every token of a frame sees the whole frame):
+#      in the first layer a token of frame n attends frames <= n + 1, in every
+#      later layer frames <= n -- so the output of frame n depends on frames
+#      <= n + 1 exactly, as the pages' s_phi(x_{<=n+1}) states (a look-ahead
+#      in every layer would reach one more frame per layer);
+#   D3 final LayerNorm, linear head to C outputs s_phi; x = x_noisy + sigma s_phi.
+
+class DenoiserBlock(Block):
+    """Weights of the denoiser: the AF block's layout with a head of C rows."""
+
+
+def lookahead_attention(q, K, V, heads, frame_len, ahead):
+    """softmax(q K^T / sqrt(hd) over keys of frames <= query frame + ahead) V,
+    for queries and keys at positions 0 .. n-1 of one sequence (D2)."""
+    n, d = q.shape
+    hd = d // heads
+    pos = np.arange(n)
+    allowed = (pos[None, :] // frame_len) <= (pos[:, None] // frame_len) + ahead
+    out = np.empty_like(q)
+    for h in range(heads):
+        sl = slice(h * hd, (h + 1) * hd)
+        S = (q[:, sl] @ K[:, sl].T) / math.sqrt(hd)
+        S = np.where(allowed, S, -np.inf)
+        S = S - S.max(axis=1, keepdims=True)
+        E = np.exp(S)
+        out[:, sl] = (E / E.sum(axis=1, keepdims=True)) @ V[:, sl]
+    return out
+
+
+def denoiser_scores(blk: DenoiserBlock, x_noisy: np.ndarray) -> np.ndarray:
+    """s_phi of one sequence [n, C] (D1-D3)."""
+    n = x_noisy.shape[0]
+    d = blk.d
+    h = linear(_f(x_noisy), blk.w_in, blk.b_in) + positions(blk, np.arange(n))
+    for l, P in enumerate(blk.L_):
+        a = layer_norm(h, P["ln1_g"], P["ln1_b"])
+        qkv = linear(a, P["w_qkv"], P["b_qkv"])
+        q, k, v = qkv[:, :d], qkv[:, d:2 * d], qkv[:, 2 * d:]
+        att = lookahead_attention(q, k, v, blk.heads, blk.frame_len, 1 if l == 0 else 0)
+        h = h + linear(att, P["w_o"], P["b_o"])
+        a = layer_norm(h, P["ln2_g"], P["ln2_b"])
+        h = h + linear(gelu(linear(a, P["w_1"], P["b_1"])), P["w_2"], P["b_2"])
+    return linear(layer_norm(h, blk.lnf_g, blk.lnf_b), blk.w_head, blk.b_head)
+
+
+def denoise(blk: DenoiserBlock, x_noisy: np.ndarray, sigma: float) -> np.ndarray:
+    """x_noisy [batch, L, C] -> x_noisy + sigma * s_phi(x_noisy) (float64)."""
+    return np.stack([_f(xb) + sigma * denoiser_scores(blk, xb) for xb in x_noisy])
+
+
+# ----------------------------------------------------------------------------
 # brute-force Jacobian (pins the log-determinant on tiny inputs)
 
 def jacobian_bruteforce(blk: Block, x: np.ndarray, direction: int, h: float = 1e-6):

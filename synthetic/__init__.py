@@ -150,6 +150,36 @@ def make_weights(s: ModelShape, seed: int = WEIGHT_SEED, block: int = 0,
     return out
 
 
+def denoiser_specs(s: ModelShape):
+    """Tensor order of the flow-score-matching denoiser: the AF block's, with a
+    head of C rows (s_phi has one output per channel)."""
+    spec = tensor_specs(s)
+    return spec[:-2] + [("w_head", (s.C, s.d), "w"), ("b_head", (s.C,), "bias")]
+
+
+def make_denoiser_weights(s: ModelShape, seed: int = WEIGHT_SEED, block: int = 100,
+                          perturb: bool = False) -> List[np.ndarray]:
+    """Seeded fp32 denoiser weights in ``denoiser_specs`` order (head ~ N(0, 0.02^2)
+    like the other projections)."""
+    rng = np.random.default_rng([seed, block])
+    out = []
+    for name, shape, kind in denoiser_specs(s):
+        if kind in ("w", "pos"):
+            a = rng.standard_normal(shape, dtype=np.float32) * np.float32(0.02)
+        elif kind in ("bias", "shift"):
+            a = (rng.standard_normal(shape, dtype=np.float32) * np.float32(0.02)
+                 if perturb else np.zeros(shape, np.float32))
+        else:  # gain
+            a = (np.float32(1.0) + rng.standard_normal(shape, dtype=np.float32) * np.float32(0.1)
+                 if perturb else np.ones(shape, np.float32))
+        out.append(np.ascontiguousarray(a, dtype=np.float32))
+    return out
+
+
+# the denoiser of the pipeline: 8 layers at the shallow blocks' width, frames of 390 tokens
+DENOISER = ModelShape(C=192, d=768, heads=12, layers=8, mlp_ratio=4, frame_len=390, max_frames=21, dtype="bf16")
+
+
 def make_stack_weights(w: Workload, **kw) -> List[List[np.ndarray]]:
     return [make_weights(w.shape, block=t, **kw) for t in range(w.T)]
 

@@ -89,6 +89,17 @@ def _warm_from_previous_block(xw, zw, P, Q, frame_len):
     return np.array([xw[p - B] if p - B >= 0 else zw[p] for p in range(P, Q)])
 
 
+_orig_look = O.lookahead_attention
+
+
+def _lookahead_every_layer(q, K, V, heads, frame_len, ahead):
+    return _orig_look(q, K, V, heads, frame_len, 1)
+
+
+def _no_lookahead(q, K, V, heads, frame_len, ahead):
+    return _orig_look(q, K, V, heads, frame_len, 0)
+
+
 def _positions_no_time(blk, p):
     return np.asarray(blk.pos_space, np.float64)[p % blk.frame_len]
 
@@ -109,6 +120,8 @@ MUTATIONS = {
     "residual_denominator_old_iterate": ("jacobi_residual", _residual_old_den),
     "positions_without_time_rows": ("positions", _positions_no_time),
     "warm_start_from_previous_block": ("warm_start_guess", _warm_from_previous_block),
+    "denoiser_lookahead_in_every_layer": ("lookahead_attention", _lookahead_every_layer),
+    "denoiser_without_lookahead": ("lookahead_attention", _no_lookahead),
     "positions_time_index_by_length": ("positions", _positions_time_by_length),
 }
 
@@ -124,6 +137,7 @@ def _any_pin_fails():
     checks.append(P.pin_roundtrip_seq(O.R2L) > 1e-12)
     checks.append(P.pin_positions_hand_written() != 0.0)
     checks.append(P.pin_warm_start_guess() != 0.0)
+    checks.append(P.pin_denoiser_vs_torch() > 1e-12)
     try:
         test_jacobi_iteration_count_closed_form(True)
         checks.append(False)

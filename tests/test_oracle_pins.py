@@ -405,3 +405,82 @@ def pin_warm_start_guess():
 
 def test_warm_start_reaches_back_whole_frames():
     assert pin_warm_start_guess() == 0.0
+
+
+# ---------------------------------------------------------------------------- the denoiser s_phi
+
+DEN = syn.ModelShape(C=4, d=16, heads=2, layers=2, mlp_ratio=4, frame_len=2, max_frames=3, dtype="fp32")
+
+# frames of 2 tokens, 3 frames, written out by hand: row i (query), column j
+# (key); 1 = attends.  First layer: one frame of look-ahead; later layers:
+# frames up to the query's own.
+LOOKAHEAD_MASK_F2_N6 = np.array([[1, 1, 1, 1, 0, 0],
+                                 [1, 1, 1, 1, 0, 0],
+                                 [1, 1, 1, 1, 1, 1],
+                                 [1, 1, 1, 1, 1, 1],
+                                 [1, 1, 1, 1, 1, 1],
+                                 [1, 1, 1, 1, 1, 1]], bool)
+FRAME_CAUSAL_MASK_F2_N6 = np.array([[1, 1, 0, 0, 0, 0],
+                                    [1, 1, 0, 0, 0, 0],
+                                    [1, 1, 1, 1, 0, 0],
+                                    [1, 1, 1, 1, 0, 0],
+                                    [1, 1, 1, 1, 1, 1],
+                                    [1, 1, 1, 1, 1, 1]], bool)
+
+
+def pin_denoiser_vs_torch():
+    """s_phi of the oracle vs torch.nn pre-LN TransformerEncoderLayers built
+    from the same weights, with the hand-written look-ahead mask."""
+    w = syn.make_denoiser_weights(DEN, perturb=True)
+    blk = O.DenoiserBlock(DEN, w)
+    x = np.random.default_rng(17).standard_normal((6, DEN.C))
+    t = lambda a: torch.tensor(np.asarray(a, np.float64))
+    d, C = DEN.d, DEN.C
+    inp = torch.nn.Linear(C, d, dtype=torch.float64)
+    inp.weight.data, inp.bias.data = t(blk.w_in), t(blk.b_in)
+    layers = []
+    for P in blk.L_:
+        L = torch.nn.TransformerEncoderLayer(d, DEN.heads, DEN.mlp_ratio * d, dropout=0.0, activation="gelu",
+                                             layer_norm_eps=1e-5, batch_first=True, norm_first=True,
+                                             dtype=torch.float64)
+        L.self_attn.in_proj_weight.data, L.self_attn.in_proj_bias.data = t(P["w_qkv"]), t(P["b_qkv"])
+        L.self_attn.out_proj.weight.data, L.self_attn.out_proj.bias.data = t(P["w_o"]), t(P["b_o"])
+        L.linear1.weight.data, L.linear1.bias.data = t(P["w_1"]), t(P["b_1"])
+        L.linear2.weight.data, L.linear2.bias.data = t(P["w_2"]), t(P["b_2"])
+        L.norm1.weight.data, L.norm1.bias.data = t(P["ln1_g"]), t(P["ln1_b"])
+        L.norm2.weight.data, L.norm2.bias.data = t(P["ln2_g"]), t(P["ln2_b"])
+        layers.append(L.train(False))
+    lnf = torch.nn.LayerNorm(d, eps=1e-5, dtype=torch.float64)
+    lnf.weight.data, lnf.bias.data = t(blk.lnf_g), t(blk.lnf_b)
+    head = torch.nn.Linear(d, C, dtype=torch.float64)
+    head.weight.data, head.bias.data = t(blk.w_head), t(blk.b_head)
+    pos = torch.arange(6)
+    masks = [torch.tensor(~LOOKAHEAD_MASK_F2_N6), torch.tensor(~FRAME_CAUSAL_MASK_F2_N6)]   # True = masked out
+    with torch.no_grad():
+        h = inp(t(x)) + t(blk.pos_space)[pos % DEN.frame_len] + t(blk.pos_time)[pos // DEN.frame_len]
+        h = h[None]
+        for l, L in enumerate(layers):
+            h = L(h, src_mask=masks[0 if l == 0 else 1])
+        ref = head(lnf(h))[0].numpy()
+    return rel(O.denoiser_scores(blk, x), ref)
+
+
+def test_denoiser_matches_torch_with_lookahead_mask():
+    assert pin_denoiser_vs_torch() < 1e-12
+
+
+def test_denoiser_looks_exactly_one_frame_ahead():
+    """The output of frame n depends on frames <= n + 1 (the pages' s_phi(x_{<=n+1}))."""
+    blk = O.DenoiserBlock(DEN, syn.make_denoiser_weights(DEN, perturb=True))
+    x = np.random.default_rng(18).standard_normal((1, 6, DEN.C))
+    y = O.denoise(blk, x, 0.3)
+    x2 = x.copy()
+    x2[0, 4:] += 1.0                                      # frame 2
+    y2 = O.denoise(blk, x2, 0.3)
+    np.testing.assert_array_equal(y2[0, :2], y[0, :2])    # frame 0 does not see frame 2
+    assert np.abs(y2[0, 2:4] - y[0, 2:4]).max() > 1e-6    # frame 1 does
+    x3 = x.copy()
+    x3[0, 2:4] += 1.0                                     # frame 1
+    y3 = O.denoise(blk, x3, 0.3)
+    assert np.abs(y3[0, :2] - y[0, :2]).max() > 1e-6      # frame 0 sees frame 1
+    np.testing.assert_array_equal(O.denoise(blk, x, 0.0), x)   # sigma = 0 leaves x unchanged
