@@ -166,6 +166,25 @@ af_status af_inverse_jacobi_schedule(const af_model* m, const float* z, int batc
 af_status af_prefix_encode(const af_model* m, const float* x, int batch, int L, af_dir dir, int B, int n_tokens,
                            void* ws, size_t ws_bytes, void* stream);
 
+/* Streaming generation past the model's length ("A complete example": a
+ * sliding window over the deep flow -- after a chunk of latents is
+ * produced, f_D is re-run on the last `overlap` latents to rebuild the KV
+ * cache, and the next frames are generated).  z, x: [batch, n_frames *
+ * frame_len, C], any n_frames; direction L->R, one frame per Jacobi block.
+ * Window w covers `window` frames (<= max_frames) starting at frame
+ * s_w = w * (window - overlap) (the last window may be shorter); it runs at
+ * the model's positions 0 .. window*frame_len - 1.  Its first `overlap`
+ * frames (after the first window) are the previous window's output,
+ * flow-encoded into the cache (af_prefix_encode); the rest are generated by
+ * block-Jacobi (tau, max_iter, warm_start as in af_inverse_jacobi).
+ * iters [batch, n_frames] holds each frame's count from the window that
+ * generated it.  ws: af_stream_workspace_bytes(m, batch, window) (a
+ * window's workspace plus staging of its x and z).  0 <= overlap < window. */
+size_t af_stream_workspace_bytes(const af_model* m, int batch, int window);
+af_status af_inverse_jacobi_stream(const af_model* m, const float* z, int batch, int n_frames, int window, int overlap,
+                                   float tau, int max_iter, int warm_start, float* x, int32_t* iters, void* ws,
+                                   size_t ws_bytes, void* stream);
+
 /* Bytes of the shallow-side workspace of flow_pipeline_inverse for T shallow
  * blocks (config of `shallow`), `batch` videos, frames of frame_len tokens. */
 size_t flow_pipeline_workspace_bytes(const af_model* shallow, int T, int batch, int frame_len);
@@ -195,6 +214,30 @@ af_status flow_pipeline_inverse(const af_model* deep, const af_model* const* sha
                                 int32_t* iters_shallow, void* ws_deep, size_t ws_deep_bytes, void* ws_shallow,
                                 size_t ws_shallow_bytes, void* stream_deep, void* stream_shallow);
 
+/* The flow-score-matching denoiser s_phi ("Key design 2": a light causal
+ * Transformer trained to regress sigma * grad log p of the flow at the noisy
+ * sample, with one frame of look-ahead, s_phi(x_{<=n+1}) ~ (sigma grad log
+ * p)_n; it refines the flow's slightly noisy output).  Same af_config and
+ * tensor order as af_model_create except the head: W_head [C, d], b_head [C]
+ * (plain outputs, no (mu, s) pairs).  Readings (the pages give only "8-layer
+ * Transformer, width of the shallow blocks"): the input is x_noisy itself
+ * (no shift); h = x W_in^T + b_in + P_space[p mod frame_len] + P_time[p div
+ * frame_len]; pre-LN layers as in the AF block, with attention by frames of
+ * frame_len tokens -- in the first layer a token of frame n attends every
+ * token of frames <= n + 1, in later layers frames <= n -- so frame n's
+ * output depends on frames <= n + 1 exactly; final LayerNorm and head give
+ * s_phi.  AF_BF16 / AF_FP32 as for the AF block.  The model can only be used
+ * with af_denoise (the flow calls reject it). */
+int af_denoiser_num_tensors(const af_config* cfg);
+af_status af_denoiser_create(const af_config* cfg, const float* const* tensors, int n_tensors,
+                             af_model** out);
+
+/* x = x_noisy + sigma * s_phi(x_noisy) (the Tweedie step with s_phi ~ sigma
+ * grad log p), x_noisy and x [batch, L, C], L <= max_len, sigma finite.
+ * ws: af_workspace_bytes(m, batch, L, L). */
+af_status af_denoise(const af_model* m, const float* x_noisy, int batch, int L, float sigma, float* x, void* ws,
+                     size_t ws_bytes, void* stream);
+
 /* af_forward for callers that cannot allocate device memory -- a host that
  * owns the whole GPU memory through its own allocator, or a plugin that is
  * handed only its input and output buffers, and so cannot provide a
@@ -217,8 +260,21 @@ af_status af_forward_noalloc(const af_model* m, const float* x, int batch, int L
  * (*n_unconverged set). */
 af_status af_last_convergence(void* ws, int* n_unconverged, void* stream);
 
-/* Synchronises the device and returns AF_ERR_DEVICE (and clears the flag)
- * if any kernel of this model gave up a bounded wait; *code says where. */
+/* Failure detection: every wait of the tensor-core kernels' pipelines (on a
+ * TMA load, an MMA, a buffer hand-off between warps) is bounded.  A wait that
+ * runs past `seconds` (default 2) makes its CTA abort: every role stops, the
+ * loads and MMAs already in flight are waited for (each with its own 2 s
+ * bound), tensor memory is freed, and the model's error word is set for
+ * af_device_error.  The results of that call are then undefined; later calls
+ * are unaffected.  Applies to calls enqueued after it (graphs captured with
+ * another limit are captured anew).  AF_ERR_ARG unless 0 < seconds <= 60.
+ * No counterpart in the paper. */
+af_status af_set_wait_limit(af_model* m, double seconds);
+
+/* Synchronises the device and returns AF_ERR_DEVICE (and clears the word)
+ * if any kernel of this model gave up a bounded wait; *code is a bit mask of
+ * where: 1 a GEMM pipeline wait, 4 an attention pipeline wait, 2 a drain
+ * after an abort that did not see its in-flight work complete in time. */
 af_status af_device_error(const af_model* m, int* code);
 
 const char* af_status_string(af_status s);

@@ -382,6 +382,45 @@ def af_inverse_jacobi(blk: Block, z: np.ndarray, direction: int, B, tau: float,
             np.stack([o[2] for o in out]))
 
 
+def window_starts(n_frames: int, window: int, overlap: int) -> List[int]:
+    """First frames of the windows of a stream of n_frames frames: windows of
+    `window` frames, each after the first repeating the last `overlap` frames
+    of the one before ([N] "A complete example": streaming generation)."""
+    assert 0 <= overlap < window
+    starts = [0]
+    while starts[-1] + window < n_frames:
+        starts.append(starts[-1] + window - overlap)
+    return starts
+
+
+def af_inverse_jacobi_stream(blk: Block, z: np.ndarray, frame_len: int, window: int, overlap: int,
+                             tau: float, max_iter: int, warm_start: bool):
+    """Streaming block-Jacobi inverse past the model's length ([N] "A complete
+    example": after a latent chunk is produced, f_D is re-run on the last
+    `overlap` latents to rebuild the KV cache, and the next window_frames -
+    overlap frames are generated).  z [batch, n_frames*frame_len, C], L->R,
+    one frame per block.  Window w covers frames s_w .. s_w + window - 1
+    (window_starts), at positions 0 .. window*frame_len - 1 of the model; its
+    first `overlap` frames (after the first window) are the previous window's
+    output, observed (flow-encoded into the cache), and the rest are
+    generated.  Returns (x, iters [batch, n_frames]; observed frames count 0
+    in the window that observes them, their own generating window's count is
+    kept)."""
+    batch, L, C = z.shape
+    n_frames = L // frame_len
+    x = np.zeros((batch, L, C))
+    iters = np.zeros((batch, n_frames), np.int64)
+    for i, s0 in enumerate(window_starts(n_frames, window, overlap)):
+        nf = min(window, n_frames - s0)
+        lo, hi = s0 * frame_len, (s0 + nf) * frame_len
+        n_obs = overlap if i > 0 else 0
+        xw, it, _ = af_inverse_jacobi(blk, z[:, lo:hi], L2R, frame_len, tau, max_iter, warm_start,
+                                      x_known=x[:, lo:hi] if n_obs else None, n_known=n_obs)
+        x[:, lo + n_obs * frame_len:hi] = xw[:, n_obs * frame_len:]
+        iters[:, s0 + n_obs:s0 + nf] = it[:, n_obs:]
+    return x, iters
+
+
 # ----------------------------------------------------------------------------
 # stacks of alternating-direction blocks ([N] key design 1: T >= 3 blocks of
 # alternating direction; inversion undoes them last-to-first)

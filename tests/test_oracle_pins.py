@@ -484,3 +484,38 @@ def test_denoiser_looks_exactly_one_frame_ahead():
     y3 = O.denoise(blk, x3, 0.3)
     assert np.abs(y3[0, :2] - y[0, :2]).max() > 1e-6      # frame 0 sees frame 1
     np.testing.assert_array_equal(O.denoise(blk, x, 0.0), x)   # sigma = 0 leaves x unchanged
+
+
+# ---------------------------------------------------------------------------- streaming window
+
+def test_window_starts():
+    assert O.window_starts(7, 4, 1) == [0, 3]            # frames 0-3, then 3-6
+    assert O.window_starts(4, 4, 1) == [0]
+    assert O.window_starts(5, 4, 2) == [0, 2]
+    assert O.window_starts(10, 3, 0) == [0, 3, 6, 9]
+
+
+def test_stream_with_one_window_is_the_plain_inverse():
+    blk = tiny_block(head_std=0.2)
+    z = np.random.default_rng(19).standard_normal((2, 24, TINY.C))
+    x1, it1, _ = O.af_inverse_jacobi(blk, z, O.L2R, 8, 1e-6, 8, True)
+    x2, it2 = O.af_inverse_jacobi_stream(blk, z, 8, 3, 1, 1e-6, 8, True)
+    np.testing.assert_array_equal(x1, x2)
+    np.testing.assert_array_equal(it1, it2)
+
+
+def test_stream_windows_invert_their_own_forward():
+    """Each window is an exact inverse problem (tau = 0, B sweeps): the stream
+    reproduces x wherever z was made by the forward pass of the same window
+    with the observed frames in front."""
+    blk = tiny_block(head_std=0.3)                    # frames of 8 tokens, the model holds 3
+    F, W, D = 8, 3, 1
+    rng = np.random.default_rng(20)
+    x_true = rng.standard_normal((1, 5 * F, TINY.C))   # 5 frames: windows [0,3) and [2,5)
+    z = np.zeros_like(x_true)
+    z[:, :3 * F], _ = O.af_forward(blk, x_true[:, :3 * F], O.L2R)
+    zw, _ = O.af_forward(blk, x_true[:, 2 * F:5 * F], O.L2R)
+    z[:, 3 * F:] = zw[:, F:]
+    x, it = O.af_inverse_jacobi_stream(blk, z, F, W, D, 0.0, F, True)
+    assert rel(x, x_true) < 1e-12
+    assert it.shape == (1, 5) and (it == F).all()

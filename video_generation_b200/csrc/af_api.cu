@@ -76,6 +76,8 @@ struct af_model {
   int num_sms;
   int device;         // the CUDA device holding the weights
   int pdl;            // launch with programmatic dependent launch (see af_kernels.h)
+  uint64_t wait_ns;   // limit of one pipeline wait in the tensor-core kernels
+  int kind;           // KIND_FLOW (an AF block) or KIND_DENOISER
   std::vector<void*> allocs;
   // graph cache (keyed by every pointer and scalar baked into the graph)
   std::map<std::string, cudaGraphExec_t> graphs;
@@ -85,6 +87,12 @@ struct af_model {
 };
 
 namespace {
+
+// What an af_model computes: an affine AF block (input shifted by one token,
+// token-causal attention, head of interleaved (mu, s) pairs) or the
+// flow-score-matching denoiser (input unshifted, attention by frames with one
+// frame of look-ahead in the first layer, head of C plain outputs).
+enum { KIND_FLOW = 0, KIND_DENOISER = 1 };
 
 // ------------------------------------------------------------------ workspace
 
@@ -148,9 +156,10 @@ Bufs carve(const af_model* m, void* ws, int batch, int L, int B) {
 // ------------------------------------------------------------------ one pass
 
 struct HeadIO {
-  int mode;             // 0 forward, 1 Jacobi update
-  const float* xin_f;   // forward: x   inverse: z
-  float* xout_f;        // forward: z   inverse: x
+  int mode;             // 0 forward, 1 Jacobi update, 2 denoise
+  const float* xin_f;   // forward: x   inverse: z   denoise: x_noisy
+  float* xout_f;        // forward: z   inverse: x   denoise: x
+  float sigma;          // denoise: the noise level
 };
 
 // One pass of the AF block over the rows described by ctl (see af_common.cuh):
@@ -165,6 +174,7 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
   e.ctl = b.ctl;
   e.h = b.h;
   e.d = d;
+  e.wait_ns = m->wait_ns;
   e.Lc = L;
   e.pos_space = m->pos_space;
   e.pos_time = m->pos_time;
@@ -175,6 +185,15 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
   EpiArgs eh = e;
   eh.bias = m->b_head;
   eh.head_mode = hio.mode;
+  eh.sigma = hio.sigma;
+  // the AF block's self-exclusive mask is a one-token input shift with
+  // token-causal attention; the denoiser reads its input unshifted and
+  // attends by frames, one frame ahead in its first layer only
+  const bool den = m->kind == KIND_DENOISER;
+  const int shift = den ? 0 : 1;
+  const int head_n = den ? C : 2 * C;
+  auto mask_frame = [&](int l) { return den ? c.frame_len : 0; };
+  auto mask_ahead = [&](int l) { return den && l == 0 ? 1 : 0; };
   eh.L = L;
   eh.C = C;
   eh.dir = dir;
@@ -188,7 +207,7 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
     float* a = (float*)b.a;
     float* q = (float*)b.q;
     float* u = (float*)b.u;
-    launch_gather<float>(b.ctl, xsrc, L, C, dir, xin, m_max, st);
+    launch_gather<float>(b.ctl, xsrc, L, C, dir, shift, xin, m_max, st);
     e.bias = m->b_in;
     launch_gemm_simt(EPI_INPROJ, xin, (const float*)m->w_in, d, C, m_max, e, st);
     for (int l = 0; l < c.layers; ++l) {
@@ -201,7 +220,8 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
       eq.kc = kvl;
       eq.vc = kvl + kv_layer;
       launch_gemm_simt(EPI_QKV, a, (const float*)w.w_qkv, 3 * d, d, m_max, eq, st);
-      launch_attn_simt(b.ctl, q, (const float*)kvl, (const float*)(kvl + kv_layer), a, batch, L, d, c.heads, m_max, st);
+      launch_attn_simt(b.ctl, q, (const float*)kvl, (const float*)(kvl + kv_layer), a, batch, L, d, c.heads, m_max,
+                       mask_frame(l), mask_ahead(l), st);
       EpiArgs eo = e;
       eo.bias = w.b_o;
       launch_gemm_simt(EPI_RESID, a, (const float*)w.w_o, d, d, m_max, eo, st);
@@ -216,7 +236,7 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
       launch_gemm_simt(EPI_RESID, u, (const float*)w.w_2, d, fd, m_max, ed, st);
     }
     launch_layernorm<float>(b.ctl, b.h, m->lnf_g, m->lnf_b, a, d, m_max, st);
-    launch_head_simt(a, (const float*)m->w_head, 2 * C, d, m_max, eh, st);
+    launch_head_simt(a, (const float*)m->w_head, head_n, d, m_max, eh, st);
   } else {
     bf16* xin = (bf16*)b.xin;
     bf16* a = (bf16*)b.a;
@@ -238,7 +258,7 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
                      m_max, ea, m->d_err, ns, st);
       return true;
     };
-    launch_gather<bf16>(b.ctl, xsrc, L, C, dir, xin, m_max, st);
+    launch_gather<bf16>(b.ctl, xsrc, L, C, dir, shift, xin, m_max, st);
     e.bias = m->b_in;
     if (!gemm(EPI_INPROJ, tA_x, m->w_in, d, C, e)) { set_err("GEMM plan failed (in-proj)"); return AF_ERR_CUDA; }
     for (int l = 0; l < c.layers; ++l) {
@@ -256,7 +276,8 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
       }
       if (!gemm(EPI_QKV, tA_a, w.w_qkv, 3 * d, d, eq)) { set_err("GEMM plan failed (qkv)"); return AF_ERR_CUDA; }
       if (!launch_attn_tc2(b.ctl, q, (const bf16*)kvl, (const bf16*)(kvl + kv_layer), a, b.opart, b.mlpart, b.nsplit,
-                           batch, L, d, c.heads, r_max, m_max, m->num_sms, m->d_err, st)) {
+                           batch, L, d, c.heads, r_max, m_max, m->num_sms, m->wait_ns, mask_frame(l), mask_ahead(l),
+                           m->d_err, st)) {
         set_err("attention plan failed");
         return AF_ERR_CUDA;
       }
@@ -274,7 +295,7 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
       if (!gemm(EPI_RESID, tA_u, w.w_2, d, fd, ed)) { set_err("GEMM plan failed (mlp down)"); return AF_ERR_CUDA; }
     }
     launch_layernorm<bf16>(b.ctl, b.h, m->lnf_g, m->lnf_b, a, d, m_max, st);
-    if (!gemm(EPI_HEAD, tA_a, m->w_head, 2 * C, d, eh)) { set_err("GEMM plan failed (head)"); return AF_ERR_CUDA; }
+    if (!gemm(EPI_HEAD, tA_a, m->w_head, head_n, d, eh)) { set_err("GEMM plan failed (head)"); return AF_ERR_CUDA; }
   }
   (void)G;
   CK(cudaGetLastError());
@@ -399,7 +420,7 @@ af_status capture_jacobi(const JacobiJob& jb, const Bufs& b, int batch, int L, i
     if (cudaStreamBeginCaptureToGraph(cs2, body_inner, nullptr, nullptr, 0, cudaStreamCaptureModeRelaxed) != cudaSuccess) {
       set_err("capture of the update loop failed"); rc = AF_ERR_CUDA; break;
     }
-    HeadIO hio{1, jb.z, jb.x};
+    HeadIO hio{1, jb.z, jb.x, 0.f};
     rc = enqueue_pass(m, b, batch, L, jb.dir, m_max, r_max, jb.x, hio, cs2);
     if (!rc) launch_jacobi_step(b.ctl, b.btab, b.active, b.part, batch, G, tau, max_iter, jb.iters, h_inner, cs2);
     if (cudaStreamEndCapture(cs2, &dummy) != cudaSuccess && !rc) { set_err("end of update capture failed"); rc = AF_ERR_CUDA; }
@@ -501,7 +522,7 @@ af_status build_forward(void* vctx, cudaStream_t cs) {
     const float* in = t == 0 ? c->x : (((c->T - t) % 2 == 0) ? c->z : c->b.tmp);
     float* out = ((c->T - 1 - t) % 2 == 0) ? c->z : c->b.tmp;
     launch_ctl_forward(c->b.ctl, c->batch, c->L, cs);
-    HeadIO hio{0, in, out};
+    HeadIO hio{0, in, out, 0.f};
     af_status s = enqueue_pass(c->blocks[t], c->b, c->batch, c->L, c->dirs[t], m_max, c->L, in, hio, cs);
     if (s) return s;
     launch_logdet_finalize(c->b.part, c->batch, c->L, G, c->logdet, t > 0, cs);
@@ -550,7 +571,7 @@ af_status run_inverse(const af_model* const* blocks, const af_dir* dirs, int T, 
   uint32_t taubits;
   memcpy(&taubits, &tau, 4);
   std::string key = keyf("inv", {(long long)z, (long long)x, (long long)iters, (long long)ws, batch, L, sc.B_max, nb,
-                                 (long long)taubits, max_iter, c.warm, T});
+                                 (long long)taubits, max_iter, c.warm, T, (long long)blocks[0]->wait_ns});
   for (int t = 0; t < T; ++t) key += keyf("", {(long long)blocks[t], dirs[t]});
   return graph_run(blocks[0], key, st, build_inverse, &c);
 }
@@ -596,10 +617,30 @@ af_status build_encode(void* vctx, cudaStream_t cs) {
   for (int p0 = 0; p0 < c->n_tokens; p0 += r_max) {
     const int R = (c->n_tokens - p0) < r_max ? (c->n_tokens - p0) : r_max;
     launch_set_pass(c->b.ctl, p0, R, c->batch, vtail, 2 * kv_layer, m->cfg.layers, c->L, m->cfg.d, cs);
-    HeadIO hio{1, c->x, c->b.tmp};                 // no row reaches the head's output
+    HeadIO hio{1, c->x, c->b.tmp, 0.f};            // no row reaches the head's output
     af_status s = enqueue_pass(m, c->b, c->batch, c->L, c->dir, m_max, r_max, c->x, hio, cs);
     if (s) return s;
   }
+  CK(cudaGetLastError());
+  return AF_OK;
+}
+
+struct DenCtx {
+  const af_model* m;
+  const float* xn;
+  float* x;
+  int batch, L;
+  float sigma;
+  Bufs b;
+};
+
+// The denoiser's forward pass over all positions of every sequence.
+af_status build_denoise(void* vctx, cudaStream_t cs) {
+  DenCtx* c = static_cast<DenCtx*>(vctx);
+  launch_ctl_forward(c->b.ctl, c->batch, c->L, cs);
+  HeadIO hio{2, c->xn, c->x, c->sigma};
+  af_status s = enqueue_pass(c->m, c->b, c->batch, c->L, AF_L2R, c->batch * c->L, c->L, c->xn, hio, cs);
+  if (s) return s;
   CK(cudaGetLastError());
   return AF_OK;
 }
@@ -608,6 +649,7 @@ af_status stack_checks(const af_model* const* blocks, const af_dir* dirs, int T,
   if (!blocks || !dirs || T < 1) { set_err("blocks/dirs/T"); return AF_ERR_ARG; }
   for (int t = 0; t < T; ++t) {
     if (!blocks[t]) { set_err("null block %d", t); return AF_ERR_ARG; }
+    if (blocks[t]->kind != KIND_FLOW) { set_err("block %d is a denoiser, not an AF block", t); return AF_ERR_ARG; }
     if (!same_cfg(blocks[t]->cfg, blocks[0]->cfg)) { set_err("blocks must share one config"); return AF_ERR_ARG; }
     if (dirs[t] != AF_L2R && dirs[t] != AF_R2L) { set_err("bad direction"); return AF_ERR_ARG; }
     if (blocks[t]->device != blocks[0]->device) { set_err("blocks must live on one device"); return AF_ERR_ARG; }
@@ -651,7 +693,11 @@ extern "C" {
 
 int af_num_tensors(const af_config* cfg) { return cfg ? 4 + 12 * cfg->layers + 4 : 0; }
 
-af_status af_model_create(const af_config* cfg, const float* const* tensors, int n_tensors, af_model** out) {
+}  // extern "C"
+
+namespace {
+
+af_status create_model(const af_config* cfg, const float* const* tensors, int n_tensors, af_model** out, int kind) {
   if (!cfg || !tensors || !out) { set_err("null argument"); return AF_ERR_ARG; }
   const af_config c = *cfg;
   if (c.C <= 0 || c.d <= 0 || c.heads <= 0 || c.layers <= 0 || c.mlp_ratio <= 0 || c.frame_len <= 0 ||
@@ -676,7 +722,9 @@ af_status af_model_create(const af_config* cfg, const float* const* tensors, int
     if (!tensors[i]) { set_err("null tensor %d", i); return AF_ERR_ARG; }
 
   af_model* m = new af_model();
+  m->kind = kind;
   m->pdl = 1;
+  m->wait_ns = 2000000000ull;
   if (const char* v = getenv("AF_PDL")) m->pdl = atoi(v) != 0;
   m->cfg = c;
   m->fd = c.mlp_ratio * c.d;
@@ -746,7 +794,11 @@ af_status af_model_create(const af_config* cfg, const float* const* tensors, int
   }
   m->lnf_g = upload_v(tensors[k++], d);
   m->lnf_b = upload_v(tensors[k++], d);
-  {
+  if (kind == KIND_DENOISER) {                  // head [C, d], b [C] as given
+    m->w_head = upload_w(tensors[k], C * d);
+    m->b_head = upload_v(tensors[k + 1], C);
+    k += 2;
+  } else {
     const float* wh = tensors[k++];
     const float* bh = tensors[k++];
     std::vector<float> wi(2 * C * d), bi(2 * C);
@@ -774,6 +826,20 @@ af_status af_model_create(const af_config* cfg, const float* const* tensors, int
   }
   *out = m;
   return AF_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+af_status af_model_create(const af_config* cfg, const float* const* tensors, int n_tensors, af_model** out) {
+  return create_model(cfg, tensors, n_tensors, out, KIND_FLOW);
+}
+
+int af_denoiser_num_tensors(const af_config* cfg) { return af_num_tensors(cfg); }
+
+af_status af_denoiser_create(const af_config* cfg, const float* const* tensors, int n_tensors, af_model** out) {
+  return create_model(cfg, tensors, n_tensors, out, KIND_DENOISER);
 }
 
 af_status af_model_destroy(af_model* m) {
@@ -808,7 +874,8 @@ af_status flow_stack_forward(const af_model* const* blocks, const af_dir* dirs, 
   if (!x || !z || !logdet || x == z) { set_err("x/z/logdet (x and z must not alias)"); return AF_ERR_ARG; }
   if (af_status s = check_ws(blocks[0], ws, ws_bytes, batch, L, L)) return s;
   FwdCtx c{blocks, dirs, T, batch, L, x, z, logdet, carve(blocks[0], ws, batch, L, L)};
-  std::vector<long long> kv = {(long long)x, (long long)z, (long long)logdet, (long long)ws, batch, L, T};
+  std::vector<long long> kv = {(long long)x, (long long)z, (long long)logdet, (long long)ws, batch, L, T,
+                               (long long)blocks[0]->wait_ns};
   std::string key = keyf("fwd", {});
   for (int t = 0; t < T; ++t) key += keyf("", {(long long)blocks[t], dirs[t]});
   for (long long v : kv) key += keyf("", {v});
@@ -880,7 +947,7 @@ af_status af_prefix_encode(const af_model* m, const float* x, int batch, int L, 
   const int Bc = B < L ? B : L;
   EncCtx c{m, x, batch, L, Bc, n_tokens, dir, carve(m, ws, batch, L, Bc)};
   g_pdl = m->pdl;
-  std::string key = keyf("enc", {(long long)x, (long long)ws, batch, L, Bc, n_tokens, dir});
+  std::string key = keyf("enc", {(long long)x, (long long)ws, batch, L, Bc, n_tokens, dir, (long long)m->wait_ns});
   return graph_run(m, key, (cudaStream_t)stream, build_encode, &c);
 }
 
@@ -963,6 +1030,71 @@ af_status flow_pipeline_inverse(const af_model* deep, const af_model* const* sha
   return AF_OK;
 }
 
+size_t af_stream_workspace_bytes(const af_model* m, int batch, int window) {
+  if (!m || batch < 1 || window < 1) return 0;
+  const int F = m->cfg.frame_len;
+  const int Lw = window * F;
+  const size_t base = af_workspace_bytes(m, batch, Lw, F);
+  if (!base) return 0;
+  const size_t frames = align256((size_t)batch * Lw * m->cfg.C * sizeof(float));
+  return base + 2 * frames + align256((size_t)batch * window * sizeof(int32_t));
+}
+
+af_status af_inverse_jacobi_stream(const af_model* m, const float* z, int batch, int n_frames, int window, int overlap,
+                                   float tau, int max_iter, int warm_start, float* x, int32_t* iters, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  af_dir dirs[1] = {AF_L2R};
+  const af_model* blocks[1] = {m};
+  cudaStream_t st = (cudaStream_t)stream;
+  if (af_status s = stack_checks(blocks, dirs, 1, st)) return s;
+  if (!z || !x || !iters || x == z) { set_err("z/x/iters (x and z must not alias)"); return AF_ERR_ARG; }
+  const int F = m->cfg.frame_len, C = m->cfg.C;
+  if (n_frames < 1 || window < 1 || window > m->cfg.max_frames || overlap < 0 || overlap >= window ||
+      max_iter < 1 || !(tau >= 0.f) || tau == INFINITY) {
+    set_err("need n_frames >= 1, 1 <= window <= max_frames, 0 <= overlap < window, max_iter >= 1, finite tau >= 0");
+    return AF_ERR_ARG;
+  }
+  const size_t need = af_stream_workspace_bytes(m, batch, window);
+  if (!need || !ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < need) {
+    set_err("stream workspace: need %zu bytes, 256-aligned; got %zu", need, ws_bytes);
+    return AF_ERR_WORKSPACE;
+  }
+  // the window's own workspace, then the staged window of x and z and its counts
+  const size_t win_bytes = af_workspace_bytes(m, batch, window * F, F);
+  const size_t frames = align256((size_t)batch * window * F * C * sizeof(float));
+  char* base = static_cast<char*>(ws);
+  float* xw = (float*)(base + win_bytes);
+  float* zw = (float*)(base + win_bytes + frames);
+  int32_t* itw = (int32_t*)(base + win_bytes + 2 * frames);
+  const size_t rowL = (size_t)n_frames * F * C * sizeof(float);     // pitch of z and x
+  for (int s0 = 0, i = 0;; s0 += window - overlap, ++i) {
+    const int nf = (n_frames - s0) < window ? (n_frames - s0) : window;
+    const int Lw = nf * F;
+    const int n_obs = i > 0 ? overlap : 0;
+    const size_t rowW = (size_t)Lw * C * sizeof(float);
+    const size_t off = (size_t)s0 * F * C;
+    CK(cudaMemcpy2DAsync(zw, rowW, z + off, rowL, rowW, batch, cudaMemcpyDeviceToDevice, st));
+    std::vector<int> sizes(nf, F);
+    if (n_obs) {
+      // the previous window's last frames, observed: flow-encoded into the cache
+      const size_t rowO = (size_t)n_obs * F * C * sizeof(float);
+      CK(cudaMemcpy2DAsync(xw, rowW, x + off, rowL, rowO, batch, cudaMemcpyDeviceToDevice, st));
+      if (af_status s = af_prefix_encode(m, xw, batch, Lw, AF_L2R, F, n_obs * F, ws, win_bytes, stream)) return s;
+    }
+    if (af_status s = af_inverse_jacobi_schedule(m, zw, batch, Lw, AF_L2R, sizes.data(), nf, n_obs, nf, tau, max_iter,
+                                                 warm_start, xw, itw, ws, win_bytes, stream))
+      return s;
+    const size_t skip = (size_t)n_obs * F * C;
+    CK(cudaMemcpy2DAsync(x + off + skip, rowL, xw + skip, rowW, rowW - skip * sizeof(float), batch,
+                         cudaMemcpyDeviceToDevice, st));
+    CK(cudaMemcpy2DAsync(iters + s0 + n_obs, (size_t)n_frames * sizeof(int32_t), itw + n_obs,
+                         (size_t)nf * sizeof(int32_t), (size_t)(nf - n_obs) * sizeof(int32_t), batch,
+                         cudaMemcpyDeviceToDevice, st));
+    if (s0 + window >= n_frames) break;
+  }
+  return AF_OK;
+}
+
 af_status af_last_convergence(void* ws, int* n_unconverged, void* stream) {
   if (!ws || !n_unconverged) { set_err("null argument"); return AF_ERR_ARG; }
   CK(cudaStreamSynchronize((cudaStream_t)stream));
@@ -970,6 +1102,29 @@ af_status af_last_convergence(void* ws, int* n_unconverged, void* stream) {
   CK(cudaMemcpy(&c, ws, sizeof c, cudaMemcpyDeviceToHost));
   *n_unconverged = c.nonconv;
   return c.nonconv ? AF_NOT_CONVERGED : AF_OK;
+}
+
+af_status af_denoise(const af_model* m, const float* x_noisy, int batch, int L, float sigma, float* x, void* ws,
+                     size_t ws_bytes, void* stream) {
+  if (!m || m->kind != KIND_DENOISER) { set_err("af_denoise needs a model from af_denoiser_create"); return AF_ERR_ARG; }
+  if (af_status s = device_checks(m, (cudaStream_t)stream)) return s;
+  if (!x_noisy || !x || x == x_noisy) { set_err("x_noisy/x (they must not alias)"); return AF_ERR_ARG; }
+  if (!(sigma == sigma) || sigma == INFINITY || sigma == -INFINITY) { set_err("sigma must be finite"); return AF_ERR_ARG; }
+  if (af_status s = check_ws(m, ws, ws_bytes, batch, L, L)) return s;
+  DenCtx c{m, x_noisy, x, batch, L, sigma, carve(m, ws, batch, L, L)};
+  g_pdl = m->pdl;
+  uint32_t sb;
+  memcpy(&sb, &sigma, 4);
+  std::string key = keyf("den", {(long long)x_noisy, (long long)x, (long long)ws, batch, L, (long long)sb,
+                                 (long long)m->wait_ns});
+  return graph_run(m, key, (cudaStream_t)stream, build_denoise, &c);
+}
+
+af_status af_set_wait_limit(af_model* m, double seconds) {
+  if (!m || !(seconds > 0.0) || seconds > 60.0) { set_err("need a model and 0 < seconds <= 60"); return AF_ERR_ARG; }
+  m->wait_ns = (uint64_t)(seconds * 1e9);
+  if (m->wait_ns < 1) m->wait_ns = 1;
+  return AF_OK;
 }
 
 af_status af_device_error(const af_model* m, int* code) {

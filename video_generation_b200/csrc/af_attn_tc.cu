@@ -94,22 +94,28 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-__device__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+// The CTA's abort flag and the limit of its pipeline waits (the model's
+// wait limit, 2 s by default; the drains after an abort keep kWaitLimitNs).
+struct Abort {
+  volatile int* flag;
+  uint64_t limit_ns;
+};
+__device__ bool mbar_wait(uint32_t bar, uint32_t parity, const Abort& ab) {
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try(bar, parity)) return true;
     if ((i & 63u) == 0u) {
-      if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        *abort_flag = 1;
+      if (*ab.flag) return false;
+      if (globaltimer_ns() - t0 > ab.limit_ns) {
+        *ab.flag = 1;
         return false;
       }
     }
   }
 }
-__device__ __forceinline__ bool wait_fast(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-  return mbar_try(bar, parity) || mbar_wait(bar, parity, abort_flag);
+__device__ __forceinline__ bool wait_fast(uint32_t bar, uint32_t parity, const Abort& ab) {
+  return mbar_try(bar, parity) || mbar_wait(bar, parity, ab);
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1) {
   asm volatile(
@@ -182,12 +188,27 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Which keys a query attends: token-causal (key <= query position) when F is
+// 0; otherwise by frames of F tokens -- every key of the query's frame and of
+// the `ahead` frames after it, never past the sequence (Lc positions).  The
+// last attended key is nondecreasing in the query position.
+struct KeyMask {
+  int F, ahead, Lc;
+  __host__ __device__ __forceinline__ int limit(int p) const {
+    if (F == 0) return p;
+    const int e = (p / F + 1 + ahead) * F;
+    return (e < Lc ? e : Lc) - 1;
+  }
+};
+
 struct AttnArgs {
   const Ctl* ctl;
   bf16* o;           // [Mmax, d] output (one split)
   float* opart;      // [nsplit_max, Mmax, d] unnormalised partial outputs (several splits)
   float* mlpart;     // [nsplit_max, Mmax, heads, 2] running max (log2 units) and row sum
   int Lc, d, heads, nsplit_max, m_max, batch, sms;
+  uint64_t wait_ns;  // limit of a pipeline wait before the CTA aborts
+  KeyMask km;        // which keys a query attends
 };
 
 // Key splits of a pass, decided from the rows the pass really has (ctl->R
@@ -202,10 +223,10 @@ constexpr int kMaxSplits = 32;
 constexpr int kMaxDevices = 64;
 struct SplitPlan { int q_tiles, nsplit, tps; };
 __host__ __device__ __forceinline__ SplitPlan split_plan(int R, int p0, int heads, int batch, int nsplit_max,
-                                                         int sms, int bkv) {
+                                                         int sms, int bkv, const KeyMask& km) {
   SplitPlan sp;
   sp.q_tiles = (R + BQ - 1) / BQ;
-  const int live = (p0 + R + bkv - 1) / bkv;               // key tiles up to the last key any row needs
+  const int live = km.limit(p0 + R - 1) / bkv + 1;        // key tiles up to the last key any row needs
   const int base = sp.q_tiles * heads * batch;
   int n = 1;
   if (nsplit_max > 1 && base < 2 * sms) {
@@ -232,6 +253,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   volatile int* abort_flag = &s_abort;
+  const Abort ab{abort_flag, g.wait_ns};
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // group of this warp: warps 0, 1 and 4-7 serve group 0; warps 2, 3 and 8-11 group 1
@@ -274,7 +296,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   pdl_wait();                                                 // q, the cache and the row layout come from upstream
   const Ctl* ctl = g.ctl;
   const int R = ctl->R, p0 = ctl->p0;
-  const SplitPlan plan = split_plan(R, p0, g.heads, g.batch, g.nsplit_max, g.sms, BKV);
+  const SplitPlan plan = split_plan(R, p0, g.heads, g.batch, g.nsplit_max, g.sms, BKV, g.km);
   const int q_tiles = plan.q_tiles, nsplit = plan.nsplit, tps = plan.tps;
   const int n_items = q_tiles * g.heads * g.batch * nsplit;
 
@@ -296,7 +318,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     x.s = r / nsplit;
     x.q_begin = x.qt * BQ - pad;
     const int q_end = x.q_begin + BQ;
-    const int ntiles = (p0 + q_end - 1) / BKV + 1;          // key tiles up to the last needed key
+    const int ntiles = g.km.limit(p0 + q_end - 1) / BKV + 1;   // key tiles up to the last needed key
     x.t0 = x.split * tps;
     x.nt = min(ntiles, x.t0 + tps) - x.t0;
     return x;
@@ -322,7 +344,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // diagonal its light quarters share a sub-partition with group 0's
         // heavy ones (a softmax warp serves TMEM lanes 32 (warp % 4) ..).
         const int qb = iw % QB;
-        if (iw >= QB && !mbar_wait(QE + 8 * qb, (uint32_t)(((iw / QB) - 1) & 1), abort_flag)) break;
+        if (iw >= QB && !mbar_wait(QE + 8 * qb, (uint32_t)(((iw / QB) - 1) & 1), ab)) break;
         mbar_expect_tx(QF + 8 * qb, Cfg::Q_BYTES);
 #pragma unroll
         for (int kc = 0; kc < Cfg::KCH; ++kc)
@@ -333,7 +355,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         ++nq;
         for (int j = 0; j < x.nt; ++j) {
           const int krow = x.s * g.Lc + (x.t0 + j) * BKV;
-          if (!mbar_wait(KE + 8 * kst, kph ^ 1u, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(KE + 8 * kst, kph ^ 1u, ab)) { ok = false; break; }
           mbar_expect_tx(KF + 8 * kst, Cfg::KV_BYTES);
 #pragma unroll
           for (int kc = 0; kc < Cfg::KCH; ++kc)
@@ -341,7 +363,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         krow);
           ++nk;
           if (++kst == SK) { kst = 0; kph ^= 1u; }
-          if (!mbar_wait(VE + 8 * vst, vph ^ 1u, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(VE + 8 * vst, vph ^ 1u, ab)) { ok = false; break; }
           mbar_expect_tx(VF + 8 * vst, Cfg::KV_BYTES);
 #pragma unroll
           for (int kc = 0; kc < Cfg::KCH; ++kc)
@@ -364,7 +386,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const uint32_t bar = full0 + 8u * (uint32_t)(idx % stages);
             const uint32_t ph = (uint32_t)((idx / stages) & 1);
             while (!mbar_try(bar, ph)) {
-              if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+              if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                atomicOr(err, ERR_DRAIN);
+                return;
+              }
             }
           }
         };
@@ -390,9 +415,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       auto issue_pv = [&]() -> bool {
         const int u = t - 1, pb = u % PB;
         // an item's first P*V overwrites O: the group has read the previous item's O
-        if (p_j == 0 && p_iw >= 1 && !wait_fast(OR, (uint32_t)((p_iw - 1) & 1), abort_flag)) return false;
-        if (!wait_fast(PF + 8 * pb, (uint32_t)((u / PB) & 1), abort_flag)) return false;
-        if (!wait_fast(VF + 8 * p_vst, (uint32_t)p_vph, abort_flag)) return false;
+        if (p_j == 0 && p_iw >= 1 && !wait_fast(OR, (uint32_t)((p_iw - 1) & 1), ab)) return false;
+        if (!wait_fast(PF + 8 * pb, (uint32_t)((u / PB) & 1), ab)) return false;
+        if (!wait_fast(VF + 8 * p_vst, (uint32_t)p_vph, ab)) return false;
         tc_fence_after();
         const uint64_t a0 = dp + (uint64_t)(pb * (Cfg::P_BYTES >> 4));
         const uint64_t b0 = dv + (uint64_t)(p_vst * (Cfg::KV_BYTES >> 4));
@@ -409,11 +434,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const Item x = item_of(it);
         if (x.nt <= 0) continue;
         const int qb = iw % QB;
-        if (!wait_fast(QF + 8 * qb, (uint32_t)((iw / QB) & 1), abort_flag)) { ok = false; break; }
+        if (!wait_fast(QF + 8 * qb, (uint32_t)((iw / QB) & 1), ab)) { ok = false; break; }
         const uint64_t aq = dq + (uint64_t)(qb * (Cfg::Q_BYTES >> 4));
         for (int j = 0; j < x.nt; ++j) {
-          if (!wait_fast(KF + 8 * kst, kph, abort_flag)) { ok = false; break; }
-          if (t >= 1 && !wait_fast(SR, (uint32_t)((t - 1) & 1), abort_flag)) { ok = false; break; }
+          if (!wait_fast(KF + 8 * kst, kph, ab)) { ok = false; break; }
+          if (t >= 1 && !wait_fast(SR, (uint32_t)((t - 1) & 1), ab)) { ok = false; break; }
           tc_fence_after();
           const uint64_t bk = dk + (uint64_t)(kst * (Cfg::KV_BYTES >> 4));
 #pragma unroll
@@ -443,7 +468,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       umma_commit(DRAIN);
       const uint64_t tw0 = globaltimer_ns();
       while (!mbar_try(DRAIN, 0)) {
-        if (globaltimer_ns() - tw0 > kWaitLimitNs) { atomicExch(err, ERR_ATTN_WAIT); break; }
+        if (globaltimer_ns() - tw0 > kWaitLimitNs) { atomicOr(err, ERR_DRAIN); break; }
       }
     }
   } else {
@@ -475,16 +500,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         continue;
       }
-      const int qpos = p0 + rloc;
+      // the last key of this row and the lowest / highest of the warp's rows
+      const int qpos = g.km.limit(p0 + rloc);
       const int wrow0 = x.q_begin + quarter * 32;             // the warp's first row
       const bool wvalid = wrow0 + 31 >= 0 && wrow0 < R;       // warp-uniform
-      const int qlo = p0 + max(wrow0, 0), qhi = p0 + min(wrow0 + 31, R - 1);
+      const int qlo = g.km.limit(p0 + max(wrow0, 0)), qhi = g.km.limit(p0 + min(wrow0 + 31, R - 1));
       float m_use = -INFINITY;
       float2 l2 = make_float2(0.f, 0.f);
       int j = 0;
       for (; j < x.nt; ++j) {
         // every wait's outcome is made warp-uniform before any .aligned TMEM access
-        if (!__all_sync(0xffffffffu, mbar_wait(SF, (uint32_t)(tw & 1), abort_flag))) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(SF, (uint32_t)(tw & 1), ab))) break;
         tc_fence_after();
         const int key0 = (x.t0 + j) * BKV;
         // the row's scores move to registers and S is released at once, so the
@@ -526,7 +552,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // P tile tw % PB is free once the group's P*V of tile tw - PB has completed
         const int pb = tw % PB;
         if (tw >= PB &&
-            !__all_sync(0xffffffffu, mbar_wait(OD + 8 * pb, (uint32_t)(((tw / PB) - 1) & 1), abort_flag)))
+            !__all_sync(0xffffffffu, mbar_wait(OD + 8 * pb, (uint32_t)(((tw / PB) - 1) & 1), ab)))
           break;
         uint8_t* prow = prow0 + pb * Cfg::P_BYTES;
         if (pb == stg_buf) {
@@ -568,7 +594,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           // the max grew: rescale O, which must hold tiles 0..j-1, before this
           // tile's P*V is issued
           const int tl = tw - 1;
-          if (!__all_sync(0xffffffffu, mbar_wait(OD + 8 * (tl % PB), (uint32_t)((tl / PB) & 1), abort_flag)))
+          if (!__all_sync(0xffffffffu, mbar_wait(OD + 8 * (tl % PB), (uint32_t)((tl / PB) & 1), ab)))
             break;
           tc_fence_after();
 #pragma unroll
@@ -598,7 +624,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const size_t mrow = (size_t)xe.s * R + rloc;
       const int tl = tw - 1;
       const bool ok = __all_sync(
-          0xffffffffu, (j == x.nt) && mbar_wait(OD + 8 * (tl % PB), (uint32_t)((tl / PB) & 1), abort_flag));
+          0xffffffffu, (j == x.nt) && mbar_wait(OD + 8 * (tl % PB), (uint32_t)((tl / PB) & 1), ab));
       tc_fence_after();
       const float lt = l2.x + l2.y;
       const bool valid = ok && rloc >= 0 && rloc < R;
@@ -684,7 +710,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
   }
-  if (threadIdx.x == 0 && s_abort) atomicExch(err, ERR_ATTN_WAIT);
+  if (threadIdx.x == 0 && s_abort) atomicOr(err, ERR_ATTN_WAIT);
 }
 
 // Merge the splits' partials: o = sum_i 2^(m_i - m) o_i / sum_i 2^(m_i - m) l_i.
@@ -694,7 +720,7 @@ __global__ void __launch_bounds__(256) k_attn_combine(AttnArgs g) {
   pdl_wait();
   const int wg = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int M = g.ctl->M;
-  const int nsplit = split_plan(g.ctl->R, g.ctl->p0, g.heads, g.batch, g.nsplit_max, g.sms, AttnCfg<HD>::BKV).nsplit;
+  const int nsplit = split_plan(g.ctl->R, g.ctl->p0, g.heads, g.batch, g.nsplit_max, g.sms, AttnCfg<HD>::BKV, g.km).nsplit;
   if (nsplit == 1 || wg >= M * g.heads) return;      // one split: the attention kernel wrote o itself
   const int row = wg / g.heads, hh = wg - row * g.heads;
   float mx = -INFINITY;
@@ -759,7 +785,7 @@ int attn_tc_splits(int batch, int heads, int r_max, int Lc, int num_sms) {
 
 bool launch_attn_tc2(const Ctl* ctl, const bf16* q, const bf16* kc, const bf16* vc, bf16* o, float* opart,
                      float* mlpart, int nsplit_max, int batch, int Lc, int d, int heads, int r_max, int m_max,
-                     int num_sms, int* err, cudaStream_t st) {
+                     int num_sms, uint64_t wait_ns, int mask_frame, int mask_ahead, int* err, cudaStream_t st) {
   const int hd = d / heads;
   const int bkv = hd == 64 ? AttnCfg<64>::BKV : AttnCfg<128>::BKV;
   CUtensorMap tq, tk, tv, to;
@@ -778,6 +804,10 @@ bool launch_attn_tc2(const Ctl* ctl, const bf16* q, const bf16* kc, const bf16* 
   g.m_max = m_max;
   g.batch = batch;
   g.sms = num_sms;
+  g.wait_ns = wait_ns;
+  g.km.F = mask_frame;
+  g.km.ahead = mask_ahead;
+  g.km.Lc = Lc;
   return hd == 64 ? launch_hd<64>(tq, tk, tv, to, g, batch, r_max, err, st)
                   : launch_hd<128>(tq, tk, tv, to, g, batch, r_max, err, st);
 }

@@ -43,8 +43,10 @@ enum : int { BT_NB = 0, BT_BEGIN = 1, BT_END = 2, BT_STARTS = 4 };
 // position of block i (i = 0 .. nb; the last entry is L).
 __host__ __device__ inline size_t btab_ints(int L) { return (size_t)BT_STARTS + (size_t)L + 1; }
 
-// Error codes written to the model's device error word.
-enum : int { ERR_NONE = 0, ERR_GEMM_WAIT = 1, ERR_GEMM_DRAIN = 2, ERR_ATTN_WAIT = 3 };
+// Bits OR-ed into the model's device error word: a pipeline wait that ran
+// past the limit in a GEMM or in attention, and a drain after an abort that
+// did not see its in-flight loads or MMAs complete within its own bound.
+enum : int { ERR_NONE = 0, ERR_GEMM_WAIT = 1, ERR_DRAIN = 2, ERR_ATTN_WAIT = 4 };
 
 enum Epi : int {
   EPI_INPROJ = 0,   // h = acc + b_in + pos(p)                          (fp32 h)
@@ -71,12 +73,14 @@ struct EpiArgs {
   const float* pos_time;   // [max_frames, d]
   int frame_len;
   // head
-  int head_mode;           // 0 forward (z, logdet partials), 1 Jacobi update
+  int head_mode;           // 0 forward (z, logdet partials), 1 Jacobi update, 2 denoise (x + sigma * s)
+  float sigma;             // head_mode 2: the noise level
   int L, C, dir;
   const float* xin_f;      // forward: x (read)          inverse: z (read)
   float* xout_f;           // forward: z (write)         inverse: x (read + write)
   const int* active;       // inverse: per-sample flag
   float* part;             // [Mmax, 2C/16, 2] per-(row, 16-column group) partial sums
+  uint64_t wait_ns;        // tensor-core kernels: limit of a pipeline wait before the CTA aborts
 };
 
 __device__ __forceinline__ int tok_of(int p, int L, int dir) { return dir ? (L - 1 - p) : p; }
@@ -114,6 +118,13 @@ __device__ __forceinline__ void head_group(const EpiArgs& e, int row, int col0, 
   const int R = ctl->R;
   const int s = row / R;
   const int p = ctl->p0 + (row - s * R);
+  if (e.head_mode == 2) {
+    // denoiser: 16 plain channels, out = x_noisy + sigma * (acc + b)
+    const size_t base = ((size_t)s * e.L + p) * e.C + col0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) e.xout_f[base + j] = fmaf(e.sigma, v[j] + e.bias[col0 + j], e.xin_f[base + j]);
+    return;
+  }
   if (p < ctl->P) return;                       // commit rows give no output
   const int tok = tok_of(p, e.L, e.dir);
   const int c0 = col0 >> 1;

@@ -94,17 +94,23 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// The CTA's abort flag and the limit of its pipeline waits (the model's
+// wait limit, 2 s by default; the drains after an abort keep kWaitLimitNs).
+struct Abort {
+  volatile int* flag;
+  uint64_t limit_ns;
+};
 // Wait for the phase of `bar` with parity `parity`; false once the CTA has
-// aborted or 2 s have passed (which aborts the CTA).
-__device__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+// aborted or the wait limit has passed (which aborts the CTA).
+__device__ bool mbar_wait(uint32_t bar, uint32_t parity, const Abort& ab) {
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try(bar, parity)) return true;
     if ((i & 63u) == 0u) {
-      if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        *abort_flag = 1;
+      if (*ab.flag) return false;
+      if (globaltimer_ns() - t0 > ab.limit_ns) {
+        *ab.flag = 1;
         return false;
       }
     }
@@ -263,6 +269,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   volatile int* abort_flag = &s_abort;
+  const Abort ab{abort_flag, e.wait_ns};
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_trigger();
@@ -330,7 +337,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
         const int brow = nb * BN + (int)rank * (BN / CG);
         bool ok = true;
         for (int kb = 0; kb < kbn; ++kb) {
-          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, ab)) { ok = false; break; }
           if (rank == 0) mbar_expect_tx(full0 + 8 * stage, CG * Cfg::STAGE_BYTES);
           if (CG == 2) {
             tma_load_2d_pair(smem_u32(sA + stage * Cfg::A_BYTES), &tmA, full_lead + 8 * stage, kb * BK, arow);
@@ -344,8 +351,10 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
         }
         if (!ok) break;
       }
-      if (CG == 1) {
+      if (CG == 1 || rank == 0) {
         // drain: the last load of every stage has landed before the CTA exits
+        // (on an SM pair the leader's full barriers count the bytes of both
+        // CTAs' loads of the stages it armed)
         const long long n = issued < S ? issued : S;
         for (long long j = 1; j <= n; ++j) {
           const long long idx = issued - j;
@@ -353,11 +362,15 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
           const uint32_t ph = (uint32_t)((idx / S) & 1);
           const uint64_t t0 = globaltimer_ns();
           while (!mbar_try(full0 + 8 * st, ph)) {
-            if (globaltimer_ns() - t0 > kWaitLimitNs) { atomicExch(err, ERR_GEMM_DRAIN); break; }
+            if (globaltimer_ns() - t0 > kWaitLimitNs) { atomicOr(err, ERR_DRAIN); break; }
           }
         }
-      } else if (*abort_flag) {
-        // the pair's completion counts live on the leader; give in-flight copies time to land
+      }
+      if (CG == 2 && rank != 0 && *abort_flag) {
+        // The second CTA's loads complete on the leader's barriers, which this
+        // CTA cannot wait on; after an abort it gives them 2 ms to land (a load
+        // takes microseconds), and the pair leaves together (cluster barrier
+        // at the end) once the leader has drained.
         const uint64_t t0 = globaltimer_ns();
         while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);
       }
@@ -371,12 +384,12 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
       for (int t = unit; t < ntiles; t += nunits, ++i) {
         const int acc = i & 1;
         const uint32_t use = (uint32_t)(i >> 1);
-        if (!mbar_wait(tempty0 + 8 * acc, (use & 1u) ^ 1u, abort_flag)) break;
+        if (!mbar_wait(tempty0 + 8 * acc, (use & 1u) ^ 1u, ab)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
         bool ok = true;
         for (int kb = 0; kb < kbn; ++kb) {
-          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(full0 + 8 * stage, phase, ab)) { ok = false; break; }
           tc_fence_after();
           const uint64_t da = sw128_desc(smem_u32(sA + stage * Cfg::A_BYTES));
           const uint64_t db = sw128_desc(smem_u32(sB + stage * Cfg::B_BYTES));
@@ -398,7 +411,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
       else umma_commit(drain);
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try(drain, 0)) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) { atomicExch(err, ERR_GEMM_DRAIN); break; }
+        if (globaltimer_ns() - t0 > kWaitLimitNs) { atomicOr(err, ERR_DRAIN); break; }
       }
     }
   } else if (warp >= 4) {
@@ -448,7 +461,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) bnext[jj] = reinterpret_cast<const float4*>(e.bias + n0)[jj];
         // the wait's outcome is made warp-uniform before the .aligned TMEM loads
-        if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * acc, use & 1u, abort_flag))) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * acc, use & 1u, ab))) break;
         tc_fence_after();
         float vb[2][16];
         tmem_ld16(taddr, vb[0]);
@@ -581,7 +594,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
           hin = e.xin_f + base;
           hout = e.xout_f + base;
           hpart = e.part + (size_t)r * ((2 * e.C) >> 4) * 2;
-          head_act = head_out && (e.head_mode == 0 || e.active[sm]);
+          head_act = head_out && (e.head_mode != 1 || e.active[sm]);
         }
         // Loads that do not depend on the accumulator are issued before waiting
         // for it (bias, and the first chunk's position / x rows), and every
@@ -594,7 +607,11 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
         float4 pre[2][4], pre2[2][4];
         auto load_rows = [&](int k, float4* dst, float4* dst2) {
           if (EPI == EPI_HEAD) {
-            if (head_act) {
+            if (head_act && e.head_mode == 2) {             // denoiser: 16 plain channels
+              const float4* src = reinterpret_cast<const float4*>(hin + n0 + k * 16);
+#pragma unroll
+              for (int qq = 0; qq < 4; ++qq) dst[qq] = src[qq];
+            } else if (head_act) {
               const int c0 = (n0 + k * 16) >> 1;
               dst[0] = *reinterpret_cast<const float4*>(hin + c0);
               dst[1] = *reinterpret_cast<const float4*>(hin + c0 + 4);
@@ -616,7 +633,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
         };
         load_rows(0, pre[0], pre2[0]);
         // the wait's outcome is made warp-uniform before the .aligned TMEM loads
-        if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * acc, use & 1u, abort_flag))) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * acc, use & 1u, ab))) break;
         tc_fence_after();
         float vb[2][16];
         tmem_ld16(taddr, vb[0]);
@@ -629,6 +646,20 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
             load_rows(k + 1, pre[(k + 1) & 1], pre2[(k + 1) & 1]);
           }
           const float* v = vb[k & 1];
+          if (EPI == EPI_HEAD && e.head_mode == 2) {
+            // denoiser: x = x_noisy + sigma * (s_phi + b) for 16 plain channels
+            if (!head_out) continue;
+            const int col0 = n0 + c;
+            const float4* xn4 = pre[k & 1];
+            float4* o4 = reinterpret_cast<float4*>(hout + col0);
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+              const float4 bb = *reinterpret_cast<const float4*>(e.bias + col0 + 4 * qq);
+              o4[qq] = make_float4(fmaf(e.sigma, v[4 * qq] + bb.x, xn4[qq].x), fmaf(e.sigma, v[4 * qq + 1] + bb.y, xn4[qq].y),
+                                   fmaf(e.sigma, v[4 * qq + 2] + bb.z, xn4[qq].z), fmaf(e.sigma, v[4 * qq + 3] + bb.w, xn4[qq].w));
+            }
+            continue;
+          }
           if (EPI == EPI_HEAD) {
             // 8 channels whose (mu_c, s_c) sit at columns (2c, 2c+1)
             const int col0 = n0 + c;
@@ -692,7 +723,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
     if (CG == 2) asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
     else asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
   }
-  if (threadIdx.x == 0 && s_abort) atomicExch(err, ERR_GEMM_WAIT);
+  if (threadIdx.x == 0 && s_abort) atomicOr(err, ERR_GEMM_WAIT);
 }
 
 template <int BN, int EPI, int CG>

@@ -246,9 +246,10 @@ __global__ void k_set_pass(Ctl* ctl, int p0, int R, int batch, bf16* vtail, size
 // ------------------------------------------------------------------ row-wise
 
 // Self-exclusive mask as a one-token shift: the input of position p is
-// x_{p-1} (zero at p = 0), read through the direction flip.
+// x_{p-1} (zero at p = 0), read through the direction flip; without the shift
+// (the denoiser) the input of p is x_p.
 template <typename T>
-__global__ void k_gather(const Ctl* ctl, const float* __restrict__ x, int L, int C, int dir, T* xin) {
+__global__ void k_gather(const Ctl* ctl, const float* __restrict__ x, int L, int C, int dir, int shift, T* xin) {
   pdl_trigger();
   pdl_wait();
   const int M = ctl->M, R = ctl->R, p0 = ctl->p0;
@@ -261,7 +262,7 @@ __global__ void k_gather(const Ctl* ctl, const float* __restrict__ x, int L, int
     const int s = row / R;
     const int p = p0 + (row - s * R);
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (p > 0) v = *reinterpret_cast<const float4*>(x + ((size_t)s * L + tok_of(p - 1, L, dir)) * C + c);
+    if (p >= shift) v = *reinterpret_cast<const float4*>(x + ((size_t)s * L + tok_of(p - shift, L, dir)) * C + c);
     store4(xin + (size_t)row * C + c, v.x, v.y, v.z, v.w);
   }
 }
@@ -423,7 +424,7 @@ __global__ void k_head_simt(const float* __restrict__ A, const float* __restrict
 template <int HD>
 __global__ void __launch_bounds__(256) k_attn_simt(const Ctl* ctl, const float* __restrict__ q,
                                                    const float* __restrict__ kc, const float* __restrict__ vc,
-                                                   float* o, int Lc, int d, int heads) {
+                                                   float* o, int Lc, int d, int heads, int mF, int ahead) {
   pdl_trigger();
   pdl_wait();
   __shared__ float qs[8][HD];
@@ -441,7 +442,9 @@ __global__ void __launch_bounds__(256) k_attn_simt(const Ctl* ctl, const float* 
   float m = -INFINITY, l = 0.f, acc[HD];
 #pragma unroll
   for (int i = 0; i < HD; ++i) acc[i] = 0.f;
-  for (int j = lane; j <= p; j += 32) {
+  int last = p;                                         // the row's last key (mask, see af_kernels.h)
+  if (mF) last = min((p / mF + 1 + ahead) * mF, Lc) - 1;
+  for (int j = lane; j <= last; j += 32) {
     float sc = 0.f;
 #pragma unroll
     for (int i = 0; i < HD; ++i) sc = fmaf(qs[wib][i], K[(size_t)j * d + i], sc);
@@ -495,12 +498,13 @@ void launch_set_pass(Ctl* ctl, int p0, int R, int batch, bf16* vtail, size_t kv_
 }
 
 template <typename T>
-void launch_gather(const Ctl* ctl, const float* x, int L, int C, int dir, T* xin, int m_max,
+void launch_gather(const Ctl* ctl, const float* x, int L, int C, int dir, int shift, T* xin, int m_max,
                    cudaStream_t st) {
-  launch_k(k_gather<T>, dim3(grid_for((long long)m_max * (C / 4), kThreads)), dim3(kThreads), 0, st, ctl, x, L, C, dir, xin);
+  launch_k(k_gather<T>, dim3(grid_for((long long)m_max * (C / 4), kThreads)), dim3(kThreads), 0, st, ctl, x, L, C, dir,
+           shift, xin);
 }
-template void launch_gather<float>(const Ctl*, const float*, int, int, int, float*, int, cudaStream_t);
-template void launch_gather<bf16>(const Ctl*, const float*, int, int, int, bf16*, int, cudaStream_t);
+template void launch_gather<float>(const Ctl*, const float*, int, int, int, int, float*, int, cudaStream_t);
+template void launch_gather<bf16>(const Ctl*, const float*, int, int, int, int, bf16*, int, cudaStream_t);
 
 template <typename T>
 void launch_layernorm(const Ctl* ctl, const float* h, const float* g, const float* b, T* out, int d,
@@ -560,14 +564,15 @@ void launch_head_simt(const float* A, const float* W, int N, int K, int m_max, c
 }
 
 void launch_attn_simt(const Ctl* ctl, const float* q, const float* kc, const float* vc, float* o, int batch,
-                      int Lc, int d, int heads, int m_max, cudaStream_t st) {
+                      int Lc, int d, int heads, int m_max, int mask_frame, int mask_ahead, cudaStream_t st) {
   (void)batch;
   const int grid = (int)(((long long)m_max * heads + 7) / 8);
+  const int F = mask_frame, A = mask_ahead;
   switch (d / heads) {
-    case 16: launch_k(k_attn_simt<16>, dim3(grid), dim3(256), 0, st, ctl, q, kc, vc, o, Lc, d, heads); break;
-    case 32: launch_k(k_attn_simt<32>, dim3(grid), dim3(256), 0, st, ctl, q, kc, vc, o, Lc, d, heads); break;
-    case 64: launch_k(k_attn_simt<64>, dim3(grid), dim3(256), 0, st, ctl, q, kc, vc, o, Lc, d, heads); break;
-    default: launch_k(k_attn_simt<128>, dim3(grid), dim3(256), 0, st, ctl, q, kc, vc, o, Lc, d, heads); break;
+    case 16: launch_k(k_attn_simt<16>, dim3(grid), dim3(256), 0, st, ctl, q, kc, vc, o, Lc, d, heads, F, A); break;
+    case 32: launch_k(k_attn_simt<32>, dim3(grid), dim3(256), 0, st, ctl, q, kc, vc, o, Lc, d, heads, F, A); break;
+    case 64: launch_k(k_attn_simt<64>, dim3(grid), dim3(256), 0, st, ctl, q, kc, vc, o, Lc, d, heads, F, A); break;
+    default: launch_k(k_attn_simt<128>, dim3(grid), dim3(256), 0, st, ctl, q, kc, vc, o, Lc, d, heads, F, A); break;
   }
 }
 

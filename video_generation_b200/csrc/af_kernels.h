@@ -34,8 +34,10 @@ inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_
 // All row-wise kernels read the live row count from ctl->M and are launched
 // for `m_max` rows.
 void launch_ctl_forward(Ctl* ctl, int batch, int L, cudaStream_t st);
+// shift = 1: the input of position p is x_{p-1} (zero at p = 0), the
+// self-exclusive mask of an AF block; shift = 0: x_p itself (the denoiser).
 template <typename T>
-void launch_gather(const Ctl* ctl, const float* x, int L, int C, int dir, T* xin, int m_max,
+void launch_gather(const Ctl* ctl, const float* x, int L, int C, int dir, int shift, T* xin, int m_max,
                    cudaStream_t st);
 template <typename T>
 void launch_layernorm(const Ctl* ctl, const float* h, const float* g, const float* b, T* out,
@@ -67,8 +69,11 @@ void launch_gemm_simt(int epi, const float* A, const float* W, int N, int K, int
                       const EpiArgs& e, cudaStream_t st);
 void launch_head_simt(const float* A, const float* W, int N, int K, int m_max, const EpiArgs& e,
                       cudaStream_t st);
+// Attention masks (both paths): token-causal when mask_frame is 0, else by
+// frames of mask_frame tokens with mask_ahead frames of look-ahead.
 void launch_attn_simt(const Ctl* ctl, const float* q, const float* kc, const float* vc, float* o,
-                      int batch, int Lc, int d, int heads, int m_max, cudaStream_t st);
+                      int batch, int Lc, int d, int heads, int m_max, int mask_frame, int mask_ahead,
+                      cudaStream_t st);
 
 // ---- tensor-core bf16 path ---------------------------------------------------
 // TMA descriptor of a row-major bf16 matrix [rows, cols] tiled as boxes of
@@ -95,6 +100,6 @@ int gemm_tc_pick(int N, int m_max, int num_sms, int unit, int max_bn);
 int attn_tc_splits(int batch, int heads, int r_max, int Lc, int num_sms);
 bool launch_attn_tc2(const Ctl* ctl, const bf16* q, const bf16* kc, const bf16* vc, bf16* o, float* opart,
                      float* mlpart, int nsplit_max, int batch, int Lc, int d, int heads, int r_max, int m_max,
-                     int num_sms, int* err, cudaStream_t st);
+                     int num_sms, uint64_t wait_ns, int mask_frame, int mask_ahead, int* err, cudaStream_t st);
 
 }  // namespace af

@@ -28,7 +28,8 @@ EXPORTS = ("af_num_tensors", "af_model_create", "af_model_destroy", "af_workspac
            "af_inverse_jacobi", "flow_stack_forward", "flow_stack_inverse", "af_last_convergence",
            "af_device_error", "af_status_string", "af_last_error_string", "af_forward_noalloc",
            "af_inverse_jacobi_schedule", "af_prefix_encode", "flow_pipeline_workspace_bytes",
-           "flow_pipeline_inverse")
+           "flow_pipeline_inverse", "af_set_wait_limit", "af_denoiser_num_tensors", "af_denoiser_create",
+           "af_denoise", "af_stream_workspace_bytes", "af_inverse_jacobi_stream")
 
 
 class AFConfigC(ctypes.Structure):
@@ -56,6 +57,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.af_forward_noalloc.argtypes = [vp, vp, i, i, i, vp, vp, vp]
     lib.af_inverse_jacobi_schedule.argtypes = [vp, vp, i, i, i, P(i), i, i, i, f, i, i, vp, vp, vp, sz, vp]
     lib.af_prefix_encode.argtypes = [vp, vp, i, i, i, i, i, vp, sz, vp]
+    lib.af_set_wait_limit.argtypes = [vp, ctypes.c_double]
+    lib.af_denoiser_num_tensors.argtypes = [P(AFConfigC)]
+    lib.af_denoiser_num_tensors.restype = i
+    lib.af_denoiser_create.argtypes = [P(AFConfigC), P(vp), i, P(vp)]
+    lib.af_denoise.argtypes = [vp, vp, i, i, f, vp, vp, sz, vp]
+    lib.af_stream_workspace_bytes.argtypes = [vp, i, i]
+    lib.af_stream_workspace_bytes.restype = sz
+    lib.af_inverse_jacobi_stream.argtypes = [vp, vp, i, i, i, i, f, i, i, vp, vp, vp, sz, vp]
     lib.flow_pipeline_workspace_bytes.argtypes = [vp, i, i, i]
     lib.flow_pipeline_workspace_bytes.restype = sz
     lib.flow_pipeline_inverse.argtypes = [vp, P(vp), P(i), i, vp, i, i, i, f, i, i, i, vp, vp, vp, vp, sz, vp, sz,
@@ -68,7 +77,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.af_last_error_string.restype = ctypes.c_char_p
     for name in EXPORTS:
         if name not in ("af_status_string", "af_last_error_string", "af_num_tensors", "af_workspace_bytes",
-                        "flow_pipeline_workspace_bytes"):
+                        "flow_pipeline_workspace_bytes", "af_denoiser_num_tensors", "af_stream_workspace_bytes"):
             getattr(lib, name).restype = i
     return lib
 
@@ -106,16 +115,18 @@ def _stream(stream=None):
 
 
 class AFModel:
-    """One AF block's weights on the current CUDA device (owned by libaf)."""
+    """One AF block's weights (or, with denoiser=True, the denoiser's) on the
+    current CUDA device (owned by libaf)."""
 
-    def __init__(self, shape, tensors: Sequence[np.ndarray]):
+    def __init__(self, shape, tensors: Sequence[np.ndarray], denoiser: bool = False):
         self.shape = shape
         self.cfg = AFConfigC(shape.C, shape.d, shape.heads, shape.layers, shape.mlp_ratio, shape.frame_len,
                              shape.max_frames, BF16 if shape.dtype == "bf16" else FP32)
         arrs = [np.ascontiguousarray(t, dtype=np.float32) for t in tensors]
         ptrs = (ctypes.c_void_p * len(arrs))(*[a.ctypes.data for a in arrs])
         h = ctypes.c_void_p()
-        _check(lib().af_model_create(ctypes.byref(self.cfg), ptrs, len(arrs), ctypes.byref(h)), "af_model_create")
+        create = lib().af_denoiser_create if denoiser else lib().af_model_create
+        _check(create(ctypes.byref(self.cfg), ptrs, len(arrs), ctypes.byref(h)), "model create")
         self.handle = h
 
     def close(self):
@@ -137,6 +148,10 @@ class AFModel:
         if n == 0:
             raise AFError(AF_ERR_ARG, "af_workspace_bytes")
         return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+    def set_wait_limit(self, seconds: float):
+        """Limit of one pipeline wait in the tensor-core kernels (default 2 s)."""
+        _check(lib().af_set_wait_limit(self.handle, float(seconds)), "af_set_wait_limit")
 
     def device_error(self) -> int:
         code = ctypes.c_int(0)
@@ -262,3 +277,35 @@ def flow_pipeline_inverse(deep: AFModel, shallow: List[AFModel], shallow_dirs: S
                                        _ptr(iters_shallow), _ptr(ws_deep), ws_deep.numel(), _ptr(ws_shallow),
                                        ws_shallow.numel(), _stream(stream), _stream(s2)), "flow_pipeline_inverse")
     return x, iters_deep, iters_shallow
+
+
+def af_denoise(model: AFModel, x_noisy: torch.Tensor, sigma: float, ws: torch.Tensor | None = None,
+               x: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """x = x_noisy + sigma * s_phi(x_noisy) with the denoiser `model` (created with denoiser=True)."""
+    batch, L, _ = x_noisy.shape
+    ws = model.workspace(batch, L, device=x_noisy.device) if ws is None else ws
+    x = torch.empty_like(x_noisy) if x is None else x
+    _check(lib().af_denoise(model.handle, _ptr(x_noisy), batch, L, float(sigma), _ptr(x), _ptr(ws), ws.numel(),
+                            _stream(stream)), "af_denoise")
+    return x
+
+
+def af_inverse_jacobi_stream(model: AFModel, z: torch.Tensor, window: int, overlap: int, tau: float, max_iter: int,
+                             warm_start: bool, ws: torch.Tensor | None = None, x: torch.Tensor | None = None,
+                             iters: torch.Tensor | None = None, stream=None):
+    """Streaming block-Jacobi inverse in windows of `window` frames overlapping by `overlap`;
+    returns (x, iters [batch, n_frames])."""
+    batch, L, _ = z.shape
+    F = model.shape.frame_len
+    n_frames = L // F
+    if ws is None:
+        n = int(lib().af_stream_workspace_bytes(model.handle, batch, window))
+        if n == 0:
+            raise AFError(AF_ERR_ARG, "af_stream_workspace_bytes")
+        ws = torch.empty(n, dtype=torch.uint8, device=z.device)
+    x = torch.empty_like(z) if x is None else x
+    iters = torch.zeros((batch, n_frames), dtype=torch.int32, device=z.device) if iters is None else iters
+    _check(lib().af_inverse_jacobi_stream(model.handle, _ptr(z), batch, n_frames, window, overlap, float(tau),
+                                          int(max_iter), int(bool(warm_start)), _ptr(x), _ptr(iters), _ptr(ws),
+                                          ws.numel(), _stream(stream)), "af_inverse_jacobi_stream")
+    return x, iters
