@@ -356,6 +356,96 @@ def measure(w, args, rank, world, dist, dev, with_e2e=True):
     return r
 
 
+def time_calls(fn, warmup, steps, st):
+    """Mean device time (s) of `steps` calls of fn after `warmup` calls, CUDA events on `st`."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        fn()
+    e1.record(st)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / 1e3 / steps
+
+
+def deep_flow_extras(args, dev, peaks):
+    """The deep flow (config 4) in the shapes the pages discuss: a sweep of the
+    Jacobi block size and the asymmetric schedule (small blocks for the first
+    frame, large after it; the pages' key findings), pipelined deep -> shallow
+    decoding of the 5 s clip against its parts (key design 3), and the
+    flow-score-matching denoiser over the clip (key design 2)."""
+    import torch
+    from video_generation_b200 import flow
+    st = torch.cuda.current_stream()
+    w4, w3 = syn.WORKLOADS[4], syn.WORKLOADS[3]
+    deep = flow.AFModel(w4.shape, syn.make_weights(w4.shape))
+    z = torch.from_numpy(syn.workload_latents(w4, "z")).to(dev)
+    out = {}
+    # block-size sweep (uniform blocks) and the asymmetric schedule
+    sweep = {}
+    F = w4.shape.frame_len
+    schedules = {f"B{b}": [b] * (w4.L // b) for b in (130, 195, 390, 780, 1170)}
+    schedules["first_frame_65_then_780"] = [65] * (F // 65) + [780] * ((w4.L - F) // 780)
+    for name, sizes in schedules.items():
+        assert sum(sizes) == w4.L
+        ws = deep.workspace(1, w4.L, max(sizes), device=dev)
+        x = torch.empty_like(z)
+        it = torch.zeros((1, len(sizes)), dtype=torch.int32, device=dev)
+        run = lambda: flow.af_inverse_jacobi_schedule(deep, z, 0, sizes, w4.tau, w4.max_iter, True, ws=ws, x=x, iters=it)
+        t = time_calls(run, 3, 2, st)
+        itn = it.cpu().numpy()
+        fl = 0.0
+        starts = np.concatenate([[0], np.cumsum(sizes)])
+        for b, k in enumerate(itn[0]):
+            f1 = FL.pass_flops(w4.shape.d, w4.shape.C, w4.shape.layers, w4.shape.mlp_ratio, sizes[b],
+                               FL.causal_pairs(int(starts[b]), sizes[b]))
+            fl += float(k) * f1 + (f1 if b + 1 < len(sizes) else 0.0)
+        sweep[name] = {"ms": 1e3 * t, "tokens_per_s": w4.L / t, "tflops": fl / t / 1e12,
+                       "mean_iters": float(itn.mean()), "blocks": len(sizes)}
+        del ws
+    out["fd_5s_block_size_sweep"] = sweep
+    # pipelined decoding: f_D^{-1} then f_S^{-1} of each frame as it finishes
+    shallow = [flow.AFModel(w3.shape, syn.make_weights(w3.shape, block=t)) for t in range(w3.T)]
+    ws_d = deep.workspace(1, w4.L, w4.B, device=dev)
+    ws_s = flow.pipeline_workspace(shallow, 1, F, device=dev)
+    s2 = torch.cuda.Stream(device=dev)
+    xp = torch.empty_like(z)
+    pipe = lambda: flow.flow_pipeline_inverse(deep, shallow, w3.dirs, z, w4.B, w4.tau, w4.max_iter, w3.max_iter, True,
+                                              ws_deep=ws_d, ws_shallow=ws_s, x=xp, stream_shallow=s2)
+    t_pipe = time_calls(pipe, 3, 2, st)
+    u = torch.empty_like(z)
+    deep_only = lambda: flow.af_inverse_jacobi(deep, z, 0, w4.B, w4.tau, w4.max_iter, True, ws=ws_d, x=u)
+    t_deep = time_calls(deep_only, 3, 2, st)
+    frames = u.view(w4.L // F, F, w4.shape.C)
+    ws_b = shallow[0].workspace(w4.L // F, F, F, device=dev)
+    xs = torch.empty_like(frames)
+    shallow_batched = lambda: flow.flow_stack_inverse(shallow, w3.dirs, frames, F, w3.tau, w3.max_iter, False,
+                                                      ws=ws_b, x=xs)
+    t_sh = time_calls(shallow_batched, 3, 3, st)
+    out["pipelined_decode_5s"] = {"ms": 1e3 * t_pipe, "deep_alone_ms": 1e3 * t_deep,
+                                  "shallow_21_frames_batched_ms": 1e3 * t_sh,
+                                  "sequential_sum_ms": 1e3 * (t_deep + t_sh),
+                                  "tokens_per_s": w4.L / t_pipe}
+    for m in shallow:
+        m.close()
+    deep.close()
+    # the denoiser over the 5 s clip
+    den = flow.AFModel(syn.DENOISER, syn.make_denoiser_weights(syn.DENOISER), denoiser=True)
+    L = 21 * syn.DENOISER.frame_len
+    xn = torch.from_numpy(syn.make_latents(1, L, syn.DENOISER.C, 83)).to(dev)
+    ws_n = den.workspace(1, L, device=dev)
+    xo = torch.empty_like(xn)
+    t_den = time_calls(lambda: flow.af_denoise(den, xn, 0.1, ws=ws_n, x=xo), 3, 5, st)
+    fl = FL.denoiser_flops(syn.DENOISER, 1, L)
+    out["denoiser_5s"] = {"ms": 1e3 * t_den, "tokens_per_s": L / t_den, "tflops": fl / t_den / 1e12,
+                          "frac_of_bf16_peak": fl / t_den / 1e12 / peaks["bf16_tflops"]}
+    den.close()
+    return out
+
+
 def extra_line(w, args, dev, peaks):
     """One more workload on this GPU (single process), as a dict for the `extra` key."""
     r = measure(w, args, 0, 1, None, dev, with_e2e=False)
@@ -430,12 +520,31 @@ def main():
     if world == 1 and rank == 0:
         if not args.no_extras and args.config == 3:
             ex_args = argparse.Namespace(**vars(args))
+            fd_inv_flops = None
             for cid, steps in ((2, max(3, min(args.steps, 20))), (4, 2), (5, 1)):
                 ex_args.steps = steps
                 try:
-                    extras[syn.WORKLOADS[cid].name], _ = extra_line(syn.WORKLOADS[cid], ex_args, dev, peaks)
+                    extras[syn.WORKLOADS[cid].name], rr = extra_line(syn.WORKLOADS[cid], ex_args, dev, peaks)
+                    if cid == 5:
+                        fd_inv_flops = rr["inv_flops_rank"] / steps
                 except Exception as e:          # an extra must not lose the headline line
                     extras[syn.WORKLOADS[cid].name] = {"error": repr(e)[:200]}
+            try:
+                extras.update(deep_flow_extras(ex_args, dev, peaks))
+            except Exception as e:
+                extras["deep_flow_extras"] = {"error": repr(e)[:200]}
+            if fd_inv_flops and not args.no_cpu_baseline:
+                # the oracle's flop rate on the deep flow's first frame, and the
+                # 30 s inverse's time extrapolated from it (labelled as such)
+                w5 = syn.WORKLOADS[5]
+                tok1, _, ti1, thr1, fl1 = run_oracle_sample(w5, 1)
+                t_full = fd_inv_flops / (fl1 / ti1)
+                extras[w5.name]["cpu_baseline"] = {
+                    "kind": "oracle", "cores": thr1, "first_frame_inverse_s": ti1,
+                    "extrapolated_full_inverse_s": t_full, "extrapolated_tokens_per_s": w5.L / t_full,
+                    "sample": "the first frame (390 tokens, 24 layers) of the deep flow, Jacobi inverse",
+                    "extrapolation": "the 30 s inverse's algorithmic flops (from the GPU run's iteration counts) "
+                                     "over the oracle's measured flop rate on that frame"}
         if not args.no_cpu_baseline:
             cpu = cpu_baselines(w, args, r["inv_flops_rank"] / args.steps, r["tokens_per_step_rank"])
 

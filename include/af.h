@@ -226,8 +226,9 @@ af_status flow_pipeline_inverse(const af_model* deep, const af_model* const* sha
  * frame_len tokens -- in the first layer a token of frame n attends every
  * token of frames <= n + 1, in later layers frames <= n -- so frame n's
  * output depends on frames <= n + 1 exactly; final LayerNorm and head give
- * s_phi.  AF_BF16 / AF_FP32 as for the AF block.  The model can only be used
- * with af_denoise (the flow calls reject it). */
+ * s_phi.  AF_BF16 / AF_FP32 as for the AF block; an AF_BF16 denoiser also
+ * needs C % 128 == 0 or C % 192 == 0 (its head has C outputs).  The model
+ * can only be used with af_denoise (the flow calls reject it). */
 int af_denoiser_num_tensors(const af_config* cfg);
 af_status af_denoiser_create(const af_config* cfg, const float* const* tensors, int n_tensors,
                              af_model** out);

@@ -19,7 +19,7 @@ pytestmark = pytest.mark.gpu
 
 TOL32, BF_X_TOL, BF_PART_TOL = 1e-5, 2e-2, 3e-2
 FP32 = syn.ModelShape(C=16, d=64, heads=2, layers=3, mlp_ratio=4, frame_len=16, max_frames=4, dtype="fp32")
-BF16 = syn.ModelShape(C=64, d=128, heads=2, layers=2, mlp_ratio=4, frame_len=130, max_frames=4, dtype="bf16")
+BF16 = syn.ModelShape(C=128, d=128, heads=2, layers=2, mlp_ratio=4, frame_len=130, max_frames=4, dtype="bf16")
 
 
 @pytest.fixture(scope="module")
@@ -92,3 +92,9 @@ def test_denoiser_and_flow_calls_reject_each_others_models(flow):
         flow.af_denoise(fl, x, 0.1, ws=fl.workspace(1, 64))
     with pytest.raises(flow.AFError):
         flow.af_forward(den, x, 0, ws=den.workspace(1, 64))
+
+
+def test_bf16_denoiser_needs_a_head_tile_width(flow):
+    bad = syn.ModelShape(C=64, d=128, heads=2, layers=1, mlp_ratio=4, frame_len=130, max_frames=1, dtype="bf16")
+    with pytest.raises(flow.AFError):
+        flow.AFModel(bad, syn.make_denoiser_weights(bad), denoiser=True)

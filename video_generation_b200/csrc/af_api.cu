@@ -78,6 +78,7 @@ struct af_model {
   int pdl;            // launch with programmatic dependent launch (see af_kernels.h)
   uint64_t wait_ns;   // limit of one pipeline wait in the tensor-core kernels
   int kind;           // KIND_FLOW (an AF block) or KIND_DENOISER
+  int l2_keep;        // keep the hidden state / residual stream / attention output in L2 (evict_last stores)
   std::vector<void*> allocs;
   // graph cache (keyed by every pointer and scalar baked into the graph)
   std::map<std::string, cudaGraphExec_t> graphs;
@@ -175,6 +176,7 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
   e.h = b.h;
   e.d = d;
   e.wait_ns = m->wait_ns;
+  e.l2_keep = m->l2_keep;
   e.Lc = L;
   e.pos_space = m->pos_space;
   e.pos_time = m->pos_time;
@@ -277,7 +279,7 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
       if (!gemm(EPI_QKV, tA_a, w.w_qkv, 3 * d, d, eq)) { set_err("GEMM plan failed (qkv)"); return AF_ERR_CUDA; }
       if (!launch_attn_tc2(b.ctl, q, (const bf16*)kvl, (const bf16*)(kvl + kv_layer), a, b.opart, b.mlpart, b.nsplit,
                            batch, L, d, c.heads, r_max, m_max, m->num_sms, m->wait_ns, mask_frame(l), mask_ahead(l),
-                           m->d_err, st)) {
+                           m->l2_keep, m->d_err, st)) {
         set_err("attention plan failed");
         return AF_ERR_CUDA;
       }
@@ -717,6 +719,10 @@ af_status create_model(const af_config* cfg, const float* const* tensors, int n_
     set_err("bad dtype");
     return AF_ERR_ARG;
   }
+  if (kind == KIND_DENOISER && c.dtype == AF_BF16 && c.C % 128 && c.C % 192) {
+    set_err("bf16 denoiser: the head's C outputs need C %% 128 == 0 or C %% 192 == 0 (tensor-core tile widths)");
+    return AF_ERR_ARG;
+  }
   if (n_tensors != af_num_tensors(cfg)) { set_err("expected %d tensors, got %d", af_num_tensors(cfg), n_tensors); return AF_ERR_ARG; }
   for (int i = 0; i < n_tensors; ++i)
     if (!tensors[i]) { set_err("null tensor %d", i); return AF_ERR_ARG; }
@@ -725,6 +731,8 @@ af_status create_model(const af_config* cfg, const float* const* tensors, int n_
   m->kind = kind;
   m->pdl = 1;
   m->wait_ns = 2000000000ull;
+  m->l2_keep = 1;
+  if (const char* v = getenv("AF_L2_KEEP")) m->l2_keep = atoi(v) != 0;
   if (const char* v = getenv("AF_PDL")) m->pdl = atoi(v) != 0;
   m->cfg = c;
   m->fd = c.mlp_ratio * c.d;

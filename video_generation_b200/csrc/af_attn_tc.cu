@@ -102,15 +102,15 @@ struct Abort {
 };
 __device__ bool mbar_wait(uint32_t bar, uint32_t parity, const Abort& ab) {
   if (mbar_try(bar, parity)) return true;
+  // slow path: every poll (a try_wait may itself block for a while) checks
+  // the CTA's abort flag and the time
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 1;; ++i) {
+  for (;;) {
     if (mbar_try(bar, parity)) return true;
-    if ((i & 63u) == 0u) {
-      if (*ab.flag) return false;
-      if (globaltimer_ns() - t0 > ab.limit_ns) {
-        *ab.flag = 1;
-        return false;
-      }
+    if (*ab.flag) return false;
+    if (globaltimer_ns() - t0 > ab.limit_ns) {
+      *ab.flag = 1;
+      return false;
     }
   }
 }
@@ -184,6 +184,17 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
                "r"(src), "r"(c0), "r"(c1)
                : "memory");
 }
+__device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap* map, uint32_t src, int c0, int c1, uint64_t pol) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(c0), "r"(c1), "l"(pol)
+               : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
@@ -209,6 +220,7 @@ struct AttnArgs {
   int Lc, d, heads, nsplit_max, m_max, batch, sms;
   uint64_t wait_ns;  // limit of a pipeline wait before the CTA aborts
   KeyMask km;        // which keys a query attends
+  int l2_keep;       // output stored with an L2 evict_last policy (read by the next GEMM at once)
 };
 
 // Key splits of a pass, decided from the rows the pass really has (ctl->R
@@ -688,8 +700,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         __syncwarp();
         if (lane == 0) {
 #pragma unroll
-          for (int ch = 0; ch < HD / 16; ++ch)
-            tma_store_2d(&tmO, smem_u32(stg + ch * 1024), xe.hh * HD + ch * 16, xe.s * R + q0);
+          if (g.l2_keep) {
+            const uint64_t pol = policy_evict_last();
+            for (int ch = 0; ch < HD / 16; ++ch)
+              tma_store_2d_hint(&tmO, smem_u32(stg + ch * 1024), xe.hh * HD + ch * 16, xe.s * R + q0, pol);
+          } else {
+            for (int ch = 0; ch < HD / 16; ++ch)
+              tma_store_2d(&tmO, smem_u32(stg + ch * 1024), xe.hh * HD + ch * 16, xe.s * R + q0);
+          }
           bulk_commit();
         }
         stg_buf = sb;
@@ -785,7 +803,8 @@ int attn_tc_splits(int batch, int heads, int r_max, int Lc, int num_sms) {
 
 bool launch_attn_tc2(const Ctl* ctl, const bf16* q, const bf16* kc, const bf16* vc, bf16* o, float* opart,
                      float* mlpart, int nsplit_max, int batch, int Lc, int d, int heads, int r_max, int m_max,
-                     int num_sms, uint64_t wait_ns, int mask_frame, int mask_ahead, int* err, cudaStream_t st) {
+                     int num_sms, uint64_t wait_ns, int mask_frame, int mask_ahead, int l2_keep, int* err,
+                     cudaStream_t st) {
   const int hd = d / heads;
   const int bkv = hd == 64 ? AttnCfg<64>::BKV : AttnCfg<128>::BKV;
   CUtensorMap tq, tk, tv, to;
@@ -808,6 +827,7 @@ bool launch_attn_tc2(const Ctl* ctl, const bf16* q, const bf16* kc, const bf16* 
   g.km.F = mask_frame;
   g.km.ahead = mask_ahead;
   g.km.Lc = Lc;
+  g.l2_keep = l2_keep;
   return hd == 64 ? launch_hd<64>(tq, tk, tv, to, g, batch, r_max, err, st)
                   : launch_hd<128>(tq, tk, tv, to, g, batch, r_max, err, st);
 }

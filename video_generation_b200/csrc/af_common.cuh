@@ -81,6 +81,7 @@ struct EpiArgs {
   const int* active;       // inverse: per-sample flag
   float* part;             // [Mmax, 2C/16, 2] per-(row, 16-column group) partial sums
   uint64_t wait_ns;        // tensor-core kernels: limit of a pipeline wait before the CTA aborts
+  int l2_keep;             // TMA outputs (residual adds, GELU) stored with an L2 evict_last policy
 };
 
 __device__ __forceinline__ int tok_of(int p, int L, int dir) { return dir ? (L - 1 - p) : p; }

@@ -104,15 +104,15 @@ struct Abort {
 // aborted or the wait limit has passed (which aborts the CTA).
 __device__ bool mbar_wait(uint32_t bar, uint32_t parity, const Abort& ab) {
   if (mbar_try(bar, parity)) return true;
+  // slow path: every poll (a try_wait may itself block for a while) checks
+  // the CTA's abort flag and the time
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 1;; ++i) {
+  for (;;) {
     if (mbar_try(bar, parity)) return true;
-    if ((i & 63u) == 0u) {
-      if (*ab.flag) return false;
-      if (globaltimer_ns() - t0 > ab.limit_ns) {
-        *ab.flag = 1;
-        return false;
-      }
+    if (*ab.flag) return false;
+    if (globaltimer_ns() - t0 > ab.limit_ns) {
+      *ab.flag = 1;
+      return false;
     }
   }
 }
@@ -244,6 +244,27 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
                    reinterpret_cast<uint64_t>(map)),
                "r"(src), "r"(c0), "r"(c1)
                : "memory");
+}
+// The same with an L2 cache policy (createpolicy): outputs the next kernel
+// reads at once are kept in L2 with evict_last.
+__device__ __forceinline__ void tma_reduce_add_2d_hint(const CUtensorMap* map, uint32_t src, int c0, int c1,
+                                                       uint64_t pol) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(c0), "r"(c1), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap* map, uint32_t src, int c0, int c1, uint64_t pol) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(c0), "r"(c1), "l"(pol)
+               : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // at most one group still reading its shared-memory source
@@ -435,6 +456,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
       constexpr int NCH = HALF / 16;
       uint8_t* stg0 = reinterpret_cast<uint8_t*>(sEpi) + ew * 2 * SLOT;
       const int R = e.ctl->R, p0 = e.ctl->p0;
+      const uint64_t keep_pol = e.l2_keep ? policy_evict_last() : 0ull;
       int cc = 0;                                       // chunks sent by this warp
       int i = 0;
       for (int t = unit; t < ntiles; t += nunits, ++i) {
@@ -532,7 +554,9 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) {
-              if (EPI == EPI_RESID) tma_reduce_add_2d(&tmC, smem_u32(slot), col, row0);
+              if (e.l2_keep && EPI == EPI_RESID) tma_reduce_add_2d_hint(&tmC, smem_u32(slot), col, row0, keep_pol);
+              else if (EPI == EPI_RESID) tma_reduce_add_2d(&tmC, smem_u32(slot), col, row0);
+              else if (e.l2_keep && EPI == EPI_GELU) tma_store_2d_hint(&tmC, smem_u32(slot), col, row0, keep_pol);
               else if (EPI == EPI_GELU || which == 0) tma_store_2d(&tmC, smem_u32(slot), col - which * e.d, row0);
               else tma_store_2d(which == 1 ? &tmC2 : &tmC3, smem_u32(slot), col - which * e.d, ycache);
               bulk_commit();

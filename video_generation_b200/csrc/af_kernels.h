@@ -100,6 +100,7 @@ int gemm_tc_pick(int N, int m_max, int num_sms, int unit, int max_bn);
 int attn_tc_splits(int batch, int heads, int r_max, int Lc, int num_sms);
 bool launch_attn_tc2(const Ctl* ctl, const bf16* q, const bf16* kc, const bf16* vc, bf16* o, float* opart,
                      float* mlpart, int nsplit_max, int batch, int Lc, int d, int heads, int r_max, int m_max,
-                     int num_sms, uint64_t wait_ns, int mask_frame, int mask_ahead, int* err, cudaStream_t st);
+                     int num_sms, uint64_t wait_ns, int mask_frame, int mask_ahead, int l2_keep, int* err,
+                     cudaStream_t st);
 
 }  // namespace af

@@ -35,3 +35,17 @@ def jacobi_flops(shape, iters, L: int, B: int) -> float:
                 if b + 1 < nb:
                     total += f          # the K/V commit of block b
     return total
+
+
+def denoiser_flops(shape, batch: int, L: int) -> float:
+    """One forward pass of the flow-score-matching denoiser: the dense
+    contractions of every row, plus 4*d flops per (query, key) pair that its
+    frame masks allow (one frame of look-ahead in the first layer, frames up
+    to the query's own in the others)."""
+    F = shape.frame_len
+    d, C = shape.d, shape.C
+    dense = L * (shape.layers * (2 * d * 3 * d + 2 * d * d + 2 * 2 * shape.mlp_ratio * d * d) + 2 * C * d + 2 * C * d)
+    pairs_first = sum(min((p // F + 2) * F, L) for p in range(L))
+    pairs_rest = sum(min((p // F + 1) * F, L) for p in range(L))
+    att = 4.0 * d * (pairs_first + (shape.layers - 1) * pairs_rest)
+    return float(batch) * (dense + att)
