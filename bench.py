@@ -462,6 +462,30 @@ def extra_line(w, args, dev, peaks):
 
 # ----------------------------------------------------------------------------- main
 
+def fd_passes(args, dev):
+    """The deep flow's Jacobi passes in a graph ncu can profile: the flow-encode
+    of the 5 s clip in passes of 390 query rows, each attending the cache of
+    the frames before it -- the shape of one Jacobi update of each block (the
+    Jacobi graph itself has conditional nodes, whose kernels ncu does not
+    profile).  Prints one JSON line (not the throughput contract's)."""
+    import torch
+    from video_generation_b200 import flow
+    w = syn.WORKLOADS[4]
+    model = flow.AFModel(w.shape, syn.make_weights(w.shape))
+    x = torch.from_numpy(syn.workload_latents(w, "x")).to(dev)
+    B = w.B // 2                                   # passes of 2B = 390 rows
+    ws = model.workspace(1, w.L, B, device=dev)
+    st = torch.cuda.current_stream()
+    t = time_calls(lambda: flow.af_prefix_encode(model, x, 0, B, w.L, ws), args.warmup, args.steps, st)
+    n_pass = w.L // (2 * B)
+    fl = sum(FL.pass_flops(w.shape.d, w.shape.C, w.shape.layers, w.shape.mlp_ratio, 2 * B,
+                           FL.causal_pairs(i * 2 * B, 2 * B)) for i in range(n_pass))
+    peaks, kind = load_peaks()
+    print(json.dumps({"mode": "fd_passes", "workload": w.name, "passes": n_pass, "rows_per_pass": 2 * B,
+                      "ms_per_pass": 1e3 * t / n_pass, "tflops": fl / t / 1e12,
+                      "frac_of_bf16_peak": fl / t / 1e12 / peaks["bf16_tflops"], "peak_kind": kind}), flush=True)
+
+
 def relaunch_under_torchrun(args):
     s = socket.socket()
     s.bind(("127.0.0.1", 0))
@@ -483,6 +507,8 @@ def main():
     ap.add_argument("--cpu-frames", type=int, default=2, help="frames in the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip configs 2, 4, 5 in a one-GPU run")
+    ap.add_argument("--fd-passes", action="store_true",
+                    help="time (or profile) the deep flow's 390-row Jacobi passes outside the Jacobi graph")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -506,6 +532,9 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.fd_passes:
+        fd_passes(args, dev)
+        return
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)

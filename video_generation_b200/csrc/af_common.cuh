@@ -54,7 +54,9 @@ enum Epi : int {
   EPI_RESID = 2,    // h += acc + b                                      (fp32 h)
   EPI_GELU = 3,     // u = gelu(acc + b)                                 (act type)
   EPI_HEAD = 4,     // affine map from interleaved (mu_c, s_c) columns   (fp32 x/z)
-  EPI_RAW = 5       // out32 = acc                                       (fp32 scratch)
+  EPI_RAW = 5,      // out32 = acc                                       (fp32 scratch)
+  EPI_DENOISE = 6,  // x = x_noisy + sigma * (acc + b), plain columns    (fp32 x)
+  EPI_RESID_SPLIT = 7  // EPI_RESID over K split across CTAs (fixed-order sum of partials)
 };
 
 // Everything an epilogue may touch.  Pointers not used by a kind stay null.
@@ -82,6 +84,12 @@ struct EpiArgs {
   float* part;             // [Mmax, 2C/16, 2] per-(row, 16-column group) partial sums
   uint64_t wait_ns;        // tensor-core kernels: limit of a pipeline wait before the CTA aborts
   int l2_keep;             // TMA outputs (residual adds, GELU) stored with an L2 evict_last policy
+  // split-K of the residual GEMMs (ksplit > 1): fp32 partials [ksplit][kpart_rows][N]
+  // and one arrival counter per (tile, CTA of the pair, epilogue warp), zero at rest
+  int ksplit;
+  float* kpart;
+  int* kcnt;
+  int kpart_rows;
 };
 
 __device__ __forceinline__ int tok_of(int p, int L, int dir) { return dir ? (L - 1 - p) : p; }

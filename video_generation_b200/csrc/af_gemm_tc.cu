@@ -43,8 +43,8 @@ template <int EPI> struct EpiShape {
   // residual add, GELU and QKV leave through TMA: each warp stages 32 rows x
   // 16 columns (two slots, alternating) in the output tensor map's swizzle and
   // issues a bulk reduce-add (h += tile) or a bulk store (u, q, K / V cache)
-  static constexpr bool TMA_OUT = EPI == EPI_RESID || EPI == EPI_GELU || EPI == EPI_QKV;
-  static constexpr uint32_t SLOT = EPI == EPI_RESID ? 32 * 16 * 4 : 32 * 16 * 2;
+  static constexpr bool TMA_OUT = EPI == EPI_RESID || EPI == EPI_RESID_SPLIT || EPI == EPI_GELU || EPI == EPI_QKV;
+  static constexpr uint32_t SLOT = (EPI == EPI_RESID || EPI == EPI_RESID_SPLIT) ? 32 * 16 * 4 : 32 * 16 * 2;
 };
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kMaxDevices = 64;
@@ -345,6 +345,10 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
   const int M = e.ctl->M;
   const int tiles_m = (M + TM - 1) / TM;
   const int ntiles = tiles_m * tiles_n;
+  // Work unit t: tile t % ntiles, K range t / ntiles of KS equal ranges
+  // (KS = 1 except for split residual GEMMs).
+  const int KS = EPI == EPI_RESID_SPLIT ? e.ksplit : 1;
+  const int nwork = ntiles * KS;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -352,12 +356,14 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       long long issued = 0;
-      for (int t = unit; t < ntiles; t += nunits) {
-        const int mb = t % tiles_m, nb = t / tiles_m;
+      for (int t = unit; t < nwork; t += nunits) {
+        const int tb = t % ntiles, ks = t / ntiles;
+        const int mb = tb % tiles_m, nb = tb / tiles_m;
         const int arow = mb * TM + (int)rank * BM;
         const int brow = nb * BN + (int)rank * (BN / CG);
+        const int kb0 = ks * kbn / KS, kb1 = (ks + 1) * kbn / KS;
         bool ok = true;
-        for (int kb = 0; kb < kbn; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, ab)) { ok = false; break; }
           if (rank == 0) mbar_expect_tx(full0 + 8 * stage, CG * Cfg::STAGE_BYTES);
           if (CG == 2) {
@@ -402,22 +408,25 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       int i = 0;
-      for (int t = unit; t < ntiles; t += nunits, ++i) {
+      for (int t = unit; t < nwork; t += nunits, ++i) {
         const int acc = i & 1;
         const uint32_t use = (uint32_t)(i >> 1);
+        const int ks = t / ntiles;
+        const int kb0 = ks * kbn / KS, kb1 = (ks + 1) * kbn / KS;
         if (!mbar_wait(tempty0 + 8 * acc, (use & 1u) ^ 1u, ab)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
         bool ok = true;
-        for (int kb = 0; kb < kbn; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(full0 + 8 * stage, phase, ab)) { ok = false; break; }
           tc_fence_after();
           const uint64_t da = sw128_desc(smem_u32(sA + stage * Cfg::A_BYTES));
           const uint64_t db = sw128_desc(smem_u32(sB + stage * Cfg::B_BYTES));
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            if (CG == 2) umma_bf16_pair(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), Cfg::IDESC, (kb | k) != 0);
-            else umma_bf16(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), Cfg::IDESC, (kb | k) != 0);
+            const uint32_t accum = ((kb - kb0) | k) != 0;
+            if (CG == 2) umma_bf16_pair(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), Cfg::IDESC, accum);
+            else umma_bf16(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), Cfg::IDESC, accum);
           }
           if (CG == 2) umma_commit_pair(empty0 + 8 * stage);
           else umma_commit(empty0 + 8 * stage);
@@ -459,6 +468,86 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
       const uint64_t keep_pol = e.l2_keep ? policy_evict_last() : 0ull;
       int cc = 0;                                       // chunks sent by this warp
       int i = 0;
+      if constexpr (EPI == EPI_RESID_SPLIT) {
+        // Split K: each of the KS units of a tile stores its fp32 partial
+        // (thread = row, 16 columns a chunk) and counts itself in a counter of
+        // (tile, CTA, warp); the last to arrive adds the KS partials in split
+        // order, adds the bias and sends the sum into h by TMA reduce-add -- one
+        // add per element of h, and the same sum whichever unit finishes last.
+        for (int t = unit; t < nwork; t += nunits, ++i) {
+          const int acc = i & 1;
+          const uint32_t use = (uint32_t)(i >> 1);
+          const int tb = t % ntiles, ks = t / ntiles;
+          const int mb = tb % tiles_m, nb = tb / tiles_m;
+          const int row0 = mb * TM + (int)rank * BM + q * 32;
+          const int n0 = nb * BN + hf * HALF;
+          const uint32_t taddr = tmem + (uint32_t)(acc * BN + hf * HALF) + ((uint32_t)(q * 32) << 16);
+          const int r = row0 + lane;
+          const bool rok = r < e.kpart_rows;
+          const size_t ld = (size_t)tiles_n * BN;                       // N
+          if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * acc, use & 1u, ab))) break;
+          tc_fence_after();
+          float* mine = e.kpart + ((size_t)ks * e.kpart_rows + r) * ld + n0;
+#pragma unroll
+          for (int k = 0; k < NCH; ++k) {
+            float v[16];
+            tmem_ld16(taddr + k * 16, v);
+            tmem_wait_ld();
+            if (rok) {
+              float4* dst = reinterpret_cast<float4*>(mine + k * 16);
+#pragma unroll
+              for (int jj = 0; jj < 4; ++jj) dst[jj] = make_float4(v[4 * jj], v[4 * jj + 1], v[4 * jj + 2], v[4 * jj + 3]);
+            }
+          }
+          tc_fence_before();
+          if (CG == 2) mbar_arrive_cluster(tempty_lead + 8 * acc);
+          else mbar_arrive(tempty0 + 8 * acc);
+          __threadfence();
+          __syncwarp();
+          int* cnt = e.kcnt + ((size_t)tb * CG + rank) * Cfg::EPI_WARPS + ew;
+          int before = 0;
+          if (lane == 0) before = atomicAdd(cnt, 1);
+          before = __shfl_sync(0xffffffffu, before, 0);
+          if (before != KS - 1) continue;                 // another unit finishes this tile
+          __threadfence();
+#pragma unroll
+          for (int k = 0; k < NCH; ++k) {
+            const int col = n0 + k * 16;
+            float v[16];
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) v[jj] = 0.f;
+            if (rok) {
+              for (int sk = 0; sk < KS; ++sk) {
+                const float4* src = reinterpret_cast<const float4*>(e.kpart + ((size_t)sk * e.kpart_rows + r) * ld + col);
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                  const float4 a4 = __ldcg(src + jj);
+                  v[4 * jj] += a4.x; v[4 * jj + 1] += a4.y; v[4 * jj + 2] += a4.z; v[4 * jj + 3] += a4.w;
+                }
+              }
+            }
+            uint8_t* slot = stg0 + (cc & 1) * SLOT;
+            if (lane == 0) bulk_wait_read1();             // the slot's previous tile has been read
+            __syncwarp();
+            uint8_t* rp = slot + lane * 64;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              const float4 bb = reinterpret_cast<const float4*>(e.bias + col)[jj];
+              *reinterpret_cast<float4*>(rp + ((jj ^ ((lane >> 1) & 3)) << 4)) =
+                  make_float4(v[4 * jj] + bb.x, v[4 * jj + 1] + bb.y, v[4 * jj + 2] + bb.z, v[4 * jj + 3] + bb.w);
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
+              if (e.l2_keep) tma_reduce_add_2d_hint(&tmC, smem_u32(slot), col, row0, keep_pol);
+              else tma_reduce_add_2d(&tmC, smem_u32(slot), col, row0);
+              bulk_commit();
+            }
+            ++cc;
+          }
+          if (lane == 0) atomicExch(cnt, 0);              // zero again for the next launch
+        }
+      } else {
       for (int t = unit; t < ntiles; t += nunits, ++i) {
         const int acc = i & 1;
         const uint32_t use = (uint32_t)(i >> 1);
@@ -565,6 +654,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
           }
         }
       }
+      }
       if (lane == 0) bulk_wait_all();                   // the bulk writes are complete before the CTA exits
       __syncwarp();
     } else {
@@ -574,7 +664,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
       // 8 it + l / 4, columns 4 (l % 4) .. + 3: each store covers eight 64-byte
       // row segments.  The head keeps thread = row.  Row -> (sample, position)
       // and the row pointers are computed once per tile.
-      static_assert(EPI == EPI_INPROJ || EPI == EPI_HEAD, "epilogue without a TMA path");
+      static_assert(EPI == EPI_INPROJ || EPI == EPI_HEAD || EPI == EPI_DENOISE, "epilogue without a TMA path");
       float* stg = sEpi + ew * 32 * 16;
       const int rl = lane >> 2, cq = lane & 3;
       const int sw_w = (lane >> 1) & 3;            // swizzle of the row this lane writes
@@ -609,7 +699,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
         const float* hin = nullptr;
         float* hout = nullptr;
         float* hpart = nullptr;
-        if (EPI == EPI_HEAD) {
+        if (EPI == EPI_HEAD || EPI == EPI_DENOISE) {
           const int r = row0 + lane;
           const int sm = r / R;
           const int p = p0 + (r - sm * R);
@@ -618,7 +708,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
           hin = e.xin_f + base;
           hout = e.xout_f + base;
           hpart = e.part + (size_t)r * ((2 * e.C) >> 4) * 2;
-          head_act = head_out && (e.head_mode != 1 || e.active[sm]);
+          head_act = head_out && (EPI == EPI_DENOISE || e.head_mode == 0 || e.active[sm]);
         }
         // Loads that do not depend on the accumulator are issued before waiting
         // for it (bias, and the first chunk's position / x rows), and every
@@ -630,12 +720,16 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
         for (int k = 0; k < NCH; ++k) bias4[k] = *reinterpret_cast<const float4*>(e.bias + n0 + k * 16 + cq * 4);
         float4 pre[2][4], pre2[2][4];
         auto load_rows = [&](int k, float4* dst, float4* dst2) {
-          if (EPI == EPI_HEAD) {
-            if (head_act && e.head_mode == 2) {             // denoiser: 16 plain channels
+          if (EPI == EPI_DENOISE) {                         // 16 plain channels
+            if (head_act) {
               const float4* src = reinterpret_cast<const float4*>(hin + n0 + k * 16);
 #pragma unroll
               for (int qq = 0; qq < 4; ++qq) dst[qq] = src[qq];
-            } else if (head_act) {
+            }
+            return;
+          }
+          if (EPI == EPI_HEAD) {
+            if (head_act) {
               const int c0 = (n0 + k * 16) >> 1;
               dst[0] = *reinterpret_cast<const float4*>(hin + c0);
               dst[1] = *reinterpret_cast<const float4*>(hin + c0 + 4);
@@ -670,7 +764,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
             load_rows(k + 1, pre[(k + 1) & 1], pre2[(k + 1) & 1]);
           }
           const float* v = vb[k & 1];
-          if (EPI == EPI_HEAD && e.head_mode == 2) {
+          if (EPI == EPI_DENOISE) {
             // denoiser: x = x_noisy + sigma * (s_phi + b) for 16 plain channels
             if (!head_out) continue;
             const int col0 = n0 + c;
@@ -779,7 +873,7 @@ void launch_bn_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtenso
         max_units = clusters;
     }
   }
-  const int tiles = ((m_max + BM * CG - 1) / (BM * CG)) * (N / BN);
+  const int tiles = ((m_max + BM * CG - 1) / (BM * CG)) * (N / BN) * (EPI == EPI_RESID_SPLIT ? e.ksplit : 1);
   const int units = tiles < max_units ? tiles : max_units;
   if (CG == 1) {
     launch_k(k_gemm_tc<BN, EPI, 1>, dim3(units), dim3(Cfg::THREADS), Cfg::SMEM, st, tmA, tmB, tmC, tmC2, tmC3, N, K, e, err);
@@ -809,7 +903,11 @@ void launch_bn(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, const CU
     case EPI_QKV: launch_bn_epi<BN, EPI_QKV, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st); break;
     case EPI_RESID: launch_bn_epi<BN, EPI_RESID, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st); break;
     case EPI_GELU: launch_bn_epi<BN, EPI_GELU, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st); break;
-    default: launch_bn_epi<BN, EPI_HEAD, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st); break;
+    case EPI_HEAD: launch_bn_epi<BN, EPI_HEAD, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st); break;
+    case EPI_RESID_SPLIT:
+      launch_bn_epi<BN, EPI_RESID_SPLIT, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st);
+      break;
+    default: launch_bn_epi<BN, EPI_DENOISE, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st); break;
   }
 }
 
@@ -874,6 +972,27 @@ int gemm_tc_pick(int N, int m_max, int num_sms, int unit, int max_bn) {
     if (!best || cost < best_cost) { best = bn; best_cost = cost; }
   }
   return best ? best * 10 + cg : 0;
+}
+
+// K splits of a residual GEMM (see the split-K epilogue): when its tiles
+// leave SM pairs idle, up to 4 splits of at least 4 k-blocks each, so that
+// tiles * splits fills the GPU at most once.
+int gemm_tc_ksplit(int pick, int N, int K, int m_max, int num_sms) {
+  const int bn = pick / 10, cg = pick % 10;
+  if (!bn) return 1;
+  const int units = num_sms / cg;
+  const int tiles = ((m_max + BM * cg - 1) / (BM * cg)) * (N / bn);
+  if (tiles >= units) return 1;
+  int ks = units / tiles;
+  if (ks > 4) ks = 4;
+  const int by_k = (K / BK) / 4;
+  if (ks > by_k) ks = by_k;
+  return ks < 1 ? 1 : ks;
+}
+
+int gemm_tc_tiles(int pick, int N, int m_max) {
+  const int bn = pick / 10, cg = pick % 10;
+  return bn ? ((m_max + BM * cg - 1) / (BM * cg)) * (N / bn) : 0;
 }
 
 void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap* tmC,

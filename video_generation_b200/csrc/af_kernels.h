@@ -91,6 +91,9 @@ void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, con
                     const CUtensorMap* tmC2, const CUtensorMap* tmC3, int pick, int N, int K, int m_max,
                     const EpiArgs& e, int* err, int num_sms, cudaStream_t st);
 int gemm_tc_pick(int N, int m_max, int num_sms, int unit, int max_bn);
+// K splits of a residual GEMM with tile shape `pick` (1 = none), and its tile count.
+int gemm_tc_ksplit(int pick, int N, int K, int m_max, int num_sms);
+int gemm_tc_tiles(int pick, int N, int m_max);
 
 // Causal attention over the KV cache on tcgen05 (af_attn_tc.cu).  Each pass
 // splits its live key range into at most nsplit_max splits (attn_tc_splits
