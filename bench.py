@@ -387,7 +387,7 @@ def deep_flow_extras(args, dev, peaks):
     # block-size sweep (uniform blocks) and the asymmetric schedule
     sweep = {}
     F = w4.shape.frame_len
-    schedules = {f"B{b}": [b] * (w4.L // b) for b in (130, 195, 390, 780, 1170)}
+    schedules = {f"B{b}": [b] * (w4.L // b) for b in (130, 195, 390, 819, 1170, 1638)}   # divisors of 8190
     schedules["first_frame_65_then_780"] = [65] * (F // 65) + [780] * ((w4.L - F) // 780)
     for name, sizes in schedules.items():
         assert sum(sizes) == w4.L

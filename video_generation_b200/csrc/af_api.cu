@@ -158,9 +158,11 @@ Bufs carve(const af_model* m, void* ws, int batch, int L, int B) {
   if (m->bf) {
     // the residual GEMMs (N = d; K = d and K = mlp width) split K when their
     // tiles leave SM pairs idle
+    // (a Jacobi workspace's passes carry half its rows except on a commit)
     const int pick = gemm_tc_pick(c.d, (int)mmax, m->num_sms, 0, 256);
-    const int ks1 = gemm_tc_ksplit(pick, c.d, c.d, (int)mmax, m->num_sms);
-    const int ks2 = gemm_tc_ksplit(pick, c.d, m->fd, (int)mmax, m->num_sms);
+    const int fewest = B < L ? (int)(mmax / 2) : (int)mmax;
+    const int ks1 = gemm_tc_ksplit(pick, c.d, c.d, fewest, m->num_sms);
+    const int ks2 = gemm_tc_ksplit(pick, c.d, m->fd, fewest, m->num_sms);
     b.ksplit = ks1 > ks2 ? ks1 : ks2;
     if (b.ksplit > 1) {
       b.kpart = (float*)take(sizeof(float) * (size_t)b.ksplit * mmax * c.d);
@@ -276,7 +278,7 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
       EpiArgs ea = ea0;
       ea.ksplit = 1;
       if (epi == EPI_RESID && b.ksplit > 1) {
-        ea.ksplit = gemm_tc_ksplit(pick, N, K, m_max, ns);
+        ea.ksplit = gemm_tc_ksplit(pick, N, K, m_max == r_max * batch && r_max < L ? m_max / 2 : m_max, ns);
         ea.kpart = b.kpart;
         ea.kcnt = b.kcnt;
         ea.kpart_rows = m_max;

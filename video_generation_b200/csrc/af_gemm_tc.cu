@@ -346,8 +346,16 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
   const int tiles_m = (M + TM - 1) / TM;
   const int ntiles = tiles_m * tiles_n;
   // Work unit t: tile t % ntiles, K range t / ntiles of KS equal ranges
-  // (KS = 1 except for split residual GEMMs).
-  const int KS = EPI == EPI_RESID_SPLIT ? e.ksplit : 1;
+  // (KS = 1 except for split residual GEMMs, whose KS is chosen here from the
+  // live tile count: as many splits, up to e.ksplit and at least 4 k-blocks
+  // each, as the launched units can run at once).
+  int KS = 1;
+  if (EPI == EPI_RESID_SPLIT) {
+    KS = nunits / ntiles;
+    if (KS > e.ksplit) KS = e.ksplit;
+    if (KS > kbn / 4) KS = kbn / 4;
+    if (KS < 1) KS = 1;
+  }
   const int nwork = ntiles * KS;
 
   if (warp == 0) {
@@ -505,11 +513,13 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
           __threadfence();
           __syncwarp();
           int* cnt = e.kcnt + ((size_t)tb * CG + rank) * Cfg::EPI_WARPS + ew;
-          int before = 0;
-          if (lane == 0) before = atomicAdd(cnt, 1);
-          before = __shfl_sync(0xffffffffu, before, 0);
-          if (before != KS - 1) continue;                 // another unit finishes this tile
-          __threadfence();
+          if (KS > 1) {
+            int before = 0;
+            if (lane == 0) before = atomicAdd(cnt, 1);
+            before = __shfl_sync(0xffffffffu, before, 0);
+            if (before != KS - 1) continue;               // another unit finishes this tile
+            __threadfence();
+          }
 #pragma unroll
           for (int k = 0; k < NCH; ++k) {
             const int col = n0 + k * 16;
@@ -545,7 +555,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
             }
             ++cc;
           }
-          if (lane == 0) atomicExch(cnt, 0);              // zero again for the next launch
+          if (KS > 1 && lane == 0) atomicExch(cnt, 0);    // zero again for the next launch
         }
       } else {
       for (int t = unit; t < ntiles; t += nunits, ++i) {
@@ -974,14 +984,15 @@ int gemm_tc_pick(int N, int m_max, int num_sms, int unit, int max_bn) {
   return best ? best * 10 + cg : 0;
 }
 
-// K splits of a residual GEMM (see the split-K epilogue): when its tiles
-// leave SM pairs idle, up to 4 splits of at least 4 k-blocks each, so that
-// tiles * splits fills the GPU at most once.
-int gemm_tc_ksplit(int pick, int N, int K, int m_max, int num_sms) {
+// The most K splits a residual GEMM may use (see the split-K epilogue): up
+// to 4, at least 4 k-blocks each, when a pass of m_rows rows (the fewest a
+// call's passes have) leaves SM pairs idle; the kernel picks the count for
+// the live rows of each launch.
+int gemm_tc_ksplit(int pick, int N, int K, int m_rows, int num_sms) {
   const int bn = pick / 10, cg = pick % 10;
-  if (!bn) return 1;
+  if (!bn || m_rows < 1) return 1;
   const int units = num_sms / cg;
-  const int tiles = ((m_max + BM * cg - 1) / (BM * cg)) * (N / bn);
+  const int tiles = ((m_rows + BM * cg - 1) / (BM * cg)) * (N / bn);
   if (tiles >= units) return 1;
   int ks = units / tiles;
   if (ks > 4) ks = 4;
