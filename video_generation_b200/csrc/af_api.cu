@@ -154,17 +154,18 @@ Bufs carve(const af_model* m, void* ws, int batch, int L, int B) {
     b.opart = (float*)take(sizeof(float) * (size_t)b.nsplit * mmax * c.d);
     b.mlpart = (float*)take(sizeof(float) * (size_t)b.nsplit * mmax * c.heads * 2);
   }
-  b.ksplit = 1;
+  b.ksplit = 0;
   if (m->bf) {
-    // the residual GEMMs (N = d; K = d and K = mlp width) split K when their
-    // tiles leave SM pairs idle
-    // (a Jacobi workspace's passes carry half its rows except on a commit)
+    // the residual GEMMs (N = d; K = d and K = mlp width) run stream-K when
+    // whole tiles would leave SM pairs idle; the partial slots are sized for
+    // the fewest rows a pass of this workspace has (a Jacobi workspace's
+    // passes carry half its rows except on a commit)
     const int pick = gemm_tc_pick(c.d, (int)mmax, m->num_sms, 0, 256);
     const int fewest = B < L ? (int)(mmax / 2) : (int)mmax;
     const int ks1 = gemm_tc_ksplit(pick, c.d, c.d, fewest, m->num_sms);
     const int ks2 = gemm_tc_ksplit(pick, c.d, m->fd, fewest, m->num_sms);
     b.ksplit = ks1 > ks2 ? ks1 : ks2;
-    if (b.ksplit > 1) {
+    if (b.ksplit > 0) {
       b.kpart = (float*)take(sizeof(float) * (size_t)b.ksplit * mmax * c.d);
       b.kcnt_bytes = sizeof(int) * (size_t)gemm_tc_tiles(pick, c.d, (int)mmax) * 2 * 16;
       b.kcnt = (int*)take(b.kcnt_bytes);
@@ -276,13 +277,18 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
       const int pick = gemm_tc_pick(N, m_max, ns, epi == EPI_QKV ? d : 0, epi == EPI_INPROJ ? 192 : 256);
       if (!pick || !make_tmap_bf16(&tB, W, N, K, (pick / 10) / (pick % 10))) return false;
       EpiArgs ea = ea0;
-      ea.ksplit = 1;
-      if (epi == EPI_RESID && b.ksplit > 1) {
-        ea.ksplit = gemm_tc_ksplit(pick, N, K, m_max == r_max * batch && r_max < L ? m_max / 2 : m_max, ns);
-        ea.kpart = b.kpart;
-        ea.kcnt = b.kcnt;
-        ea.kpart_rows = m_max;
-        if (ea.ksplit > 1) epi = EPI_RESID_SPLIT;
+      ea.ksplit = 0;
+      if (epi == EPI_RESID && b.ksplit > 0) {
+        // stream-K when this GEMM's whole tiles would leave SM pairs idle; the
+        // kernel cuts the live tiles' k-blocks evenly across the pairs
+        const int slots = gemm_tc_ksplit(pick, N, K, r_max < L ? m_max / 2 : m_max, ns);
+        if (slots > 0) {
+          ea.ksplit = b.ksplit;
+          ea.kpart = b.kpart;
+          ea.kcnt = b.kcnt;
+          ea.kpart_rows = m_max;
+          epi = EPI_RESID_SPLIT;
+        }
       }
       const CUtensorMap* tC = (epi == EPI_RESID || epi == EPI_RESID_SPLIT) ? &tC_h
                               : (epi == EPI_GELU ? &tC_u : (epi == EPI_QKV ? &tC_q : nullptr));

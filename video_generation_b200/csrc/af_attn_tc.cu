@@ -228,7 +228,8 @@ struct AttnArgs {
 // length: a pass whose (query tile, head, sample) items already fill the GPU
 // twice over runs unsplit; otherwise the live key range (keys 0 .. p0 + R - 1)
 // is cut into up to nsplit_max splits of at least kMinSplitTiles 64-key tiles,
-// aiming at about 4 items per SM.  The attention kernel and the combine kernel
+// aiming at about 2 items per SM (one per pipeline of a CTA), which bounds the
+// partials the combine kernel reads.  The attention kernel and the combine kernel
 // evaluate this from the same control block, so they agree.
 constexpr int kMinSplitTiles = 8;
 constexpr int kMaxSplits = 32;
@@ -242,7 +243,7 @@ __host__ __device__ __forceinline__ SplitPlan split_plan(int R, int p0, int head
   const int base = sp.q_tiles * heads * batch;
   int n = 1;
   if (nsplit_max > 1 && base < 2 * sms) {
-    const int want = (4 * sms + base - 1) / base;
+    const int want = (2 * sms + base - 1) / base;
     const int by_len = (live + kMinSplitTiles - 1) / kMinSplitTiles;
     n = want < by_len ? want : by_len;
     if (n > nsplit_max) n = nsplit_max;
@@ -793,7 +794,7 @@ int attn_tc_splits(int batch, int heads, int r_max, int Lc, int num_sms) {
   const int bkv = 64;
   const int base_min = heads * batch;                       // a pass with a single query tile
   if (base_min >= 2 * num_sms) return 1;
-  const int want = (4 * num_sms + base_min - 1) / base_min;
+  const int want = (2 * num_sms + base_min - 1) / base_min;
   const int key_tiles = (Lc + bkv - 1) / bkv;
   const int by_len = (key_tiles + kMinSplitTiles - 1) / kMinSplitTiles;
   int n = want < by_len ? want : by_len;
