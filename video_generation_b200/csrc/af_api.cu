@@ -113,10 +113,6 @@ struct Bufs {
   float* opart;   // split-attention partials (bf16 path)
   float* mlpart;
   int nsplit;
-  float* kpart;   // split-K partials of the residual GEMMs (bf16 path, when their tiles leave SMs idle)
-  int* kcnt;      // their arrival counters, zeroed at the start of every call
-  size_t kcnt_bytes;
-  int ksplit;     // the most splits a residual GEMM of this workspace may use
   size_t total;
 };
 
@@ -153,23 +149,6 @@ Bufs carve(const af_model* m, void* ws, int batch, int L, int B) {
   if (b.nsplit > 1) {
     b.opart = (float*)take(sizeof(float) * (size_t)b.nsplit * mmax * c.d);
     b.mlpart = (float*)take(sizeof(float) * (size_t)b.nsplit * mmax * c.heads * 2);
-  }
-  b.ksplit = 0;
-  if (m->bf) {
-    // the residual GEMMs (N = d; K = d and K = mlp width) run stream-K when
-    // whole tiles would leave SM pairs idle; the partial slots are sized for
-    // the fewest rows a pass of this workspace has (a Jacobi workspace's
-    // passes carry half its rows except on a commit)
-    const int pick = gemm_tc_pick(c.d, (int)mmax, m->num_sms, 0, 256);
-    const int fewest = B < L ? (int)(mmax / 2) : (int)mmax;
-    const int ks1 = gemm_tc_ksplit(pick, c.d, c.d, fewest, m->num_sms);
-    const int ks2 = gemm_tc_ksplit(pick, c.d, m->fd, fewest, m->num_sms);
-    b.ksplit = ks1 > ks2 ? ks1 : ks2;
-    if (b.ksplit > 0) {
-      b.kpart = (float*)take(sizeof(float) * (size_t)b.ksplit * mmax * c.d);
-      b.kcnt_bytes = sizeof(int) * (size_t)gemm_tc_tiles(pick, c.d, (int)mmax) * 2 * 16;
-      b.kcnt = (int*)take(b.kcnt_bytes);
-    }
   }
   b.total = off;
   return b;
@@ -271,27 +250,12 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
               make_tmap_bf16(&tA_u, u, m_max, fd, 128) && make_tmap_out(&tC_h, b.h, true, m_max, d) &&
               make_tmap_out(&tC_u, u, false, m_max, fd) && make_tmap_out(&tC_q, q, false, m_max, d);
     if (!ok) { set_err("cuTensorMapEncodeTiled failed for an activation"); return AF_ERR_CUDA; }
-    auto gemm = [&](int epi, const CUtensorMap& tA, const void* W, int N, int K, const EpiArgs& ea0) -> bool {
+    auto gemm = [&](int epi, const CUtensorMap& tA, const void* W, int N, int K, const EpiArgs& ea) -> bool {
       // a QKV tile must fall inside one of q, k, v; the position-add epilogue
       // keeps two row sets in flight and stays at <= 192 columns
       const int pick = gemm_tc_pick(N, m_max, ns, epi == EPI_QKV ? d : 0, epi == EPI_INPROJ ? 192 : 256);
       if (!pick || !make_tmap_bf16(&tB, W, N, K, (pick / 10) / (pick % 10))) return false;
-      EpiArgs ea = ea0;
-      ea.ksplit = 0;
-      if (epi == EPI_RESID && b.ksplit > 0) {
-        // stream-K when this GEMM's whole tiles would leave SM pairs idle; the
-        // kernel cuts the live tiles' k-blocks evenly across the pairs
-        const int slots = gemm_tc_ksplit(pick, N, K, r_max < L ? m_max / 2 : m_max, ns);
-        if (slots > 0) {
-          ea.ksplit = b.ksplit;
-          ea.kpart = b.kpart;
-          ea.kcnt = b.kcnt;
-          ea.kpart_rows = m_max;
-          epi = EPI_RESID_SPLIT;
-        }
-      }
-      const CUtensorMap* tC = (epi == EPI_RESID || epi == EPI_RESID_SPLIT) ? &tC_h
-                              : (epi == EPI_GELU ? &tC_u : (epi == EPI_QKV ? &tC_q : nullptr));
+      const CUtensorMap* tC = epi == EPI_RESID ? &tC_h : (epi == EPI_GELU ? &tC_u : (epi == EPI_QKV ? &tC_q : nullptr));
       launch_gemm_tc(epi, tA, tB, tC, epi == EPI_QKV ? &tC_k : nullptr, epi == EPI_QKV ? &tC_v : nullptr, pick, N, K,
                      m_max, ea, m->d_err, ns, st);
       return true;
@@ -558,7 +522,6 @@ af_status build_forward(void* vctx, cudaStream_t cs) {
   // its attention reads them; the key tile past a sample's last position
   // holds the next sample's rows (written by the same pass) or lies past the
   // cache, where the TMA load fills zeros.
-  if (c->b.kcnt) CK(cudaMemsetAsync(c->b.kcnt, 0, c->b.kcnt_bytes, cs));
   for (int t = 0; t < c->T; ++t) {
     // block t writes z when T-1-t is even, else tmp; block t reads what t-1 wrote
     const float* in = t == 0 ? c->x : (((c->T - t) % 2 == 0) ? c->z : c->b.tmp);
@@ -587,7 +550,6 @@ struct InvCtx {
 af_status build_inverse(void* vctx, cudaStream_t cs) {
   InvCtx* c = static_cast<InvCtx*>(vctx);
   // the masked V rows each block's attention reads are zeroed by its block init
-  if (c->b.kcnt) CK(cudaMemsetAsync(c->b.kcnt, 0, c->b.kcnt_bytes, cs));
   for (int t = c->T - 1; t >= 0; --t) {
     float* out = (t % 2 == 0) ? c->x : c->b.tmp;
     const float* in = (t == c->T - 1) ? c->z : ((((t + 1) % 2) == 0) ? c->x : c->b.tmp);
@@ -657,7 +619,6 @@ af_status build_encode(void* vctx, cudaStream_t cs) {
   const int m_max = c->batch * r_max;
   const size_t kv_layer = (size_t)c->batch * c->L * m->cfg.d * 2;
   bf16* vtail = m->bf ? (bf16*)((char*)c->b.kv + kv_layer) : nullptr;
-  if (c->b.kcnt) CK(cudaMemsetAsync(c->b.kcnt, 0, c->b.kcnt_bytes, cs));
   for (int p0 = 0; p0 < c->n_tokens; p0 += r_max) {
     const int R = (c->n_tokens - p0) < r_max ? (c->n_tokens - p0) : r_max;
     launch_set_pass(c->b.ctl, p0, R, c->batch, vtail, 2 * kv_layer, m->cfg.layers, c->L, m->cfg.d, cs);
@@ -681,7 +642,6 @@ struct DenCtx {
 // The denoiser's forward pass over all positions of every sequence.
 af_status build_denoise(void* vctx, cudaStream_t cs) {
   DenCtx* c = static_cast<DenCtx*>(vctx);
-  if (c->b.kcnt) CK(cudaMemsetAsync(c->b.kcnt, 0, c->b.kcnt_bytes, cs));
   launch_ctl_forward(c->b.ctl, c->batch, c->L, cs);
   HeadIO hio{2, c->xn, c->x, c->sigma};
   af_status s = enqueue_pass(c->m, c->b, c->batch, c->L, AF_L2R, c->batch * c->L, c->L, c->xn, hio, cs);

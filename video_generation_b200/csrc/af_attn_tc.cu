@@ -336,9 +336,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     x.nt = min(ntiles, x.t0 + tps) - x.t0;
     return x;
   };
-  // The CTA's k-th item (k = 0, 1, ...) is global item blockIdx.x + k * gridDim.x
-  // and belongs to group k % 2; every role of a group walks the same items.
-  auto global_item = [&](int k) { return (int)blockIdx.x + k * (int)gridDim.x; };
+  // Each pipeline (group g of CTA c) is one of 2 * gridDim.x slots, s =
+  // g * gridDim.x + c.  Items (heaviest first) are dealt to the slots in
+  // rounds, forward in even rounds and backward in odd ones, so that a slot
+  // that took one of the heaviest items of a round takes one of the lightest
+  // of the next.  A group's k-th call (k = g, g + 2, ...) is round k / 2;
+  // every role of a group walks the same items.
+  const int n_slots = 2 * (int)gridDim.x;
+  const int my_slot = grp * (int)gridDim.x + (int)blockIdx.x;
+  auto global_item = [&](int k) {
+    const int r = k >> 1;
+    return r * n_slots + ((r & 1) ? n_slots - 1 - my_slot : my_slot);
+  };
 
   if (warp < 4 && (warp & 1) == 0) {
     if (lane == 0) {

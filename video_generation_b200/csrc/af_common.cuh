@@ -55,8 +55,7 @@ enum Epi : int {
   EPI_GELU = 3,     // u = gelu(acc + b)                                 (act type)
   EPI_HEAD = 4,     // affine map from interleaved (mu_c, s_c) columns   (fp32 x/z)
   EPI_RAW = 5,      // out32 = acc                                       (fp32 scratch)
-  EPI_DENOISE = 6,  // x = x_noisy + sigma * (acc + b), plain columns    (fp32 x)
-  EPI_RESID_SPLIT = 7  // EPI_RESID as stream-K: tiles cut across CTAs, fixed-order sum of pieces
+  EPI_DENOISE = 6   // x = x_noisy + sigma * (acc + b), plain columns    (fp32 x)
 };
 
 // Everything an epilogue may touch.  Pointers not used by a kind stay null.
@@ -84,13 +83,6 @@ struct EpiArgs {
   float* part;             // [Mmax, 2C/16, 2] per-(row, 16-column group) partial sums
   uint64_t wait_ns;        // tensor-core kernels: limit of a pipeline wait before the CTA aborts
   int l2_keep;             // TMA outputs (residual adds, GELU) stored with an L2 evict_last policy
-  // stream-K residual GEMMs: fp32 partials of cut tiles' pieces 1.. in
-  // ksplit slots [ksplit][kpart_rows][N], and one arrival counter per (tile,
-  // CTA of the pair, epilogue warp), zero at rest
-  int ksplit;
-  float* kpart;
-  int* kcnt;
-  int kpart_rows;
 };
 
 __device__ __forceinline__ int tok_of(int p, int L, int dir) { return dir ? (L - 1 - p) : p; }

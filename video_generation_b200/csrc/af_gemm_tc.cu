@@ -43,8 +43,8 @@ template <int EPI> struct EpiShape {
   // residual add, GELU and QKV leave through TMA: each warp stages 32 rows x
   // 16 columns (two slots, alternating) in the output tensor map's swizzle and
   // issues a bulk reduce-add (h += tile) or a bulk store (u, q, K / V cache)
-  static constexpr bool TMA_OUT = EPI == EPI_RESID || EPI == EPI_RESID_SPLIT || EPI == EPI_GELU || EPI == EPI_QKV;
-  static constexpr uint32_t SLOT = (EPI == EPI_RESID || EPI == EPI_RESID_SPLIT) ? 32 * 16 * 4 : 32 * 16 * 2;
+  static constexpr bool TMA_OUT = EPI == EPI_RESID || EPI == EPI_GELU || EPI == EPI_QKV;
+  static constexpr uint32_t SLOT = EPI == EPI_RESID ? 32 * 16 * 4 : 32 * 16 * 2;
 };
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kMaxDevices = 64;
@@ -121,14 +121,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
       : "memory");
-}
-// Prefetch a tile into L2 (no shared-memory destination, no completion):
-// the weight tiles of the k-blocks one ring ahead of the loads, so that a
-// weight matrix streamed from HBM reaches the ring from L2.
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int c0, int c1) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),
-               "r"(c0), "r"(c1)
-               : "memory");
 }
 // Shared-memory matrix descriptor of a K-major tile written by TMA with
 // 128-byte swizzle: rows of 64 bf16 (128 B), 8-row groups 1024 B apart.
@@ -280,65 +272,6 @@ __device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 
-// Work of one CTA (pair): a sequence of segments, each a tile and a range of
-// its k-blocks.  Plain GEMMs: whole tiles t = unit, unit + nunits, ...
-// Stream-K residual GEMMs: the tiles' k-blocks in tile-major order, cut into
-// nunits equal contiguous ranges, one per unit; a tile cut across units is
-// made of pieces 0 .. npieces-1 in k order, piece 0 at the end of the range of
-// the first unit covering it.
-struct Seg { int tile, kb0, kb1, piece, npieces; };
-__device__ __forceinline__ long long sk_start(int u, int nunits, long long W) { return (long long)u * W / nunits; }
-__device__ __forceinline__ int sk_unit_of(long long pos, int nunits, long long W) {
-  int u = (int)(pos * nunits / W);
-  while (u + 1 < nunits && sk_start(u + 1, nunits, W) <= pos) ++u;
-  while (u > 0 && sk_start(u, nunits, W) > pos) --u;
-  return u;
-}
-struct SegIter {
-  bool sk;
-  int unit, nunits, ntiles, kbn, t;
-  long long W, pos, end;
-  // slots: the partial slots of the workspace; a tile may be cut into at most
-  // slots + 1 pieces
-  __device__ SegIter(bool sk_, int unit_, int nunits_, int ntiles_, int kbn_, int slots)
-      : sk(sk_), unit(unit_), nunits(nunits_), ntiles(ntiles_), kbn(kbn_), t(unit_) {
-    W = (long long)ntiles * kbn;
-    if (sk) {
-      // Ranges of at least 4 k-blocks, so that none is empty (every unit
-      // counted among a tile's pieces holds one) and partials stay few, and
-      // of at least ceil(kbn / slots), so that a tile spans at most slots + 1
-      // ranges whatever the live row count.
-      long long min_len = (kbn + slots - 1) / (slots > 0 ? slots : 1);
-      if (min_len < 4) min_len = 4;
-      long long cap = W / min_len;
-      if (cap < 1) cap = 1;
-      if (nunits > cap) nunits = (int)cap;
-    }
-    pos = (sk && unit < nunits) ? sk_start(unit, nunits, W) : 0;
-    end = (sk && unit < nunits) ? sk_start(unit + 1, nunits, W) : 0;
-  }
-  __device__ bool next(Seg& g) {
-    if (!sk) {
-      if (t >= ntiles) return false;
-      g.tile = t; g.kb0 = 0; g.kb1 = kbn; g.piece = 0; g.npieces = 1;
-      t += nunits;
-      return true;
-    }
-    if (pos >= end) return false;
-    const int tile = (int)(pos / kbn);
-    const long long tile_end = (long long)(tile + 1) * kbn;
-    const long long seg_end = tile_end < end ? tile_end : end;
-    g.tile = tile;
-    g.kb0 = (int)(pos - (long long)tile * kbn);
-    g.kb1 = g.kb0 + (int)(seg_end - pos);
-    const int u0 = sk_unit_of((long long)tile * kbn, nunits, W);
-    g.piece = unit - u0;
-    g.npieces = sk_unit_of(tile_end - 1, nunits, W) - u0 + 1;
-    pos = seg_end;
-    return true;
-  }
-};
-
 template <int BN, int EPI, int CG>
 __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -412,7 +345,6 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
   const int M = e.ctl->M;
   const int tiles_m = (M + TM - 1) / TM;
   const int ntiles = tiles_m * tiles_n;
-  constexpr bool SK = EPI == EPI_RESID_SPLIT;             // stream-K residual GEMM
 
   if (warp == 0) {
     if (lane == 0) {
@@ -420,18 +352,12 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       long long issued = 0;
-      SegIter it(SK, unit, nunits, ntiles, kbn, e.ksplit);
-      Seg g;
-      while (it.next(g)) {
-        const int mb = g.tile % tiles_m, nb = g.tile / tiles_m;
+      for (int t = unit; t < ntiles; t += nunits) {
+        const int mb = t % tiles_m, nb = t / tiles_m;
         const int arow = mb * TM + (int)rank * BM;
         const int brow = nb * BN + (int)rank * (BN / CG);
-        const int kb0 = g.kb0, kb1 = g.kb1;
-        // the weight tiles one to two rings ahead go to L2 first (the loop
-        // keeps prefetching two rings ahead of its loads)
-        for (int kb = kb0 + S; kb < kb0 + 2 * S && kb < kb1; ++kb) tma_prefetch_2d(&tmB, kb * BK, brow);
         bool ok = true;
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = 0; kb < kbn; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, ab)) { ok = false; break; }
           if (rank == 0) mbar_expect_tx(full0 + 8 * stage, CG * Cfg::STAGE_BYTES);
           if (CG == 2) {
@@ -441,7 +367,6 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
             tma_load_2d(smem_u32(sA + stage * Cfg::A_BYTES), &tmA, full0 + 8 * stage, kb * BK, arow);
             tma_load_2d(smem_u32(sB + stage * Cfg::B_BYTES), &tmB, full0 + 8 * stage, kb * BK, brow);
           }
-          if (kb + 2 * S < kb1) tma_prefetch_2d(&tmB, (kb + 2 * S) * BK, brow);
           ++issued;
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
@@ -477,24 +402,21 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       int i = 0;
-      SegIter it(SK, unit, nunits, ntiles, kbn, e.ksplit);
-      Seg g;
-      for (; it.next(g); ++i) {
+      for (int t = unit; t < ntiles; t += nunits, ++i) {
         const int acc = i & 1;
         const uint32_t use = (uint32_t)(i >> 1);
-        const int kb0 = g.kb0, kb1 = g.kb1;
         if (!mbar_wait(tempty0 + 8 * acc, (use & 1u) ^ 1u, ab)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
         bool ok = true;
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = 0; kb < kbn; ++kb) {
           if (!mbar_wait(full0 + 8 * stage, phase, ab)) { ok = false; break; }
           tc_fence_after();
           const uint64_t da = sw128_desc(smem_u32(sA + stage * Cfg::A_BYTES));
           const uint64_t db = sw128_desc(smem_u32(sB + stage * Cfg::B_BYTES));
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            const uint32_t accum = ((kb - kb0) | k) != 0;
+            const uint32_t accum = (kb | k) != 0;
             if (CG == 2) umma_bf16_pair(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), Cfg::IDESC, accum);
             else umma_bf16(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), Cfg::IDESC, accum);
           }
@@ -538,111 +460,6 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
       const uint64_t keep_pol = e.l2_keep ? policy_evict_last() : 0ull;
       int cc = 0;                                       // chunks sent by this warp
       int i = 0;
-      if constexpr (EPI == EPI_RESID_SPLIT) {
-        // Stream-K: a whole tile leaves as in the residual path; a tile cut
-        // into pieces is finished by piece 0 -- its unit processes it last --
-        // which waits (bounded) until the other pieces have stored their fp32
-        // partials, adds them to its own accumulator in piece order, adds the
-        // bias and sends the sum into h by TMA reduce-add: one add per element
-        // of h, the same sum whatever the timing.
-        SegIter it(true, unit, nunits, ntiles, kbn, e.ksplit);
-        Seg g;
-        const size_t ld = (size_t)tiles_n * BN;                         // N
-        for (; it.next(g); ++i) {
-          const int acc = i & 1;
-          const uint32_t use = (uint32_t)(i >> 1);
-          const int mb = g.tile % tiles_m, nb = g.tile / tiles_m;
-          const int row0 = mb * TM + (int)rank * BM + q * 32;
-          const int n0 = nb * BN + hf * HALF;
-          const uint32_t taddr = tmem + (uint32_t)(acc * BN + hf * HALF) + ((uint32_t)(q * 32) << 16);
-          const int r = row0 + lane;
-          const bool rok = r < e.kpart_rows;
-          int* cnt = e.kcnt + ((size_t)g.tile * CG + rank) * Cfg::EPI_WARPS + ew;
-          if (g.piece > e.ksplit) {                       // more pieces than partial slots: not planned for
-            if (lane == 0) atomicOr(err, ERR_GEMM_WAIT);
-            *abort_flag = 1;
-            break;
-          }
-          if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * acc, use & 1u, ab))) break;
-          tc_fence_after();
-          if (g.piece > 0) {
-            // a later piece: store the partial, release the accumulator, count in
-            float* mine = e.kpart + ((size_t)(g.piece - 1) * e.kpart_rows + r) * ld + n0;
-#pragma unroll
-            for (int k = 0; k < NCH; ++k) {
-              float v[16];
-              tmem_ld16(taddr + k * 16, v);
-              tmem_wait_ld();
-              if (rok) {
-                float4* dst = reinterpret_cast<float4*>(mine + k * 16);
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) dst[jj] = make_float4(v[4 * jj], v[4 * jj + 1], v[4 * jj + 2], v[4 * jj + 3]);
-              }
-            }
-            tc_fence_before();
-            if (CG == 2) mbar_arrive_cluster(tempty_lead + 8 * acc);
-            else mbar_arrive(tempty0 + 8 * acc);
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) atomicAdd(cnt, 1);
-            continue;
-          }
-          if (g.npieces > 1) {
-            // piece 0: the other pieces' partials are complete before reading them
-            bool ok = true;
-            if (lane == 0) {
-              const uint64_t t0 = globaltimer_ns();
-              while (*reinterpret_cast<volatile int*>(cnt) < g.npieces - 1) {
-                if (*abort_flag || globaltimer_ns() - t0 > ab.limit_ns) { *abort_flag = 1; ok = false; break; }
-              }
-              if (ok) atomicExch(cnt, 0);                   // zero again for the next launch
-            }
-            if (!__shfl_sync(0xffffffffu, (int)ok, 0)) break;
-            __threadfence();
-          }
-#pragma unroll
-          for (int k = 0; k < NCH; ++k) {
-            const int col = n0 + k * 16;
-            float v[16];
-            tmem_ld16(taddr + k * 16, v);
-            tmem_wait_ld();
-            if (k + 1 == NCH) {                             // every TMEM read of this tile is done
-              tc_fence_before();
-              if (CG == 2) mbar_arrive_cluster(tempty_lead + 8 * acc);
-              else mbar_arrive(tempty0 + 8 * acc);
-            }
-            if (rok) {
-              for (int pc = 1; pc < g.npieces; ++pc) {
-                const float4* src =
-                    reinterpret_cast<const float4*>(e.kpart + ((size_t)(pc - 1) * e.kpart_rows + r) * ld + col);
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                  const float4 a4 = __ldcg(src + jj);
-                  v[4 * jj] += a4.x; v[4 * jj + 1] += a4.y; v[4 * jj + 2] += a4.z; v[4 * jj + 3] += a4.w;
-                }
-              }
-            }
-            uint8_t* slot = stg0 + (cc & 1) * SLOT;
-            if (lane == 0) bulk_wait_read1();             // the slot's previous tile has been read
-            __syncwarp();
-            uint8_t* rp = slot + lane * 64;
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-              const float4 bb = reinterpret_cast<const float4*>(e.bias + col)[jj];
-              *reinterpret_cast<float4*>(rp + ((jj ^ ((lane >> 1) & 3)) << 4)) =
-                  make_float4(v[4 * jj] + bb.x, v[4 * jj + 1] + bb.y, v[4 * jj + 2] + bb.z, v[4 * jj + 3] + bb.w);
-            }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncwarp();
-            if (lane == 0) {
-              if (e.l2_keep) tma_reduce_add_2d_hint(&tmC, smem_u32(slot), col, row0, keep_pol);
-              else tma_reduce_add_2d(&tmC, smem_u32(slot), col, row0);
-              bulk_commit();
-            }
-            ++cc;
-          }
-        }
-      } else {
       for (int t = unit; t < ntiles; t += nunits, ++i) {
         const int acc = i & 1;
         const uint32_t use = (uint32_t)(i >> 1);
@@ -748,7 +565,6 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
             ++cc;
           }
         }
-      }
       }
       if (lane == 0) bulk_wait_all();                   // the bulk writes are complete before the CTA exits
       __syncwarp();
@@ -969,7 +785,7 @@ void launch_bn_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtenso
     }
   }
   const int tiles = ((m_max + BM * CG - 1) / (BM * CG)) * (N / BN);
-  const int units = (EPI == EPI_RESID_SPLIT || tiles > max_units) ? max_units : tiles;   // stream-K: every unit
+  const int units = tiles > max_units ? max_units : tiles;
   if (CG == 1) {
     launch_k(k_gemm_tc<BN, EPI, 1>, dim3(units), dim3(Cfg::THREADS), Cfg::SMEM, st, tmA, tmB, tmC, tmC2, tmC3, N, K, e, err);
   } else {
@@ -999,9 +815,6 @@ void launch_bn(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, const CU
     case EPI_RESID: launch_bn_epi<BN, EPI_RESID, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st); break;
     case EPI_GELU: launch_bn_epi<BN, EPI_GELU, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st); break;
     case EPI_HEAD: launch_bn_epi<BN, EPI_HEAD, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st); break;
-    case EPI_RESID_SPLIT:
-      launch_bn_epi<BN, EPI_RESID_SPLIT, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st);
-      break;
     default: launch_bn_epi<BN, EPI_DENOISE, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st); break;
   }
 }
@@ -1067,32 +880,6 @@ int gemm_tc_pick(int N, int m_max, int num_sms, int unit, int max_bn) {
     if (!best || cost < best_cost) { best = bn; best_cost = cost; }
   }
   return best ? best * 10 + cg : 0;
-}
-
-// Stream-K for a residual GEMM of tile shape `pick`: 0 when whole tiles
-// already fill the SM pairs evenly (>= 90% of the last wave busy) for passes
-// of m_rows rows, else the partial slots a tile cut into pieces may need:
-// a tile of K/64 k-blocks spans at most ceil(kbn / per-unit range) + 1 unit
-// ranges, all but its piece 0 storing a partial.
-int gemm_tc_ksplit(int pick, int N, int K, int m_rows, int num_sms) {
-  const int bn = pick / 10, cg = pick % 10;
-  if (!bn || m_rows < 1) return 0;
-  const int units = num_sms / cg;
-  const long long tiles = (long long)((m_rows + BM * cg - 1) / (BM * cg)) * (N / bn);
-  const long long waves = (tiles + units - 1) / units;
-  if (tiles * 10 >= waves * units * 9) return 0;
-  const int kbn = K / BK;
-  const long long W = tiles * kbn;
-  long long used = W / 4 > 1 ? W / 4 : 1;                // the kernel's ranges hold >= 4 k-blocks
-  if (used > units) used = units;
-  long long per_unit = W / used;
-  if (per_unit < 1) per_unit = 1;
-  return (int)((kbn + per_unit - 1) / per_unit);
-}
-
-int gemm_tc_tiles(int pick, int N, int m_max) {
-  const int bn = pick / 10, cg = pick % 10;
-  return bn ? ((m_max + BM * cg - 1) / (BM * cg)) * (N / bn) : 0;
 }
 
 void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap* tmC,

@@ -91,11 +91,6 @@ void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, con
                     const CUtensorMap* tmC2, const CUtensorMap* tmC3, int pick, int N, int K, int m_max,
                     const EpiArgs& e, int* err, int num_sms, cudaStream_t st);
 int gemm_tc_pick(int N, int m_max, int num_sms, int unit, int max_bn);
-// Stream-K of a residual GEMM with tile shape `pick` for passes of m_rows
-// rows: 0 when whole tiles fill the SM pairs evenly, else the partial slots
-// a cut tile may need; and the GEMM's tile count.
-int gemm_tc_ksplit(int pick, int N, int K, int m_rows, int num_sms);
-int gemm_tc_tiles(int pick, int N, int m_max);
 
 // Causal attention over the KV cache on tcgen05 (af_attn_tc.cu).  Each pass
 // splits its live key range into at most nsplit_max splits (attn_tc_splits
