@@ -186,31 +186,38 @@ af_status af_inverse_jacobi_stream(const af_model* m, const float* z, int batch,
                                    size_t ws_bytes, void* stream);
 
 /* Bytes of the shallow-side workspace of flow_pipeline_inverse for T shallow
- * blocks (config of `shallow`), `batch` videos, frames of frame_len tokens. */
-size_t flow_pipeline_workspace_bytes(const af_model* shallow, int T, int batch, int frame_len);
+ * blocks (config of `shallow`), `batch` videos, frames of frame_len tokens,
+ * `group` frames per shallow call; 0 on a bad argument. */
+size_t flow_pipeline_workspace_bytes(const af_model* shallow, int T, int batch, int frame_len, int group);
 
 /* Pipelined deep -> shallow decoding ("Key design 3": the deep flow
  * f_D runs without pause while the shallow blocks f_S consume its output
  * frame by frame; end-to-end latency is set by the deep block):
  * x = f_S^{-1}(f_D^{-1}(z)) with f_S applied to each frame on its own.
  * f_D^{-1} (`deep`, direction L->R, blocks of B tokens, tau, max_iter_deep,
- * warm_start) runs on stream_deep, one frame's blocks per graph launch;
- * after each frame an event lets stream_shallow run the T-block stack
- * inverse of that frame (blocks shallow[0..T-1], directions shallow_dirs,
- * one Jacobi block per frame, no warm start, tau, max_iter_shallow) while
- * the deep flow moves on.  z, x: [batch, L, C]; frame_len = the deep model's
- * frame_len (the shallow models must accept frames of that length and C);
- * L % frame_len == 0 and frame_len % B == 0.  iters_deep [batch, L/B],
- * iters_shallow [T, batch, L/frame_len].  ws_deep: af_workspace_bytes(deep,
- * batch, L, B); ws_shallow: flow_pipeline_workspace_bytes(shallow[0], T,
- * batch, frame_len).  The two streams may be the same stream (no overlap).
- * On return all work is enqueued; stream_deep waits for the last frame's
- * shallow work, so synchronising stream_deep covers the whole call.  The
- * result is bit-identical to af_inverse_jacobi followed by
- * flow_stack_inverse of each frame. */
+ * warm_start) runs on stream_deep, one frame's blocks per graph launch.
+ * Frames are handed to the shallow side in groups of `group` consecutive
+ * frames (the last group may be shorter; 1 <= group <= L / frame_len): when
+ * the deep flow has finished a group, an event lets stream_shallow run the
+ * T-block stack inverse of the group's frames of every video as one batch of
+ * batch * group one-frame samples (blocks shallow[0..T-1], directions
+ * shallow_dirs, one Jacobi block per frame, no warm start, tau,
+ * max_iter_shallow) while the deep flow moves on.  group 1 hands over every
+ * frame at once (the shortest tail after the deep flow ends); larger groups
+ * run fewer, larger shallow calls beside it.  z, x: [batch, L, C];
+ * frame_len = the deep model's frame_len (the shallow models must accept
+ * frames of that length and C); L % frame_len == 0 and frame_len % B == 0.
+ * iters_deep [batch, L/B], iters_shallow [T, batch, L/frame_len].  ws_deep:
+ * af_workspace_bytes(deep, batch, L, B); ws_shallow:
+ * flow_pipeline_workspace_bytes(shallow[0], T, batch, frame_len, group).  The
+ * two streams may be the same stream (no overlap).  On return all work is
+ * enqueued; stream_deep waits for the last group's shallow work, so
+ * synchronising stream_deep covers the whole call.  The result is
+ * bit-identical to af_inverse_jacobi followed by flow_stack_inverse of each
+ * group's frames as one batch. */
 af_status flow_pipeline_inverse(const af_model* deep, const af_model* const* shallow, const af_dir* shallow_dirs, int T,
                                 const float* z, int batch, int L, int B, float tau, int max_iter_deep,
-                                int max_iter_shallow, int warm_start, float* x, int32_t* iters_deep,
+                                int max_iter_shallow, int warm_start, int group, float* x, int32_t* iters_deep,
                                 int32_t* iters_shallow, void* ws_deep, size_t ws_deep_bytes, void* ws_shallow,
                                 size_t ws_shallow_bytes, void* stream_deep, void* stream_shallow);
 

@@ -8,9 +8,12 @@ nanosecond, so that waits run out during a normal forward pass; the call must
 return, af_device_error must report a pipeline wait (GEMM or attention, not a
 failed drain), and the next call at the default limit must match the oracle.
 
-The pass has fewer than 256 rows, so its GEMMs run on single SMs: on an SM
-pair the second CTA's loads complete on the leader's barriers, which it cannot
-wait on, so the pair's abort drain is not exercised here.
+One sample (200 rows) runs the GEMMs on single SMs; two samples (400 rows)
+run them on SM pairs, whose second CTA's loads complete on the leader's
+barriers: the second CTA reports how many loads it issued and the leader's
+drain waits for them (completing by hand the bytes of loads it counted but the
+second CTA never issued), so a pair that aborts at different k-blocks in its
+two CTAs still drains every load before it exits.
 """
 import numpy as np
 import pytest
@@ -35,9 +38,10 @@ def flow():
     return F
 
 
-def test_expired_waits_abort_cleanly_and_report(flow):
+@pytest.mark.parametrize("batch", [1, 2], ids=["single_sm", "sm_pair"])
+def test_expired_waits_abort_cleanly_and_report(flow, batch):
     pair = Pair(flow, SHAPE, perturb=True, head_std=1e-2)
-    x = syn.make_latents(1, 200, SHAPE.C, 71)
+    x = syn.make_latents(batch, 200, SHAPE.C, 71)
     xd = to_dev(x)
     assert pair.model.device_error() == 0
     pair.model.set_wait_limit(1e-9)

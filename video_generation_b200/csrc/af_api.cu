@@ -962,17 +962,18 @@ af_status af_prefix_encode(const af_model* m, const float* x, int batch, int L, 
   return graph_run(m, key, (cudaStream_t)stream, build_encode, &c);
 }
 
-size_t flow_pipeline_workspace_bytes(const af_model* shallow, int T, int batch, int frame_len) {
-  if (!shallow || T < 1) return 0;
-  const size_t stack = af_workspace_bytes(shallow, batch, frame_len, frame_len);
+size_t flow_pipeline_workspace_bytes(const af_model* shallow, int T, int batch, int frame_len, int group) {
+  if (!shallow || T < 1 || batch < 1 || group < 1) return 0;
+  const int nb = batch * group;                    // a shallow call's samples: group frames of every video
+  const size_t stack = af_workspace_bytes(shallow, nb, frame_len, frame_len);
   if (!stack) return 0;
-  const size_t frame = align256((size_t)batch * frame_len * shallow->cfg.C * sizeof(float));
-  return stack + 2 * frame + align256((size_t)T * batch * sizeof(int32_t));
+  const size_t frames = align256((size_t)nb * frame_len * shallow->cfg.C * sizeof(float));
+  return stack + 2 * frames + align256((size_t)T * nb * sizeof(int32_t));
 }
 
 af_status flow_pipeline_inverse(const af_model* deep, const af_model* const* shallow, const af_dir* shallow_dirs, int T,
                                 const float* z, int batch, int L, int B, float tau, int max_iter_deep,
-                                int max_iter_shallow, int warm_start, float* x, int32_t* iters_deep,
+                                int max_iter_shallow, int warm_start, int group, float* x, int32_t* iters_deep,
                                 int32_t* iters_shallow, void* ws_deep, size_t ws_deep_bytes, void* ws_shallow,
                                 size_t ws_shallow_bytes, void* stream_deep, void* stream_shallow) {
   cudaStream_t sd = (cudaStream_t)stream_deep, ss = (cudaStream_t)stream_shallow;
@@ -992,8 +993,10 @@ af_status flow_pipeline_inverse(const af_model* deep, const af_model* const* sha
     set_err("need L %% frame_len == 0, frame_len %% B == 0, max_iter >= 1, finite tau >= 0");
     return AF_ERR_ARG;
   }
+  const int nf = L / F;
+  if (group < 1 || group > nf) { set_err("need 1 <= group <= L / frame_len (%d), got %d", nf, group); return AF_ERR_ARG; }
   if (af_status s = check_ws(deep, ws_deep, ws_deep_bytes, batch, L, B)) return s;
-  const size_t need_s = flow_pipeline_workspace_bytes(shallow[0], T, batch, F);
+  const size_t need_s = flow_pipeline_workspace_bytes(shallow[0], T, batch, F, group);
   if (!ws_shallow || (reinterpret_cast<uintptr_t>(ws_shallow) & 255u) || ws_shallow_bytes < need_s) {
     set_err("shallow workspace: need %zu bytes, 256-aligned; got %zu", need_s, ws_shallow_bytes);
     return AF_ERR_WORKSPACE;
@@ -1003,18 +1006,21 @@ af_status flow_pipeline_inverse(const af_model* deep, const af_model* const* sha
     CK(cudaEventCreateWithFlags(&dm->ev_frame, cudaEventDisableTiming));
     CK(cudaEventCreateWithFlags(&dm->ev_done, cudaEventDisableTiming));
   }
-  // the shallow side's workspace: the stack's own, then the staged frame in / out and counts
-  const size_t stack_bytes = af_workspace_bytes(shallow[0], batch, F, F);
-  const size_t frame = align256((size_t)batch * F * C * sizeof(float));
+  // the shallow side's workspace: the stack's own (for batch * group samples),
+  // then the staged frames in / out and the counts
+  const int nbmax = batch * group;
+  const size_t stack_bytes = af_workspace_bytes(shallow[0], nbmax, F, F);
+  const size_t frames = align256((size_t)nbmax * F * C * sizeof(float));
   char* wsS = static_cast<char*>(ws_shallow);
   float* stage_in = (float*)(wsS + stack_bytes);
-  float* stage_out = (float*)(wsS + stack_bytes + frame);
-  int32_t* stage_it = (int32_t*)(wsS + stack_bytes + 2 * frame);
+  float* stage_out = (float*)(wsS + stack_bytes + frames);
+  int32_t* stage_it = (int32_t*)(wsS + stack_bytes + 2 * frames);
   // the deep flow's output u (the shallow stack's input) stays in its workspace
   float* u = carve(deep, ws_deep, batch, L, B).tmp;
-  const int nf = L / F, bpf = F / B;
+  const int bpf = F / B;
   Schedule sc = uniform_schedule(L, B);
-  const size_t row = (size_t)F * C * sizeof(float);
+  const size_t frame_bytes = (size_t)F * C * sizeof(float);
+  const size_t video_pitch = (size_t)L * C * sizeof(float);
   for (int f = 0; f < nf; ++f) {
     // f_D^{-1}: the blocks of frame f (the table once, then only the range)
     sc.b_begin = f * bpf;
@@ -1023,18 +1029,22 @@ af_status flow_pipeline_inverse(const af_model* deep, const af_model* const* sha
     if (af_status s = run_inverse(dblk, ddir, 1, z, batch, L, sc, tau, max_iter_deep, warm_start, u, iters_deep,
                                   ws_deep, sd, f == 0))
       return s;
+    const int f0 = (f / group) * group;           // first frame of f's group
+    const int g = (f0 + group <= nf ? group : nf - f0);
+    if (f != f0 + g - 1) continue;                // the group is not complete yet
     CK(cudaEventRecord(dm->ev_frame, sd));
-    // f_S^{-1} of frame f on the second stream, while f_D goes on with frame f + 1
+    // f_S^{-1} of frames f0 .. f on the second stream, while f_D goes on:
+    // every video's g frames, each frame a sample of its own ([batch * g, F, C])
     CK(cudaStreamWaitEvent(ss, dm->ev_frame, 0));
-    CK(cudaMemcpy2DAsync(stage_in, row, u + (size_t)f * F * C, (size_t)L * C * sizeof(float), row, batch,
-                         cudaMemcpyDeviceToDevice, ss));
-    if (af_status s = flow_stack_inverse(shallow, shallow_dirs, T, stage_in, batch, F, F, tau, max_iter_shallow, 0,
+    const size_t run = (size_t)g * frame_bytes;
+    CK(cudaMemcpy2DAsync(stage_in, run, u + (size_t)f0 * F * C, video_pitch, run, batch, cudaMemcpyDeviceToDevice, ss));
+    if (af_status s = flow_stack_inverse(shallow, shallow_dirs, T, stage_in, batch * g, F, F, tau, max_iter_shallow, 0,
                                          stage_out, stage_it, ws_shallow, stack_bytes, ss))
       return s;
-    CK(cudaMemcpy2DAsync(x + (size_t)f * F * C, (size_t)L * C * sizeof(float), stage_out, row, row, batch,
-                         cudaMemcpyDeviceToDevice, ss));
-    CK(cudaMemcpy2DAsync(iters_shallow + f, (size_t)nf * sizeof(int32_t), stage_it, sizeof(int32_t), sizeof(int32_t),
-                         (size_t)T * batch, cudaMemcpyDeviceToDevice, ss));
+    CK(cudaMemcpy2DAsync(x + (size_t)f0 * F * C, video_pitch, stage_out, run, run, batch, cudaMemcpyDeviceToDevice, ss));
+    // counts [T, batch * g] -> iters_shallow[T, batch, f0 .. f0 + g)
+    CK(cudaMemcpy2DAsync(iters_shallow + f0, (size_t)nf * sizeof(int32_t), stage_it, (size_t)g * sizeof(int32_t),
+                         (size_t)g * sizeof(int32_t), (size_t)T * batch, cudaMemcpyDeviceToDevice, ss));
   }
   CK(cudaEventRecord(dm->ev_done, ss));
   CK(cudaStreamWaitEvent(sd, dm->ev_done, 0));

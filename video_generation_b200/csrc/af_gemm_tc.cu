@@ -63,7 +63,7 @@ template <int BN, int CG, int EPI> struct TcCfg {
   // as many stages as the remaining shared memory holds (at most 8)
   static constexpr int STAGES_FIT = (int)((232448u - 1024u - 512u - EPI_BYTES) / STAGE_BYTES);
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
-  static constexpr uint32_t NBARS = 2 * STAGES + 5;
+  static constexpr uint32_t NBARS = 2 * STAGES + 6;
   static constexpr int THREADS = EpiShape<EPI>::THREADS;
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + NBARS * 8 + 16;
   static_assert(STAGES >= 3 && SMEM <= 232448, "GEMM shared memory");
@@ -96,9 +96,34 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 }
 // The CTA's abort flag and the limit of its pipeline waits (the model's
 // wait limit, 2 s by default; the drains after an abort keep kWaitLimitNs).
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+// try_wait whose acquire covers writes released at cluster scope (by the
+// other CTA of an SM pair)
+__device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// complete-tx of `bytes` on a barrier of this CTA: stands in for a load that
+// was counted on the barrier but never issued
+__device__ __forceinline__ void mbar_complete_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.complete_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+// The CTA's abort flag, the limit of its pipeline waits (the model's wait
+// limit, 2 s by default; the drains after an abort keep kWaitLimitNs) and, on
+// an SM pair, the other CTA's abort flag (shared::cluster address, else 0),
+// raised with this CTA's so that the pair gives up together.
 struct Abort {
   volatile int* flag;
   uint64_t limit_ns;
+  uint32_t peer_flag;
 };
 // Wait for the phase of `bar` with parity `parity`; false once the CTA has
 // aborted or the wait limit has passed (which aborts the CTA).
@@ -112,6 +137,7 @@ __device__ bool mbar_wait(uint32_t bar, uint32_t parity, const Abort& ab) {
     if (*ab.flag) return false;
     if (globaltimer_ns() - t0 > ab.limit_ns) {
       *ab.flag = 1;
+      if (ab.peer_flag) st_cluster_u32(ab.peer_flag, 1u);
       return false;
     }
   }
@@ -286,15 +312,16 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
   uint8_t* sB = smem + S * Cfg::A_BYTES;
   float* sEpi = reinterpret_cast<float*>(sB + S * Cfg::B_BYTES);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + S * Cfg::B_BYTES + Cfg::EPI_BYTES);
-  // bars: full[S], empty[S], tfull[2], tempty[2], drain
+  // bars: full[S], empty[S], tfull[2], tempty[2], drain, peer_done
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
+  __shared__ uint32_t s_peer_issued;      // leader: loads the pair's second CTA issued
   volatile int* abort_flag = &s_abort;
-  const Abort ab{abort_flag, e.wait_ns};
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_trigger();
   const uint32_t rank = CG == 2 ? cluster_rank() : 0u;   // 0 = the pair's leader (issues the MMAs)
+  const Abort ab{abort_flag, e.wait_ns, CG == 2 ? map_to_rank(smem_u32(&s_abort), rank ^ 1u) : 0u};
   const int unit = CG == 2 ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int nunits = CG == 2 ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   const int tiles_n = N / BN;
@@ -302,9 +329,11 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S);
   const uint32_t tfull0 = smem_u32(bars + 2 * S), tempty0 = smem_u32(bars + 2 * S + 2);
   const uint32_t drain = smem_u32(bars + 2 * S + 4);
+  const uint32_t peer_done = smem_u32(bars + 2 * S + 5);
 
   if (threadIdx.x == 0) {
     s_abort = 0;
+    s_peer_issued = 0;
     for (int i = 0; i < S; ++i) {
       mbar_init(full0 + 8 * i, 1);
       mbar_init(empty0 + 8 * i, 1);
@@ -314,6 +343,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
       mbar_init(tempty0 + 8 * i, Cfg::EPI_WARPS * 32 * CG);
     }
     mbar_init(drain, 1);
+    mbar_init(peer_done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
@@ -372,28 +402,41 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
         }
         if (!ok) break;
       }
-      if (CG == 1 || rank == 0) {
-        // drain: the last load of every stage has landed before the CTA exits
-        // (on an SM pair the leader's full barriers count the bytes of both
-        // CTAs' loads of the stages it armed)
-        const long long n = issued < S ? issued : S;
-        for (long long j = 1; j <= n; ++j) {
-          const long long idx = issued - j;
+      if (CG == 2 && rank != 0) {
+        // The second CTA's loads complete on the leader's full barriers: it
+        // tells the leader how many it issued (its own abort, or the leader's,
+        // may have stopped it at a different k-block than the leader), and the
+        // leader's drain covers them before the pair leaves together (cluster
+        // barrier at the end).
+        st_cluster_u32(map_to_rank(smem_u32(&s_peer_issued), 0), (uint32_t)issued);
+        mbar_arrive_cluster(map_to_rank(peer_done, 0));
+      } else {
+        // drain: the last load of every stage has landed before the CTA exits.
+        // On an SM pair a stage's full barrier counts both CTAs' bytes: a
+        // stage only the second CTA loaded gets the leader's arrival with the
+        // second CTA's bytes, and a stage the leader armed for both but the
+        // second CTA never loaded gets those bytes completed by hand.
+        long long hi = issued, peer = issued;
+        bool have_peer = true;
+        if (CG == 2) {
+          const uint64_t limit = ab.limit_ns + kWaitLimitNs;   // the second CTA's own waits end first
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_cluster(peer_done, 0)) {
+            if (globaltimer_ns() - t0 > limit) { atomicOr(err, ERR_DRAIN); have_peer = false; break; }
+          }
+          if (have_peer) peer = (long long)s_peer_issued;
+          if (peer > hi) hi = peer;
+        }
+        for (long long idx = (hi > S ? hi - S : 0); idx < hi && have_peer; ++idx) {
           const int st = (int)(idx % S);
           const uint32_t ph = (uint32_t)((idx / S) & 1);
+          if (CG == 2 && idx >= issued) mbar_expect_tx(full0 + 8 * st, Cfg::STAGE_BYTES);
+          if (CG == 2 && idx < issued && idx >= peer) mbar_complete_tx(full0 + 8 * st, Cfg::STAGE_BYTES);
           const uint64_t t0 = globaltimer_ns();
           while (!mbar_try(full0 + 8 * st, ph)) {
             if (globaltimer_ns() - t0 > kWaitLimitNs) { atomicOr(err, ERR_DRAIN); break; }
           }
         }
-      }
-      if (CG == 2 && rank != 0 && *abort_flag) {
-        // The second CTA's loads complete on the leader's barriers, which this
-        // CTA cannot wait on; after an abort it gives them 2 ms to land (a load
-        // takes microseconds), and the pair leaves together (cluster barrier
-        // at the end) once the leader has drained.
-        const uint64_t t0 = globaltimer_ns();
-        while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);
       }
     }
   } else if (warp == 1) {

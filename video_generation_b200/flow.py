@@ -65,9 +65,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.af_stream_workspace_bytes.argtypes = [vp, i, i]
     lib.af_stream_workspace_bytes.restype = sz
     lib.af_inverse_jacobi_stream.argtypes = [vp, vp, i, i, i, i, f, i, i, vp, vp, vp, sz, vp]
-    lib.flow_pipeline_workspace_bytes.argtypes = [vp, i, i, i]
+    lib.flow_pipeline_workspace_bytes.argtypes = [vp, i, i, i, i]
     lib.flow_pipeline_workspace_bytes.restype = sz
-    lib.flow_pipeline_inverse.argtypes = [vp, P(vp), P(i), i, vp, i, i, i, f, i, i, i, vp, vp, vp, vp, sz, vp, sz,
+    lib.flow_pipeline_inverse.argtypes = [vp, P(vp), P(i), i, vp, i, i, i, f, i, i, i, i, vp, vp, vp, vp, sz, vp, sz,
                                           vp, vp]
     lib.af_last_convergence.argtypes = [vp, P(i), vp]
     lib.af_device_error.argtypes = [vp, P(i)]
@@ -245,8 +245,9 @@ def af_prefix_encode(model: AFModel, x: torch.Tensor, direction: int, B: int, n_
                                   _stream(stream)), "af_prefix_encode")
 
 
-def pipeline_workspace(shallow: List[AFModel], batch: int, frame_len: int, device=None) -> torch.Tensor:
-    n = int(lib().flow_pipeline_workspace_bytes(shallow[0].handle, len(shallow), batch, frame_len))
+def pipeline_workspace(shallow: List[AFModel], batch: int, frame_len: int, group: int = 1,
+                       device=None) -> torch.Tensor:
+    n = int(lib().flow_pipeline_workspace_bytes(shallow[0].handle, len(shallow), batch, frame_len, group))
     if n == 0:
         raise AFError(AF_ERR_ARG, "flow_pipeline_workspace_bytes")
     return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
@@ -254,16 +255,16 @@ def pipeline_workspace(shallow: List[AFModel], batch: int, frame_len: int, devic
 
 def flow_pipeline_inverse(deep: AFModel, shallow: List[AFModel], shallow_dirs: Sequence[int], z: torch.Tensor,
                           B: int, tau: float, max_iter_deep: int, max_iter_shallow: int, warm_start: bool,
-                          ws_deep: torch.Tensor | None = None, ws_shallow: torch.Tensor | None = None,
+                          group: int = 1, ws_deep: torch.Tensor | None = None, ws_shallow: torch.Tensor | None = None,
                           x: torch.Tensor | None = None, iters_deep: torch.Tensor | None = None,
                           iters_shallow: torch.Tensor | None = None, stream=None, stream_shallow=None):
-    """x = f_S^{-1}(f_D^{-1}(z)), the shallow stack of each frame on a second stream as the deep flow
-    finishes it.  Returns (x, iters_deep [batch, L/B], iters_shallow [T, batch, L/frame_len])."""
+    """x = f_S^{-1}(f_D^{-1}(z)), the shallow stack of each group of `group` frames on a second stream as
+    the deep flow finishes it.  Returns (x, iters_deep [batch, L/B], iters_shallow [T, batch, L/frame_len])."""
     batch, L, _ = z.shape
     F = deep.shape.frame_len
     T = len(shallow)
     ws_deep = deep.workspace(batch, L, B, device=z.device) if ws_deep is None else ws_deep
-    ws_shallow = pipeline_workspace(shallow, batch, F, device=z.device) if ws_shallow is None else ws_shallow
+    ws_shallow = pipeline_workspace(shallow, batch, F, group, device=z.device) if ws_shallow is None else ws_shallow
     x = torch.empty_like(z) if x is None else x
     if iters_deep is None:
         iters_deep = torch.zeros((batch, L // B), dtype=torch.int32, device=z.device)
@@ -273,9 +274,10 @@ def flow_pipeline_inverse(deep: AFModel, shallow: List[AFModel], shallow_dirs: S
     ds = (ctypes.c_int * T)(*shallow_dirs)
     s2 = stream_shallow if stream_shallow is not None else (stream if stream is not None else torch.cuda.current_stream())
     _check(lib().flow_pipeline_inverse(deep.handle, hs, ds, T, _ptr(z), batch, L, B, float(tau), int(max_iter_deep),
-                                       int(max_iter_shallow), int(bool(warm_start)), _ptr(x), _ptr(iters_deep),
-                                       _ptr(iters_shallow), _ptr(ws_deep), ws_deep.numel(), _ptr(ws_shallow),
-                                       ws_shallow.numel(), _stream(stream), _stream(s2)), "flow_pipeline_inverse")
+                                       int(max_iter_shallow), int(bool(warm_start)), int(group), _ptr(x),
+                                       _ptr(iters_deep), _ptr(iters_shallow), _ptr(ws_deep), ws_deep.numel(),
+                                       _ptr(ws_shallow), ws_shallow.numel(), _stream(stream), _stream(s2)),
+           "flow_pipeline_inverse")
     return x, iters_deep, iters_shallow
 
 
