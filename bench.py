@@ -45,6 +45,11 @@ from video_generation_b200 import flops as FL  # noqa: E402
 from video_generation_b200 import shard  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (read + write) of one launch of the config-3 Jacobi inverse graph:
+# twice the ncu dram__bytes of one forward graph (the inverse runs the same
+# pass over the same 8190 rows 6 times, the forward 3 times), from the launch
+# list in profiles/launch_list_fs_stack_T3_21frames_forward.md.
+C3_INVERSE_DRAM_BYTES = 2 * 2.365e9
 SMS = 148
 
 
@@ -310,10 +315,11 @@ def measure(w, args, rank, world, dist, dev, with_e2e=True):
 
     if with_e2e:
         # end to end through the public API with host buffers: every step uploads
-        # its z from pinned memory and downloads its x; the copies of step i+1
-        # (upload) and i-1 (download) overlap step i on a copy stream, the buffers
-        # double-buffered
-        cp = torch.cuda.Stream(device=dev)
+        # its z from pinned memory and downloads its x.  The upload of step i+1
+        # (its own copy stream) and the download of step i-1 (another) overlap
+        # step i; device buffers are double-buffered.
+        cp_up = torch.cuda.Stream(device=dev)
+        cp_dn = torch.cuda.Stream(device=dev)
         z_host = torch.from_numpy(z_np).pin_memory()
         n_out = batch * world if sharded else batch
         x_host = torch.empty((n_out, w.L, w.shape.C), dtype=torch.float32).pin_memory()
@@ -327,24 +333,30 @@ def measure(w, args, rank, world, dist, dev, with_e2e=True):
             dist.barrier()
         torch.cuda.synchronize()
         t0.record(st)
-        cp.wait_stream(st)
+        cp_up.wait_stream(st)
+        cp_dn.wait_stream(st)
+        with torch.cuda.stream(cp_up):
+            z_dev[0].copy_(z_host, non_blocking=True)
+            up[0].record(cp_up)
         for i in range(args.steps):
             j = i % 2
-            with torch.cuda.stream(cp):
-                if i >= 2:
-                    cp.wait_event(done[j])               # z_dev[j] read by step i-2's inverse
-                z_dev[j].copy_(z_host, non_blocking=True)
-                up[j].record(cp)
+            if i + 1 < args.steps:
+                with torch.cuda.stream(cp_up):
+                    if i >= 1:
+                        cp_up.wait_event(done[1 - j])    # z_dev[1-j] read by step i-1's inverse
+                    z_dev[1 - j].copy_(z_host, non_blocking=True)
+                    up[1 - j].record(cp_up)
             st.wait_event(up[j])
             if i >= 2:
                 st.wait_event(down[j])                   # x_dev[j] downloaded by step i-2
             out = inv(z_dev[j], x_dev[j])
             done[j].record(st)
-            with torch.cuda.stream(cp):
-                cp.wait_event(done[j])
+            with torch.cuda.stream(cp_dn):
+                cp_dn.wait_event(done[j])
                 x_host.copy_(out, non_blocking=True)
-                down[j].record(cp)
-        st.wait_stream(cp)
+                down[j].record(cp_dn)
+        st.wait_stream(cp_up)
+        st.wait_stream(cp_dn)
         t1.record(st)
         torch.cuda.synchronize()
         te = shard.max_over_ranks(torch.tensor([t0.elapsed_time(t1) / 1e3], dtype=torch.float64, device=dev), dist)
@@ -613,7 +625,12 @@ def main():
         "mean_iters_per_block": float(np.mean([a.mean() for a in r["it_np"]])),
         "max_iters_per_block": int(max(a.max() for a in r["it_np"])),
         "roofline": {"bound": "tensor", "achieved": inv_tf_rank, "peak": peak, "unit": "TFLOP/s",
-                     "frac": inv_tf_rank / peak, "traffic": None,
+                     "frac": inv_tf_rank / peak,
+                     "traffic": C3_INVERSE_DRAM_BYTES if args.config == 3 else None,
+                     "traffic_note": "DRAM bytes per inverse-graph launch, from an ncu capture of the forward "
+                                     "graph scaled by passes (6 / 3); the graph moves them at "
+                                     f"{C3_INVERSE_DRAM_BYTES / (r['t_inv'] / args.steps) / 1e9:.0f} GB/s"
+                                     if args.config == 3 else None,
                      "kernel": "flow_stack_inverse graph, per GPU (tcgen05 GEMMs dominate)",
                      "peak_kind": f"bf16 dense burst, {peak_kind}",
                      "frac_of_sustained": inv_tf_rank / peaks.get("bf16_tflops_sustained", peak)},
