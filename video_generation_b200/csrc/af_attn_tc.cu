@@ -225,12 +225,14 @@ struct AttnArgs {
 
 // Key splits of a pass, decided from the rows the pass really has (ctl->R
 // query rows per sample at positions p0 ..) rather than from the cache's
-// length: a pass whose (query tile, head, sample) items already fill the GPU
-// twice over runs unsplit; otherwise the live key range (keys 0 .. p0 + R - 1)
-// is cut into up to nsplit_max splits of at least kMinSplitTiles 64-key tiles,
-// aiming at about 2 items per SM (one per pipeline of a CTA), which bounds the
-// partials the combine kernel reads.  The attention kernel and the combine kernel
-// evaluate this from the same control block, so they agree.
+// length: a pass whose (query tile, head, sample) items already give every SM
+// one runs unsplit; otherwise the live key range (keys 0 .. p0 + R - 1) is cut
+// into up to nsplit_max splits of at least kMinSplitTiles 64-key tiles, aiming
+// at about one item per SM.  (Two per SM, one per pipeline of a CTA, was
+// measured 4% slower on the deep flow's 390-row passes: the two pipelines of a
+// CTA share its SM, and more splits mean more partials for the combine kernel
+// to read.)  The attention kernel and the combine kernel evaluate this from
+// the same control block, so they agree.
 constexpr int kMinSplitTiles = 8;
 constexpr int kMaxSplits = 32;
 constexpr int kMaxDevices = 64;
@@ -242,8 +244,8 @@ __host__ __device__ __forceinline__ SplitPlan split_plan(int R, int p0, int head
   const int live = km.limit(p0 + R - 1) / bkv + 1;        // key tiles up to the last key any row needs
   const int base = sp.q_tiles * heads * batch;
   int n = 1;
-  if (nsplit_max > 1 && base < 2 * sms) {
-    const int want = (2 * sms + base - 1) / base;
+  if (nsplit_max > 1 && base < sms) {
+    const int want = (sms + base - 1) / base;
     const int by_len = (live + kMinSplitTiles - 1) / kMinSplitTiles;
     n = want < by_len ? want : by_len;
     if (n > nsplit_max) n = nsplit_max;
@@ -802,8 +804,8 @@ int attn_tc_splits(int batch, int heads, int r_max, int Lc, int num_sms) {
   (void)r_max;
   const int bkv = 64;
   const int base_min = heads * batch;                       // a pass with a single query tile
-  if (base_min >= 2 * num_sms) return 1;
-  const int want = (2 * num_sms + base_min - 1) / base_min;
+  if (base_min >= num_sms) return 1;
+  const int want = (num_sms + base_min - 1) / base_min;
   const int key_tiles = (Lc + bkv - 1) / bkv;
   const int by_len = (key_tiles + kMinSplitTiles - 1) / kMinSplitTiles;
   int n = want < by_len ? want : by_len;
