@@ -753,21 +753,45 @@ __global__ void __launch_bounds__(256) k_attn_combine(AttnArgs g) {
   const int nsplit = split_plan(g.ctl->R, g.ctl->p0, g.heads, g.batch, g.nsplit_max, g.sms, AttnCfg<HD>::BKV, g.km).nsplit;
   if (nsplit == 1 || wg >= M * g.heads) return;      // one split: the attention kernel wrote o itself
   const int row = wg / g.heads, hh = wg - row * g.heads;
-  float mx = -INFINITY;
-  for (int i = 0; i < nsplit; ++i) mx = fmaxf(mx, g.mlpart[(((size_t)i * g.m_max + row) * g.heads + hh) * 2]);
+  // lane i holds split i's (max, sum) (nsplit <= kMaxSplits = 32), so the
+  // partials' statistics arrive in one round trip; the outputs of all splits
+  // are then summed in split order with weights 2^(m_i - max).
+  const size_t mstride = (size_t)g.m_max * g.heads * 2;
+  const float* mlb = g.mlpart + ((size_t)row * g.heads + hh) * 2;
+  float mi = -INFINITY, li = 0.f;
+  if (lane < nsplit) {
+    const float2 v = *reinterpret_cast<const float2*>(mlb + lane * mstride);
+    mi = v.x;
+    li = v.y;
+  }
+  float mx = mi;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const float wi = mi == -INFINITY ? 0.f : exp2f(mi - mx);
+  float lsum = wi * li;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
   constexpr int PER = HD / 32;
   float acc[PER];
 #pragma unroll
   for (int k = 0; k < PER; ++k) acc[k] = 0.f;
-  float lsum = 0.f;
-  for (int i = 0; i < nsplit; ++i) {
-    const float* ml = g.mlpart + (((size_t)i * g.m_max + row) * g.heads + hh) * 2;
-    if (ml[0] == -INFINITY) continue;
-    const float w = exp2f(ml[0] - mx);
-    lsum += w * ml[1];
-    const float* op = g.opart + ((size_t)i * g.m_max + row) * g.d + hh * HD;
+  const float* ob = g.opart + (size_t)row * g.d + hh * HD + lane;
+  const size_t ostride = (size_t)g.m_max * g.d;
+  for (int i0 = 0; i0 < nsplit; i0 += 4) {
+    // four splits' loads in flight before their sums
+    float v[4][PER];
 #pragma unroll
-    for (int k = 0; k < PER; ++k) acc[k] = fmaf(w, op[lane + 32 * k], acc[k]);
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int k = 0; k < PER; ++k) v[u][k] = i0 + u < nsplit ? ob[(i0 + u) * ostride + 32 * k] : 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float w = __shfl_sync(0xffffffffu, wi, (i0 + u) & 31);
+      if (i0 + u < nsplit && w != 0.f) {
+#pragma unroll
+        for (int k = 0; k < PER; ++k) acc[k] = fmaf(w, v[u][k], acc[k]);
+      }
+    }
   }
   const float inv = 1.f / lsum;
 #pragma unroll
