@@ -113,6 +113,10 @@ struct Bufs {
   float* opart;   // split-attention partials (bf16 path)
   float* mlpart;
   int nsplit;
+  float* kpart;   // split-K partials of the residual GEMMs [ksplit][kpart_rows][d] (bf16 path, few tiles)
+  int* ks_out;    // the splits the last residual GEMM used
+  int ksplit;     // 1: the residual GEMMs reduce-add into h directly
+  int kpart_rows;
   size_t total;
 };
 
@@ -149,6 +153,22 @@ Bufs carve(const af_model* m, void* ws, int batch, int L, int B) {
   if (b.nsplit > 1) {
     b.opart = (float*)take(sizeof(float) * (size_t)b.nsplit * mmax * c.d);
     b.mlpart = (float*)take(sizeof(float) * (size_t)b.nsplit * mmax * c.heads * 2);
+  }
+  b.ksplit = 1;
+  if (m->bf) {
+    // The residual GEMMs (N = d) split K when the tiles of the fewest rows a
+    // pass of this workspace has (half its rows, on a Jacobi workspace whose
+    // passes carry one block except on a commit) leave half the SM pairs idle.
+    const int pick = gemm_tc_pick(c.d, (int)mmax, m->num_sms, 0, 256);
+    const int fewest = B < L ? (int)(mmax / 2) : (int)mmax;
+    const int tiles = gemm_tc_tiles(pick, c.d, fewest);
+    const int units = pick ? m->num_sms / (pick % 10) : 0;
+    if (tiles > 0 && 2 * tiles <= units) {
+      b.ksplit = units / tiles < 4 ? units / tiles : 4;
+      b.kpart_rows = (int)((mmax + 255) / 256 * 256);
+      b.kpart = (float*)take(sizeof(float) * (size_t)b.ksplit * b.kpart_rows * c.d);
+      b.ks_out = (int*)take(sizeof(int));
+    }
   }
   b.total = off;
   return b;
@@ -250,11 +270,26 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
               make_tmap_bf16(&tA_u, u, m_max, fd, 128) && make_tmap_out(&tC_h, b.h, true, m_max, d) &&
               make_tmap_out(&tC_u, u, false, m_max, fd) && make_tmap_out(&tC_q, q, false, m_max, d);
     if (!ok) { set_err("cuTensorMapEncodeTiled failed for an activation"); return AF_ERR_CUDA; }
+    CUtensorMap tC_p;
+    if (b.ksplit > 1 && !make_tmap_out(&tC_p, b.kpart, true, b.ksplit * b.kpart_rows, d)) {
+      set_err("cuTensorMapEncodeTiled failed for the split-K partials");
+      return AF_ERR_CUDA;
+    }
     auto gemm = [&](int epi, const CUtensorMap& tA, const void* W, int N, int K, const EpiArgs& ea) -> bool {
       // a QKV tile must fall inside one of q, k, v; the position-add epilogue
       // keeps two row sets in flight and stays at <= 192 columns
       const int pick = gemm_tc_pick(N, m_max, ns, epi == EPI_QKV ? d : 0, epi == EPI_INPROJ ? 192 : 256);
       if (!pick || !make_tmap_bf16(&tB, W, N, K, (pick / 10) / (pick % 10))) return false;
+      if (epi == EPI_RESID && b.ksplit > 1) {
+        // split K: the partials by TMA store, then one fixed-order sum into h
+        EpiArgs ep = ea;
+        ep.ksplit = b.ksplit;
+        ep.kpart_rows = b.kpart_rows;
+        ep.ks_out = b.ks_out;
+        launch_gemm_tc(EPI_PART, tA, tB, &tC_p, &tC_h, nullptr, pick, N, K, m_max, ep, m->d_err, ns, st);
+        launch_split_sum(b.ctl, b.kpart, b.kpart_rows, N, b.ks_out, ea.bias, b.h, m_max, st);
+        return true;
+      }
       const CUtensorMap* tC = epi == EPI_RESID ? &tC_h : (epi == EPI_GELU ? &tC_u : (epi == EPI_QKV ? &tC_q : nullptr));
       launch_gemm_tc(epi, tA, tB, tC, epi == EPI_QKV ? &tC_k : nullptr, epi == EPI_QKV ? &tC_v : nullptr, pick, N, K,
                      m_max, ea, m->d_err, ns, st);

@@ -55,7 +55,8 @@ enum Epi : int {
   EPI_GELU = 3,     // u = gelu(acc + b)                                 (act type)
   EPI_HEAD = 4,     // affine map from interleaved (mu_c, s_c) columns   (fp32 x/z)
   EPI_RAW = 5,      // out32 = acc                                       (fp32 scratch)
-  EPI_DENOISE = 6   // x = x_noisy + sigma * (acc + b), plain columns    (fp32 x)
+  EPI_DENOISE = 6,  // x = x_noisy + sigma * (acc + b), plain columns    (fp32 x)
+  EPI_PART = 7      // kpart[split] = acc over the split's k-blocks      (fp32 scratch)
 };
 
 // Everything an epilogue may touch.  Pointers not used by a kind stay null.
@@ -83,6 +84,13 @@ struct EpiArgs {
   float* part;             // [Mmax, 2C/16, 2] per-(row, 16-column group) partial sums
   uint64_t wait_ns;        // tensor-core kernels: limit of a pipeline wait before the CTA aborts
   int l2_keep;             // TMA outputs (residual adds, GELU) stored with an L2 evict_last policy
+  // EPI_PART (split-K of a residual GEMM): at most ksplit splits; split s of a
+  // tile stores its partial at rows s * kpart_rows + row of the partial map;
+  // the splits used are written to *ks_out for the kernel that sums them (0
+  // when one split: the epilogue then adds acc + b into h as EPI_RESID does)
+  int ksplit;
+  int kpart_rows;
+  int* ks_out;
 };
 
 __device__ __forceinline__ int tok_of(int p, int L, int dir) { return dir ? (L - 1 - p) : p; }

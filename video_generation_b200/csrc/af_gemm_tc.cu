@@ -49,8 +49,9 @@ template <int EPI> struct EpiShape {
   // the output tensor map's swizzle and issues a bulk reduce-add (h += tile) or
   // a bulk store (u, q, K / V cache); one slot rather than two leaves room for
   // one more operand stage (a measured 1.4% on the 768-wide layers)
-  static constexpr bool TMA_OUT = EPI == EPI_RESID || EPI == EPI_GELU || EPI == EPI_QKV;
-  static constexpr uint32_t SLOT = EPI == EPI_RESID ? 32 * 16 * 4 : 32 * 16 * 2;
+  static constexpr bool TMA_OUT = EPI == EPI_RESID || EPI == EPI_GELU || EPI == EPI_QKV || EPI == EPI_PART;
+  static constexpr bool F32_OUT = EPI == EPI_RESID || EPI == EPI_PART;
+  static constexpr uint32_t SLOT = F32_OUT ? 32 * 16 * 4 : 32 * 16 * 2;
 };
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kMaxDevices = 64;
@@ -384,6 +385,21 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
   const int M = e.ctl->M;
   const int tiles_m = (M + TM - 1) / TM;
   const int ntiles = tiles_m * tiles_n;
+  // split-K (EPI_PART): as many splits as idle units allow, at most ksplit,
+  // each an even number of k-blocks (whole stages) and at least 8 of them;
+  // unit work w = split * ntiles + tile over k-blocks [split * kbs, + kbs)
+  int ks = 1;
+  if (EPI == EPI_PART) {
+    ks = ntiles > 0 ? nunits / ntiles : 1;
+    if (ks > e.ksplit) ks = e.ksplit;
+    while (ks > 1 && (kbn % (KS * ks) != 0 || kbn / ks < 8)) --ks;
+    if (ks < 1) ks = 1;
+    // one split: the epilogue adds into h itself (ks_out 0: nothing to sum)
+    if (blockIdx.x == 0 && threadIdx.x == 0) *e.ks_out = ks > 1 ? ks : 0;
+  }
+  const bool part_store = EPI == EPI_PART && ks > 1;      // warp-uniform
+  const int kbs = kbn / ks;
+  const int nwork = ntiles * ks;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -391,13 +407,14 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       long long issued = 0;
-      for (int t = unit; t < ntiles; t += nunits) {
+      for (int w = unit; w < nwork; w += nunits) {
+        const int t = w % ntiles, kb0 = (w / ntiles) * kbs;
         const int mb = t % tiles_m, nb = t / tiles_m;
         const int arow = mb * TM + (int)rank * BM;
         const int brow = nb * BN + (int)rank * (BN / CG);
         bool ok = true;
-        for (int kb = 0; kb < kbn; kb += KS) {
-          const int nk = kbn - kb < KS ? kbn - kb : KS;
+        for (int kb = kb0; kb < kb0 + kbs; kb += KS) {
+          const int nk = kb0 + kbs - kb < KS ? kb0 + kbs - kb : KS;
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, ab)) { ok = false; break; }
           if (rank == 0) mbar_expect_tx(full0 + 8 * stage, CG * nk * Cfg::STAGE_BYTES);
           for (int j = 0; j < nk; ++j) {
@@ -429,9 +446,9 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
         // stage only the second CTA loaded gets the leader's arrival with the
         // second CTA's bytes, and a stage the leader armed for both but the
         // second CTA never loaded gets those bytes completed by hand.  Both
-        // CTAs walk the same tiles, ceil(kbn / KS) stages each, so stage idx
-        // is stage idx % spt of its tile and holds that stage's k-blocks.
-        const int spt = (kbn + KS - 1) / KS;
+        // CTAs walk the same units, ceil(kbs / KS) stages each, so stage idx
+        // is stage idx % spt of its unit and holds that stage's k-blocks.
+        const int spt = (kbs + KS - 1) / KS;
         long long hi = issued, peer = issued;
         bool have_peer = true;
         if (CG == 2) {
@@ -447,7 +464,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
           const int st = (int)(idx % S);
           const uint32_t ph = (uint32_t)((idx / S) & 1);
           const int pos = (int)(idx % spt);
-          const uint32_t peer_bytes = (uint32_t)(kbn - pos * KS < KS ? kbn - pos * KS : KS) * Cfg::STAGE_BYTES;
+          const uint32_t peer_bytes = (uint32_t)(kbs - pos * KS < KS ? kbs - pos * KS : KS) * Cfg::STAGE_BYTES;
           if (CG == 2 && idx >= issued) mbar_expect_tx(full0 + 8 * st, peer_bytes);
           if (CG == 2 && idx < issued && idx >= peer) mbar_complete_tx(full0 + 8 * st, peer_bytes);
           const uint64_t t0 = globaltimer_ns();
@@ -463,15 +480,16 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       int i = 0;
-      for (int t = unit; t < ntiles; t += nunits, ++i) {
+      for (int w = unit; w < nwork; w += nunits, ++i) {
+        const int kb0 = (w / ntiles) * kbs;
         const int acc = i & 1;
         const uint32_t use = (uint32_t)(i >> 1);
         if (!mbar_wait(tempty0 + 8 * acc, (use & 1u) ^ 1u, ab)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
         bool ok = true;
-        for (int kb = 0; kb < kbn; kb += KS) {
-          const int nk = kbn - kb < KS ? kbn - kb : KS;
+        for (int kb = kb0; kb < kb0 + kbs; kb += KS) {
+          const int nk = kb0 + kbs - kb < KS ? kb0 + kbs - kb : KS;
           if (!mbar_wait(full0 + 8 * stage, phase, ab)) { ok = false; break; }
           tc_fence_after();
           for (int j = 0; j < nk; ++j) {
@@ -480,7 +498,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
             const uint64_t db = sw128_desc(smem_u32(sB + sl * Cfg::B_BYTES));
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k) {
-              const uint32_t accum = ((kb + j) | k) != 0;
+              const uint32_t accum = ((kb - kb0 + j) | k) != 0;
               if (CG == 2) umma_bf16_pair(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), Cfg::IDESC, accum);
               else umma_bf16(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), Cfg::IDESC, accum);
             }
@@ -524,11 +542,14 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
       const int R = e.ctl->R, p0 = e.ctl->p0;
       const uint64_t keep_pol = e.l2_keep ? policy_evict_last() : 0ull;
       int i = 0;
-      for (int t = unit; t < ntiles; t += nunits, ++i) {
+      for (int w = unit; w < nwork; w += nunits, ++i) {
+        const int t = w % ntiles;
         const int acc = i & 1;
         const uint32_t use = (uint32_t)(i >> 1);
         const int mb = t % tiles_m, nb = t / tiles_m;
         const int row0 = mb * TM + (int)rank * BM + q * 32;
+        // EPI_PART: the split's partial rows
+        const int orow0 = EPI == EPI_PART ? (w / ntiles) * e.kpart_rows + row0 : row0;
         const int n0 = nb * BN + hf * HALF;
         const uint32_t taddr = tmem + (uint32_t)(acc * BN + hf * HALF) + ((uint32_t)(q * 32) << 16);
         // QKV: the tile lies in one of q, K, V (BN divides d); where its rows go
@@ -544,9 +565,11 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
         }
         // the bias of the first chunk is loaded before waiting for the accumulator,
         // each later chunk's while the previous one is processed
+        // (split-K partials take no bias: the kernel that sums them adds it)
         float4 bnext[4];
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) bnext[jj] = reinterpret_cast<const float4*>(e.bias + n0)[jj];
+        for (int jj = 0; jj < 4; ++jj)
+          bnext[jj] = part_store ? make_float4(0.f, 0.f, 0.f, 0.f) : reinterpret_cast<const float4*>(e.bias + n0)[jj];
         // the wait's outcome is made warp-uniform before the .aligned TMEM loads
         if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * acc, use & 1u, ab))) break;
         tc_fence_after();
@@ -559,7 +582,9 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
           for (int jj = 0; jj < 4; ++jj) b4[jj] = bnext[jj];
           if (k + 1 < NCH) {
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) bnext[jj] = reinterpret_cast<const float4*>(e.bias + n0 + (k + 1) * 16)[jj];
+            for (int jj = 0; jj < 4; ++jj)
+              bnext[jj] = part_store ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                     : reinterpret_cast<const float4*>(e.bias + n0 + (k + 1) * 16)[jj];
           }
           tmem_wait_ld();
           if (k + 1 < NCH) {
@@ -575,7 +600,7 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
           uint8_t* slot = stg;
           if (lane == 0) bulk_wait_read0();             // the slot's previous tile has been read
           __syncwarp();
-          if (EPI == EPI_RESID) {
+          if (EpiShape<EPI>::F32_OUT) {
             // fp32 rows of 64 B, 64-byte swizzle: 16-byte unit j of row r at j ^ ((r >> 1) & 3)
             uint8_t* rp = slot + lane * 64;
 #pragma unroll
@@ -619,7 +644,11 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) {
-              if (e.l2_keep && EPI == EPI_RESID) tma_reduce_add_2d_hint(&tmC, smem_u32(slot), col, row0, keep_pol);
+              if (part_store && e.l2_keep) tma_store_2d_hint(&tmC, smem_u32(slot), col, orow0, keep_pol);
+              else if (part_store) tma_store_2d(&tmC, smem_u32(slot), col, orow0);
+              else if (EPI == EPI_PART && e.l2_keep) tma_reduce_add_2d_hint(&tmC2, smem_u32(slot), col, row0, keep_pol);
+              else if (EPI == EPI_PART) tma_reduce_add_2d(&tmC2, smem_u32(slot), col, row0);
+              else if (e.l2_keep && EPI == EPI_RESID) tma_reduce_add_2d_hint(&tmC, smem_u32(slot), col, row0, keep_pol);
               else if (EPI == EPI_RESID) tma_reduce_add_2d(&tmC, smem_u32(slot), col, row0);
               else if (e.l2_keep && EPI == EPI_GELU) tma_store_2d_hint(&tmC, smem_u32(slot), col, row0, keep_pol);
               else if (EPI == EPI_GELU || which == 0) tma_store_2d(&tmC, smem_u32(slot), col - which * e.d, row0);
@@ -847,7 +876,7 @@ void launch_bn_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtenso
         max_units = clusters;
     }
   }
-  const int tiles = ((m_max + BM * CG - 1) / (BM * CG)) * (N / BN);
+  const int tiles = ((m_max + BM * CG - 1) / (BM * CG)) * (N / BN) * (EPI == EPI_PART ? e.ksplit : 1);
   const int units = tiles > max_units ? max_units : tiles;
   if (CG == 1) {
     launch_k(k_gemm_tc<BN, EPI, 1>, dim3(units), dim3(Cfg::THREADS), Cfg::SMEM, st, tmA, tmB, tmC, tmC2, tmC3, N, K, e, err);
@@ -878,6 +907,7 @@ void launch_bn(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, const CU
     case EPI_RESID: launch_bn_epi<BN, EPI_RESID, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st); break;
     case EPI_GELU: launch_bn_epi<BN, EPI_GELU, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st); break;
     case EPI_HEAD: launch_bn_epi<BN, EPI_HEAD, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st); break;
+    case EPI_PART: launch_bn_epi<BN, EPI_PART, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st); break;
     default: launch_bn_epi<BN, EPI_DENOISE, CG>(tmA, tmB, tmC, tmC2, tmC3, N, K, m_max, e, err, num_sms, st); break;
   }
 }
@@ -943,6 +973,11 @@ int gemm_tc_pick(int N, int m_max, int num_sms, int unit, int max_bn) {
     if (!best || cost < best_cost) { best = bn; best_cost = cost; }
   }
   return best ? best * 10 + cg : 0;
+}
+
+int gemm_tc_tiles(int pick, int N, int m_rows) {
+  const int bn = pick / 10, cg = pick % 10;
+  return bn ? ((m_rows + BM * cg - 1) / (BM * cg)) * (N / bn) : 0;
 }
 
 void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap* tmC,

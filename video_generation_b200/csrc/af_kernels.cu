@@ -314,6 +314,31 @@ __global__ void __launch_bounds__(256) k_layernorm_reg(const Ctl* ctl, const flo
   }
 }
 
+// Split-K sum of a residual GEMM: h += bias + part[0] + part[1] + ... in split
+// order (deterministic), float4 per thread, grid-stride over the live rows.
+__global__ void __launch_bounds__(256) k_split_sum(const Ctl* ctl, const float* __restrict__ part, int rows, int N,
+                                                   const int* __restrict__ ks_ptr, const float* __restrict__ bias,
+                                                   float* h) {
+  pdl_trigger();
+  pdl_wait();
+  const int M = ctl->M, ks = *ks_ptr, n4 = N / 4;
+  if (ks == 0) return;                                  // the GEMM added into h itself
+  const long long total = (long long)M * n4;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(i / n4), c = (int)(i - (long long)r * n4);
+    float4 v = reinterpret_cast<const float4*>(bias)[c];
+    for (int sp = 0; sp < ks; ++sp) {
+      const float4 p = __ldcg(reinterpret_cast<const float4*>(part + ((size_t)sp * rows + r) * N) + c);
+      v.x += p.x; v.y += p.y; v.z += p.z; v.w += p.w;
+    }
+    float4* hp = reinterpret_cast<float4*>(h + (size_t)r * N) + c;
+    float4 o = *hp;
+    o.x += v.x; o.y += v.y; o.z += v.z; o.w += v.w;
+    *hp = o;
+  }
+}
+
 template <typename T>
 __global__ void k_layernorm_gen(const Ctl* ctl, const float* __restrict__ h, const float* __restrict__ g,
                                 const float* __restrict__ b, T* out, int d) {
@@ -521,6 +546,14 @@ void launch_layernorm(const Ctl* ctl, const float* h, const float* g, const floa
 }
 template void launch_layernorm<float>(const Ctl*, const float*, const float*, const float*, float*, int, int, cudaStream_t);
 template void launch_layernorm<bf16>(const Ctl*, const float*, const float*, const float*, bf16*, int, int, cudaStream_t);
+
+void launch_split_sum(const Ctl* ctl, const float* part, int rows, int N, const int* ks, const float* bias, float* h,
+                      int m_max, cudaStream_t st) {
+  const long long work = (long long)m_max * (N / 4);
+  long long blocks = (work + 255) / 256;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  launch_k(k_split_sum, dim3((unsigned)blocks), dim3(256), 0, st, ctl, part, rows, N, ks, bias, h);
+}
 
 void launch_logdet_finalize(const float* part, int batch, int L, int G, float* logdet, int accumulate,
                             cudaStream_t st) {

@@ -85,12 +85,21 @@ bool make_tmap_out(CUtensorMap* map, const void* base, bool f32, int rows, int c
 // C[M, N] = A[M, K] W[N, K]^T with epilogue `epi`, K % 64 == 0.  `pick` =
 // BN * 10 + CG from gemm_tc_pick (N % BN == 0); tmA boxes are 128 rows, tmB
 // boxes BN / CG rows; tmC (make_tmap_out) is the output of EPI_RESID (h),
-// EPI_GELU (u) and EPI_QKV (q), tmC2 / tmC3 the K / V cache of EPI_QKV
-// ([batch * Lc, d]); unused ones may be null.
+// EPI_PART (the split-K partials, ksplit * kpart_rows rows), EPI_GELU (u) and
+// EPI_QKV (q), tmC2 / tmC3 the K / V cache of EPI_QKV ([batch * Lc, d]); tmC2
+// is h for EPI_PART (added into directly when the pass's tiles leave no room
+// for a second split); unused ones may be null.
 void launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap* tmC,
                     const CUtensorMap* tmC2, const CUtensorMap* tmC3, int pick, int N, int K, int m_max,
                     const EpiArgs& e, int* err, int num_sms, cudaStream_t st);
 int gemm_tc_pick(int N, int m_max, int num_sms, int unit, int max_bn);
+// tiles of a GEMM with tile shape `pick` (gemm_tc_pick) over m_rows rows
+int gemm_tc_tiles(int pick, int N, int m_rows);
+// h[r, :] += bias + sum over s < *ks of part[s * rows + r, :] for r < ctl->M
+// (the split-K partials of a residual GEMM, summed in split order); nothing
+// when *ks is 0 (the GEMM ran unsplit and added into h itself)
+void launch_split_sum(const Ctl* ctl, const float* part, int rows, int N, const int* ks, const float* bias, float* h,
+                      int m_max, cudaStream_t st);
 
 // Causal attention over the KV cache on tcgen05 (af_attn_tc.cu).  Each pass
 // splits its live key range into at most nsplit_max splits (attn_tc_splits
