@@ -276,9 +276,10 @@ af_status enqueue_pass(const af_model* m, const Bufs& b, int batch, int L, int d
       return AF_ERR_CUDA;
     }
     auto gemm = [&](int epi, const CUtensorMap& tA, const void* W, int N, int K, const EpiArgs& ea) -> bool {
-      // a QKV tile must fall inside one of q, k, v; the position-add epilogue
-      // keeps two row sets in flight and stays at <= 192 columns
-      const int pick = gemm_tc_pick(N, m_max, ns, epi == EPI_QKV ? d : 0, epi == EPI_INPROJ ? 192 : 256);
+      // the position-add epilogue keeps two row sets in flight and stays at
+      // <= 192 columns (a QKV tile may span q, K and V: its epilogue places
+      // each 16-column chunk)
+      const int pick = gemm_tc_pick(N, m_max, ns, 0, epi == EPI_INPROJ ? 192 : 256);
       if (!pick || !make_tmap_bf16(&tB, W, N, K, (pick / 10) / (pick % 10))) return false;
       if (epi == EPI_RESID && b.ksplit > 1) {
         // split K: the partials by TMA store, then one fixed-order sum into h

@@ -552,16 +552,14 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
         const int orow0 = EPI == EPI_PART ? (w / ntiles) * e.kpart_rows + row0 : row0;
         const int n0 = nb * BN + hf * HALF;
         const uint32_t taddr = tmem + (uint32_t)(acc * BN + hf * HALF) + ((uint32_t)(q * 32) << 16);
-        // QKV: the tile lies in one of q, K, V (BN divides d); where its rows go
-        int which = 0, ycache = 0;
-        bool tma_ok = true;                             // warp-uniform
+        // QKV: a 16-column chunk lies in one of q, K, V (16 divides d); the K
+        // and V rows of this warp go to the cache at (sample, position)
+        int ycache = 0;
+        bool cache_ok = true;                           // warp-uniform
         if (EPI == EPI_QKV) {
-          which = (nb * BN) / e.d;
-          if (which > 0) {
-            const int s0 = row0 / R;
-            tma_ok = row0 + 31 < M && (row0 + 31) / R == s0;
-            ycache = s0 * e.Lc + p0 + (row0 - s0 * R);
-          }
+          const int s0 = row0 / R;
+          cache_ok = row0 + 31 < M && (row0 + 31) / R == s0;
+          ycache = s0 * e.Lc + p0 + (row0 - s0 * R);
         }
         // the bias of the first chunk is loaded before waiting for the accumulator,
         // each later chunk's while the previous one is processed
@@ -597,6 +595,8 @@ __global__ void __launch_bounds__(EpiShape<EPI>::THREADS, 1)
           }
           const float* v = vb[k & 1];
           const int col = n0 + k * 16;
+          const int which = EPI == EPI_QKV ? col / e.d : 0;  // 0 q, 1 K, 2 V
+          const bool tma_ok = which == 0 || cache_ok;       // warp-uniform
           uint8_t* slot = stg;
           if (lane == 0) bulk_wait_read0();             // the slot's previous tile has been read
           __syncwarp();
