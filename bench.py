@@ -49,7 +49,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # twice the ncu dram__bytes of one forward graph (the inverse runs the same
 # pass over the same 8190 rows 6 times, the forward 3 times), from the launch
 # list in profiles/launch_list_fs_stack_T3_21frames_forward.md.
-C3_INVERSE_DRAM_BYTES = 2 * 2.382e9
+C3_INVERSE_DRAM_BYTES = 2 * 2.356e9
 SMS = 148
 
 
