@@ -327,13 +327,20 @@ __global__ void __launch_bounds__(256) k_split_sum(const Ctl* ctl, const float* 
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
     const int r = (int)(i / n4), c = (int)(i - (long long)r * n4);
-    float4 v = reinterpret_cast<const float4*>(bias)[c];
-    for (int sp = 0; sp < ks; ++sp) {
-      const float4 p = __ldcg(reinterpret_cast<const float4*>(part + ((size_t)sp * rows + r) * N) + c);
-      v.x += p.x; v.y += p.y; v.z += p.z; v.w += p.w;
-    }
+    // every load issued before the first add (at most 4 splits, the host's
+    // cap; the absent ones add +0)
     float4* hp = reinterpret_cast<float4*>(h + (size_t)r * N) + c;
+    float4 p[4];
+#pragma unroll
+    for (int sp = 0; sp < 4; ++sp)
+      p[sp] = sp < ks ? __ldcg(reinterpret_cast<const float4*>(part + ((size_t)sp * rows + r) * N) + c)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 v = reinterpret_cast<const float4*>(bias)[c];
     float4 o = *hp;
+#pragma unroll
+    for (int sp = 0; sp < 4; ++sp) {
+      v.x += p[sp].x; v.y += p[sp].y; v.z += p[sp].z; v.w += p[sp].w;
+    }
     o.x += v.x; o.y += v.y; o.z += v.z; o.w += v.w;
     *hp = o;
   }
