@@ -5,7 +5,10 @@
 // (bias + position add, QKV scatter into the KV cache, residual add, GELU,
 // or the affine (mu, s) head).  These are the dense contractions of the AF
 // block's causal Transformer: input projection, QKV, attention output
-// projection, the two MLP matrices and the (mu, log-sigma) head.
+// projection, the two MLP matrices and the (mu, log-sigma) head.  A residual
+// GEMM whose tiles would leave SM pairs idle runs split-K (EPI_PART): each
+// unit is a (tile, half of K) pair that stores its fp32 partial by TMA, and
+// a separate kernel sums the partials into h in split order.
 //
 // Design (persistent CTAs, one per SM, 384 or 640 threads):
 //   warp 0      TMA producer: per stage two k-blocks (the last stage of a
